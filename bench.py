@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""CSA2 decode-step benchmark: prints ONE JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload hier1m|full128k|verify|tiny]
+                    [--impl ours|reference]
+
+A step is one whole decode step of the workload: pack the step's new tokens into the FP4
+cache, the Full layer's indexer scan (hierarchical: best 2048 blocks of 8, then its own
+Top-512 inside them), every Reindex layer's rescoring, and the sparse attention of every
+layer (Reuse layers with the inherited Top-K).  Inputs are seeded synthetic tensors
+resident in HBM; the cache (1.5 GB for hier1m) is larger than L2 and L2 is also flushed
+between timed steps.  The step is captured once in a CUDA graph and replayed.
+
+N > 1 (torchrun): every rank runs the same workload on its own GPU (replicas, weak
+scaling, no data-path collective); time is the max over ranks.  `--impl reference` times
+the CPU oracle on a bounded sample of the same workload (rank 0 only).
+"""
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np
+import torch
+
+METRIC = "CSA2 decode step µs/token and HBM GB/s at 128K/1M ctx; FP4 KV pack GB/s"
+UNIT = "µs/token"
+
+WORKLOAD_TEXT = {
+    "hier1m": "hierarchical decoder at 1M context: B=4 x 1,048,576 FP4 entries, Full layer keeps 2048 "
+              "blocks of 8, then 10 Reindex + 9 Reuse layers, H=64 x 512, HI=8 x 128, Top-512, W=128",
+    "full128k": "Full-mode decode at 128K: B=32, entries U[64K,128K], flat scan + Top-512, Full + Reuse "
+                "layer, H=64 x 512, HI=8 x 128, W=128",
+    "verify": "multi-query verify: B=8 x 128K entries (2:1 of 256K tokens), Q=64 drafts, Full + Reuse layer",
+    "tiny": "tiny decode: 1 sequence, 4096 entries, H=16, HI=4, Top-512, W=128",
+}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--workload", default="hier1m", choices=list(WORKLOAD_TEXT))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--cpu-seqs", type=int, default=1, help="sequences in the oracle's timed sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ---- distributed plumbing ------------------------------------------------------------------
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---- clocks during the timed region ---------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        p = torch.cuda.get_device_properties(device)
+        self.bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.bus, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---- roofline bookkeeping -------------------------------------------------------------------
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm": p["hbm_gbs"], "bf16": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "sm_mhz": p.get("sm_max_mhz", 1965.0), "src": "measured"}
+    return {"hbm": 6650.0, "bf16": 1400.0, "sm_mhz": 1965.0, "src": "fallback"}
+
+
+def algorithmic(wl, name, count):
+    """Algorithmic bytes and flops of `count` launches of call `name` in one step."""
+    Kent, W, H = wl.K, wl.window, wl.H
+    BQ = wl.B * wl.Q
+    if name in ("index_full", "index_hier"):
+        _, n_vis = query_positions(wl)
+        # a query reads each visible 68 B key once; Q queries of a sequence share its keys
+        nbytes = sum(int(n_vis[b].max()) for b in range(wl.B)) * 68
+        flops = 2 * wl.HI * 128 * int(n_vis.sum())
+        return nbytes, flops
+    if name == "reindex":
+        return count * BQ * wl.n_blocks * wl.block * 68, count * 2 * wl.HI * 128 * BQ * wl.n_blocks * wl.block
+    if name == "attn":
+        return count * BQ * (Kent * 288 + W * 512), count * BQ * 4 * H * (Kent + W) * 512
+    if name == "pack":
+        t = wl.B * wl.new_tokens
+        return t * 1280 + (t // wl.ratio) * 356, 0
+    return 0, 0
+
+
+def query_positions(wl):
+    import synth
+    return synth.query_positions(wl)
+
+
+# ---- our implementation ---------------------------------------------------------------------
+def run_ours(args, world, rank, local):
+    import synth
+    from sparse_attention_fp4_pack_b200 import csa2
+    from sparse_attention_fp4_pack_b200.decode import CallTimer, DecodeStep
+    from sparse_attention_fp4_pack_b200.workload import build_state
+
+    csa2.lib()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl = synth.workload(args.workload)
+    sched = synth.layer_schedule(wl)
+    qd = synth.step_queries(wl)
+    x = build_state(wl, lambda b: synth.seq_tokens(wl, b, device=dev), qd, device=dev)
+    step = DecodeStep(B=wl.B, Q=wl.Q, H=wl.H, HI=wl.HI, K=wl.K, window=wl.window, ratio=wl.ratio,
+                      schedule=sched, hier=wl.hier, max_n_vis=max(wl.lengths), n_blocks=wl.n_blocks,
+                      block=wl.block, device=dev)
+    step.timer = CallTimer()
+    step.capture(x)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # 256 MB > 126 MB L2
+
+    def one(timed):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step.replay()
+        e1.record()
+        flush.fill_(1)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1), step.timer.collect()
+
+    for _ in range(args.warmup):
+        one(False)
+    step.check_status()
+    clocks = ClockSampler(dev)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    total_ms, per_call = 0.0, {}
+    for _ in range(args.steps):
+        ms, calls = one(True)
+        total_ms += ms
+        for k, v in calls.items():
+            per_call[k] = per_call.get(k, 0.0) + v
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    step.check_status()
+    t_max = max_over_ranks(total_ms, world)
+
+    # ---- end to end through the public API: pinned host inputs in, results out ----------
+    h_in = {k: getattr(x, k).cpu().pin_memory() for k in ("new_kv", "new_ik", "q", "qi", "w", "swa")}
+    h_out = {"out": torch.empty_like(step.out, device="cpu").pin_memory(),
+             "lse": torch.empty_like(step.lse, device="cpu").pin_memory(),
+             "topk": torch.empty_like(step.topk, device="cpu").pin_memory()}
+    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+    e2e_ms = 0.0
+    for i in range(args.warmup + args.steps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for k, t in h_in.items():
+            getattr(x, k).copy_(t, non_blocking=True)
+        step.replay()
+        h_out["out"].copy_(step.out, non_blocking=True)
+        h_out["lse"].copy_(step.lse, non_blocking=True)
+        h_out["topk"].copy_(step.topk, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            e2e_ms += e0.elapsed_time(e1)
+        flush.fill_(1)
+    e2e_max = max_over_ranks(e2e_ms, world)
+
+    tokens = wl.B * wl.Q * world
+    us_per_token = t_max * 1000.0 / (args.steps * tokens)
+    e2e_us = e2e_max * 1000.0 / (args.steps * tokens)
+
+    # roofline of the dominant call
+    peaks = load_peaks()
+    counts = step.timer.counts()
+    dom = max(per_call, key=lambda k: per_call[k])
+    avg_ms = per_call[dom] / args.steps / counts[dom]
+    nbytes, flops = algorithmic(wl, dom, 1)
+    kernel_info = dominant_kernel_info(dom)
+    if kernel_info["bound"] == "hbm":
+        achieved = nbytes / (avg_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm"], 4), "traffic": None}
+    elif kernel_info["bound"] == "alu":
+        fp32_peak = 148 * 128 * 2 * peaks["sm_mhz"] * 1e6 / 1e12
+        achieved = flops / (avg_ms * 1e-3) / 1e12
+        roof = {"bound": "alu", "achieved": round(achieved, 2), "peak": round(fp32_peak, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / fp32_peak, 4), "traffic": None}
+    else:
+        achieved = flops / (avg_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16"], 4), "traffic": None}
+    roof.update({"kernel": kernel_info["kernel"], "call": dom, "avg_launch_ms": round(avg_ms, 4),
+                 "algorithmic_bytes": nbytes, "algorithmic_flops": flops, "peak_src": peaks["src"]})
+
+    breakdown = {k: round(v / args.steps, 4) for k, v in per_call.items()}
+    line = {
+        "metric": METRIC, "value": round(us_per_token, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 4),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": DTYPE,
+        "data": "synthetic (seeded)",
+        "config": {"workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}", "B": wl.B, "Q": wl.Q,
+                   "H": wl.H, "HI": wl.HI, "K": wl.K, "window": wl.window, "layers": len(sched),
+                   "entries_per_seq": max(wl.lengths), "parallelism": f"replicas x{world}",
+                   "l2": "cache 1.5 GB > L2 and a 256 MB L2 flush between timed steps",
+                   "graph": "CUDA graph replay"},
+        "e2e": {"value": round(e2e_us, 3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": step.launches_per_step() * args.steps,
+        "roofline": roof,
+        "ms_per_call": breakdown,
+        "clocks": clk,
+    }
+    return line, wl, x
+
+
+def dominant_kernel_info(call):
+    return {
+        "index_hier": {"kernel": "scan_tc_kernel<hier> + select_kernel", "bound": "hbm"},
+        "index_full": {"kernel": "scan_tc_kernel<flat> + select_kernel", "bound": "hbm"},
+        "reindex": {"kernel": "scan_tc_kernel<reindex> + select_kernel", "bound": "hbm"},
+        "attn": {"kernel": "attn_tc_kernel + attn_combine_kernel", "bound": "tensor"},
+        "pack": {"kernel": "pack_kv_kernel", "bound": "hbm"},
+    }[call]
+
+
+# arithmetic of the path: int8 x int8 -> int32 indexer dots (tcgen05 kind::i8) and
+# f16 x f16 -> fp32 attention (tcgen05 kind::f16), fp32 epilogues; FP4/FP8 storage
+DTYPE = "f16+i8"
+
+
+# ---- the oracle, timed on the host cores ------------------------------------------------------
+def oracle_sample_state(wl, nseq, device):
+    """The oracle's own pool for the first `nseq` sequences (packed from the same seeded
+    tokens) plus the step inputs of those sequences."""
+    import oracle
+    import synth
+    lengths = [int(n) for n in wl.lengths[:nseq]]
+    bases = np.cumsum([0] + lengths[:-1]).astype(np.int64)
+    kv_pools, ik_pools, new_kv, new_ik = [], [], [], []
+    for b in range(nseq):
+        kv, ik = synth.seq_tokens(wl, b, device=device)
+        old = kv.shape[0] - wl.new_tokens
+        kvb = kv.cpu().view(torch.int16).numpy().astype(np.uint16)
+        ikb = ik.cpu().view(torch.int16).numpy().astype(np.uint16)
+        del kv, ik
+        a, c = oracle.pack_kv(kvb[:old], ikb[:old], wl.ratio)
+        kv_pools.append(np.concatenate([a, np.zeros((wl.new_tokens // wl.ratio, 288), np.uint8)]))
+        ik_pools.append(np.concatenate([c, np.zeros((wl.new_tokens // wl.ratio, 68), np.uint8)]))
+        new_kv.append(kvb[old:])
+        new_ik.append(ikb[old:])
+    qd = synth.step_queries(wl)
+    sl = slice(0, nseq)
+    return dict(kv_pool=np.concatenate(kv_pools), ik_pool=np.concatenate(ik_pools), base=bases,
+                lengths=lengths, new_kv=new_kv, new_ik=new_ik,
+                q=qd["q"][:, sl].numpy(), qi=qd["qi"][:, sl].numpy(), w=qd["w"][:, sl].numpy(),
+                swa=qd["swa"][:, sl].numpy(), swa_start=qd["swa_start"][sl].numpy(),
+                q_pos=qd["q_pos"][sl].numpy(), n_vis=qd["n_vis"][sl].numpy())
+
+
+def oracle_step(wl, st):
+    """One decode step of the sample, entirely in the oracle."""
+    import oracle
+    import synth
+    sched = synth.layer_schedule(wl)
+    sm = 1.0 / math.sqrt(512)
+    for b in range(len(st["lengths"])):  # pack the step's new tokens into their slots
+        a, c = oracle.pack_kv(st["new_kv"][b], st["new_ik"][b], wl.ratio)
+        e0 = st["base"][b] + st["lengths"][b] - a.shape[0]
+        st["kv_pool"][e0:e0 + a.shape[0]] = a
+        st["ik_pool"][e0:e0 + a.shape[0]] = c
+    cur = blocks = None
+    for l, mode in enumerate(sched):
+        if mode == "full":
+            if wl.hier:
+                blocks, _ = oracle.index_hier(st["qi"][l], st["w"][l], st["ik_pool"], st["base"], st["n_vis"],
+                                              wl.n_blocks, wl.block)
+                cur, _ = oracle.reindex(st["qi"][l], st["w"][l], st["ik_pool"], st["base"], st["n_vis"], blocks,
+                                        wl.K, block=wl.block)
+            else:
+                cur, _ = oracle.index_full(st["qi"][l], st["w"][l], st["ik_pool"], st["base"], st["n_vis"], wl.K)
+        elif mode == "reindex":
+            cur, _ = oracle.reindex(st["qi"][l], st["w"][l], st["ik_pool"], st["base"], st["n_vis"], blocks, wl.K,
+                                    block=wl.block)
+        oracle.sparse_attn(st["q"][l], st["kv_pool"], st["base"], cur, st["swa"][l], st["swa_start"], st["q_pos"],
+                           sm, window=wl.window)
+
+
+def time_oracle(wl, nseq, steps, warmup, device):
+    import oracle
+    st = oracle_sample_state(wl, nseq, device)
+    for _ in range(warmup):
+        oracle_step(wl, st)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle_step(wl, st)
+    dt = time.perf_counter() - t0
+    tokens = nseq * wl.Q
+    cores = min(oracle.num_threads(), nseq * wl.Q)
+    sample = (f"{nseq} of {wl.B} sequences of the {wl.name} workload (full context, all "
+              f"{wl.n_layers} layers), {steps} step(s)")
+    return dt * 1e6 / (steps * tokens), cores, sample
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        if rank == 0:
+            import synth
+            wl = synth.workload(args.workload)
+            dev = "cuda" if torch.cuda.is_available() else "cpu"
+            v, cores, sample = time_oracle(wl, args.cpu_seqs, args.steps, args.warmup, dev)
+            line = {"impl": "reference", "metric": METRIC, "value": round(v, 1), "unit": UNIT, "n_gpus": world,
+                    "steps": args.steps, "warmup": args.warmup, "higher_is_better": False, "scaling": "weak",
+                    "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+                    "config": {"workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}"},
+                    "cpu_baseline": {"value": round(v, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
+                                     "sample": sample},
+                    "e2e": {"value": round(v, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            print(json.dumps(line, ensure_ascii=False), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    line, wl, x = run_ours(args, world, rank, local)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        del x
+        torch.cuda.empty_cache()
+        v, cores, sample = time_oracle(wl, args.cpu_seqs, 1, 0, "cuda")
+        line["cpu_baseline"] = {"value": round(v, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(line, ensure_ascii=False), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

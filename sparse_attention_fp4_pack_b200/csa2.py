@@ -1,0 +1,234 @@
+"""Thin ctypes binding of libcsa2 (C ABI in include/csa2.h).
+
+Argument marshalling only: every function checks tensor devices/dtypes/shapes, passes
+raw device pointers and the current CUDA stream to the C entry point of the same name,
+and raises CSA2Error on a non-OK status.  All compute runs in libcsa2's kernels; there
+is no other code path.  Workspaces are plain uint8 device tensors from torch's
+allocator (``workspace``).
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa2.so")
+
+CSA2_OK = 0
+STATUS_NAMES = {0: "CSA2_OK", 1: "CSA2_ERR_INVALID_ARG", 2: "CSA2_ERR_UNSUPPORTED", 3: "CSA2_ERR_CUDA",
+                4: "CSA2_ERR_TIMEOUT", 5: "CSA2_ERR_DEVICE_INPUT"}
+DEV_BAD_INDEX, DEV_BAD_COUNT, DEV_TIMEOUT = 0x1, 0x2, 0x4
+
+D, DI, KV_BYTES, IK_BYTES = 512, 128, 288, 68
+
+_lib = None
+
+
+class CSA2Error(RuntimeError):
+    def __init__(self, status, what=""):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+
+
+def lib():
+    """Load libcsa2.so (raises if it was not built: there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with __graft_entry__.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, I32, SZ, F32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+        L.csa2_status_string.restype = ctypes.c_char_p
+        L.csa2_status_string.argtypes = [I32]
+        L.csa2_status_from_device_word.restype = I32
+        L.csa2_status_from_device_word.argtypes = [ctypes.c_uint32]
+        L.csa2_version.restype = I32
+        L.csa2_pack_kv.restype = I32
+        L.csa2_pack_kv.argtypes = [P, P, I64, I32, P, I64, P, P, P, P]
+        L.csa2_index_full_workspace_size.restype = SZ
+        L.csa2_index_full_workspace_size.argtypes = [I32, I32, I32, I32, I64]
+        L.csa2_index_full.restype = I32
+        L.csa2_index_full.argtypes = [P, P, P, I64, P, P, I32, I32, I32, I32, I64, P, P, P, SZ, P, P]
+        L.csa2_index_hier_workspace_size.restype = SZ
+        L.csa2_index_hier_workspace_size.argtypes = [I32, I32, I32, I32, I32, I64]
+        L.csa2_index_hier.restype = I32
+        L.csa2_index_hier.argtypes = [P, P, P, I64, P, P, I32, I32, I32, I32, I32, I64, P, P, P, SZ, P, P]
+        L.csa2_reindex_workspace_size.restype = SZ
+        L.csa2_reindex_workspace_size.argtypes = [I32, I32, I32, I32, I32, I32]
+        L.csa2_reindex.restype = I32
+        L.csa2_reindex.argtypes = [P, P, P, I64, P, P, P, I32, I32, I32, I32, I32, I32, P, P, P, SZ, P, P]
+        L.csa2_sparse_attn_workspace_size.restype = SZ
+        L.csa2_sparse_attn_workspace_size.argtypes = [I32, I32, I32, I32, I32]
+        L.csa2_sparse_attn.restype = I32
+        L.csa2_sparse_attn.argtypes = [P, P, I64, P, P, I32, P, I32, P, P, I32, I32, I32, I32, F32, P, P, P,
+                                       SZ, P, P]
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status, what):
+    if status != CSA2_OK:
+        raise CSA2Error(status, what)
+
+
+def _need(t, dtype, name, ndim=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+
+
+def workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A uint8 device buffer usable as csa2 workspace (torch's allocator aligns to 512 B)."""
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device or "cuda")
+
+
+def status_word(device=None) -> torch.Tensor:
+    """A zeroed device status word for the dev_status argument."""
+    return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+
+
+def status_from_device_word(word: int) -> int:
+    return lib().csa2_status_from_device_word(word & 0xFFFFFFFF)
+
+
+def version() -> int:
+    return lib().csa2_version()
+
+
+# ---- a1 ---------------------------------------------------------------------------------
+def csa2_pack_kv(kv, ik, ratio, kv_pool, ik_pool, dst_entry=None, dev_status=None, stream=None):
+    """kv bf16 [T,512], ik bf16 [T,128] -> entries written into kv_pool u8 [P,288] and
+    ik_pool u8 [P,68] (slots dst_entry int64 [T/ratio], or 0..T/ratio-1)."""
+    _need(kv, torch.bfloat16, "kv", 2)
+    _need(ik, torch.bfloat16, "ik", 2)
+    _need(kv_pool, torch.uint8, "kv_pool", 2)
+    _need(ik_pool, torch.uint8, "ik_pool", 2)
+    _need(dst_entry, torch.int64, "dst_entry", 1)
+    T = kv.shape[0]
+    assert kv.shape == (T, D) and ik.shape == (T, DI)
+    assert kv_pool.shape[1] == KV_BYTES and ik_pool.shape[1] == IK_BYTES and kv_pool.shape[0] == ik_pool.shape[0]
+    if dst_entry is not None and dst_entry.numel() != T // max(int(ratio), 1):
+        raise ValueError("dst_entry must hold one slot per new entry (T // ratio)")
+    _check(lib().csa2_pack_kv(_ptr(kv), _ptr(ik), T, int(ratio), _ptr(dst_entry), kv_pool.shape[0],
+                              _ptr(kv_pool), _ptr(ik_pool), _ptr(dev_status), _stream(stream)),
+           "csa2_pack_kv")
+
+
+# ---- a2/a3 ------------------------------------------------------------------------------
+def csa2_index_full_workspace_size(B, Q, HI, K, max_n_vis):
+    return lib().csa2_index_full_workspace_size(B, Q, HI, K, max_n_vis)
+
+
+def csa2_index_full(q, w, ik_pool, seq_base, n_vis, K, max_n_vis, topk, topk_score=None, ws=None,
+                    dev_status=None, stream=None):
+    """q f32 [B,Q,HI,128], w f32 [B,Q,HI], ik_pool u8 [P,68], seq_base i64 [B],
+    n_vis i32 [B,Q] -> topk i32 [B,Q,K] (+ topk_score f32 [B,Q,K])."""
+    _need(q, torch.float32, "q", 4)
+    _need(w, torch.float32, "w", 3)
+    _need(ik_pool, torch.uint8, "ik_pool", 2)
+    _need(seq_base, torch.int64, "seq_base", 1)
+    _need(n_vis, torch.int32, "n_vis", 2)
+    _need(topk, torch.int32, "topk", 3)
+    _need(topk_score, torch.float32, "topk_score", 3)
+    B, Q, HI, _ = q.shape
+    if ws is None:
+        ws = workspace(csa2_index_full_workspace_size(B, Q, HI, K, max_n_vis), q.device)
+    _check(lib().csa2_index_full(_ptr(q), _ptr(w), _ptr(ik_pool), ik_pool.shape[0], _ptr(seq_base),
+                                 _ptr(n_vis), B, Q, HI, K, int(max_n_vis), _ptr(topk), _ptr(topk_score),
+                                 _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)),
+           "csa2_index_full")
+
+
+# ---- a4 ---------------------------------------------------------------------------------
+def csa2_index_hier_workspace_size(B, Q, HI, n_blocks, block, max_n_vis):
+    return lib().csa2_index_hier_workspace_size(B, Q, HI, n_blocks, block, max_n_vis)
+
+
+def csa2_index_hier(q, w, ik_pool, seq_base, n_vis, n_blocks, block, max_n_vis, blocks, block_score=None,
+                    ws=None, dev_status=None, stream=None):
+    _need(q, torch.float32, "q", 4)
+    _need(w, torch.float32, "w", 3)
+    _need(ik_pool, torch.uint8, "ik_pool", 2)
+    _need(seq_base, torch.int64, "seq_base", 1)
+    _need(n_vis, torch.int32, "n_vis", 2)
+    _need(blocks, torch.int32, "blocks", 3)
+    _need(block_score, torch.float32, "block_score", 3)
+    B, Q, HI, _ = q.shape
+    if ws is None:
+        ws = workspace(csa2_index_hier_workspace_size(B, Q, HI, n_blocks, block, max_n_vis), q.device)
+    _check(lib().csa2_index_hier(_ptr(q), _ptr(w), _ptr(ik_pool), ik_pool.shape[0], _ptr(seq_base),
+                                 _ptr(n_vis), B, Q, HI, n_blocks, block, int(max_n_vis), _ptr(blocks),
+                                 _ptr(block_score), _ptr(ws), ws.numel(), _ptr(dev_status),
+                                 _stream(stream)),
+           "csa2_index_hier")
+
+
+# ---- a5 ---------------------------------------------------------------------------------
+def csa2_reindex_workspace_size(B, Q, HI, n_blocks, block, K):
+    return lib().csa2_reindex_workspace_size(B, Q, HI, n_blocks, block, K)
+
+
+def csa2_reindex(q, w, ik_pool, seq_base, n_vis, blocks, block, K, topk, topk_score=None, ws=None,
+                 dev_status=None, stream=None):
+    _need(q, torch.float32, "q", 4)
+    _need(w, torch.float32, "w", 3)
+    _need(ik_pool, torch.uint8, "ik_pool", 2)
+    _need(seq_base, torch.int64, "seq_base", 1)
+    _need(n_vis, torch.int32, "n_vis", 2)
+    _need(blocks, torch.int32, "blocks", 3)
+    _need(topk, torch.int32, "topk", 3)
+    _need(topk_score, torch.float32, "topk_score", 3)
+    B, Q, HI, _ = q.shape
+    n_blocks = blocks.shape[-1]
+    if ws is None:
+        ws = workspace(csa2_reindex_workspace_size(B, Q, HI, n_blocks, block, K), q.device)
+    _check(lib().csa2_reindex(_ptr(q), _ptr(w), _ptr(ik_pool), ik_pool.shape[0], _ptr(seq_base),
+                              _ptr(n_vis), _ptr(blocks), n_blocks, block, B, Q, HI, K, _ptr(topk),
+                              _ptr(topk_score), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)),
+           "csa2_reindex")
+
+
+# ---- a6/a7 ------------------------------------------------------------------------------
+def csa2_sparse_attn_workspace_size(B, Q, H, K, window):
+    return lib().csa2_sparse_attn_workspace_size(B, Q, H, K, window)
+
+
+def csa2_sparse_attn(q, kv_pool, seq_base, topk, swa, swa_start, q_pos, sm_scale, out, lse, window=128,
+                     ws=None, dev_status=None, stream=None):
+    """q f32 [B,Q,H,512]; kv_pool u8 [P,288]; topk i32 [B,Q,K]; swa u8 [B,S_w,512] or None;
+    swa_start i64 [B]; q_pos i64 [B,Q] -> out f32 [B,Q,H,512], lse f32 [B,Q,H]."""
+    _need(q, torch.float32, "q", 4)
+    _need(kv_pool, torch.uint8, "kv_pool", 2)
+    _need(seq_base, torch.int64, "seq_base", 1)
+    _need(topk, torch.int32, "topk", 3)
+    _need(swa, torch.uint8, "swa", 3)
+    _need(swa_start, torch.int64, "swa_start", 1)
+    _need(q_pos, torch.int64, "q_pos", 2)
+    _need(out, torch.float32, "out", 4)
+    _need(lse, torch.float32, "lse", 3)
+    B, Q, H, _ = q.shape
+    K = topk.shape[-1] if topk is not None else 0
+    S_w = swa.shape[1] if swa is not None else 0
+    if ws is None:
+        ws = workspace(csa2_sparse_attn_workspace_size(B, Q, H, K, window), q.device)
+    _check(lib().csa2_sparse_attn(_ptr(q), _ptr(kv_pool), kv_pool.shape[0], _ptr(seq_base), _ptr(topk), K,
+                                  _ptr(swa), S_w, _ptr(swa_start), _ptr(q_pos), int(window), B, Q, H,
+                                  float(sm_scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                  _ptr(dev_status), _stream(stream)),
+           "csa2_sparse_attn")

@@ -1,0 +1,73 @@
+// Device-side helpers shared by the libcsa2 kernels (sm_100a).
+//
+// Format facts (P3 = genexis.ai "100만 토큰을 0.9GB에, 딥시크 V4.1 논문이 KV 캐시를 줄인
+// 방법", §4비트로 적어도 되는 이유 and §레이어 40개 가운데 4개만 전역 캐시를 만듭니다):
+// E2M1 values with one E4M3 scale per 16 channels (288 B per 512-channel entry) and a
+// 68 B indexer key (64 B E2M1 codes + fp32 scale).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "csa2.h"
+
+namespace csa2 {
+
+constexpr int kD = CSA2_D;
+constexpr int kDI = CSA2_DI;
+constexpr int kKvBytes = CSA2_KV_ENTRY_BYTES;
+constexpr int kIkBytes = CSA2_IK_ENTRY_BYTES;
+
+__device__ __forceinline__ void flag(uint32_t* status, uint32_t bit) {
+  if (status) atomicOr(status, bit);
+}
+
+// bf16 pair (element 2i in the low half) -> two fp32 values.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Two non-negative fp32 values -> one byte of two E2M1 codes (lo in bits 3..0), round to
+// nearest even, saturating at 6.
+__device__ __forceinline__ uint32_t e2m1x2_rn_sat(float lo, float hi) {
+  uint16_t r;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+      "cvt.u16.u8 %0, t;\n\t}"
+      : "=h"(r)
+      : "f"(hi), "f"(lo));
+  return r & 0xFFu;
+}
+
+// Non-negative fp32 -> E4M3 byte, round to nearest even, saturating at 448.
+__device__ __forceinline__ uint32_t e4m3_rn_sat(float x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+  return r & 0xFFu;
+}
+
+// E4M3 byte (sign clear) -> fp32, exact.
+__device__ __forceinline__ float e4m3_value(uint32_t s) {
+  uint32_t e = (s >> 3) & 15u, m = s & 7u;
+  if (e == 0) return __uint2float_rn(m) * 0.001953125f;  // m * 2^-9
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// E2M1 magnitude code (0..7) -> fp32.
+__device__ __forceinline__ float e2m1_mag(uint32_t m) {
+  // 0, 0.5, 1, 1.5, 2, 3, 4, 6 : for m >= 2 the fp32 exponent is 126 + (m >> 1) and the
+  // top mantissa bit is m & 1; m = 1 is the subnormal 0.5.
+  float v = __uint_as_float(((126u + (m >> 1)) << 23) | ((m & 1u) << 22));
+  return m >= 2 ? v : (m == 1 ? 0.5f : 0.0f);
+}
+
+// Order-preserving map of an fp32 score onto uint32 (larger score -> larger key).
+// Key 0 is reserved for "no candidate" (it is the image of a negative NaN only).
+__device__ __forceinline__ uint32_t score_key(float s) {
+  uint32_t b = __float_as_uint(s);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_score(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+}  // namespace csa2

@@ -1,0 +1,142 @@
+// a1: pack new global-KV entries into the FP4 layout.
+//
+// P3 (genexis.ai "100만 토큰을 0.9GB에, 딥시크 V4.1 논문이 KV 캐시를 줄인 방법"):
+//   §레이어 40개 가운데 4개만 전역 캐시를 만듭니다 — 288 B FP4 main KV (256 B values +
+//   32 B scales) + 68 B indexer key per entry; encoder entries cover 2 tokens.
+//   §4비트로 적어도 되는 이유 — NVFP4 without the second-level global scale: one 8-bit
+//   scale per 16 channels.
+//
+// One warp packs one entry: lane l owns main-KV block l (channels 16l..16l+15, 32 B of
+// bf16 per token, so a warp reads 1 KB contiguous) and indexer dims 4l..4l+3.  The
+// kernel is HBM-bound (1280 B read + 356 B written per 1:1 entry), so the per-element
+// work is kept to a few instructions:
+//   * the main-KV quotient x/scale is formed from |x| with a correctly rounded
+//     reciprocal r = 1/scale and one FMA correction (Markstein's refinement,
+//     q = y0 + r*(|x| - scale*y0), y0 = |x|*r).  For every finite x whose block scale is
+//     scale, the E2M1 code of q equals the code of the IEEE quotient: scales have at
+//     most 4 significant bits, so the exact quotient is never within half an ulp of an
+//     E2M1 rounding midpoint unless it equals it; the parity tests check this over every
+//     bf16 value against every scale.  The sign bit is taken from x itself.
+//   * the indexer-key quotient uses IEEE division (its scale is a full fp32 value).
+#include "csa2_device.cuh"
+
+namespace csa2 {
+
+__device__ __forceinline__ float refined_quot(float a, float sd, float r) {
+  float y0 = a * r;
+  float e = fmaf(-y0, sd, a);
+  return fmaf(e, r, y0);
+}
+
+__global__ void __launch_bounds__(256) pack_kv_kernel(const uint16_t* __restrict__ kv,
+                                                      const uint16_t* __restrict__ ik, int64_t E,
+                                                      int ratio, const int64_t* __restrict__ dst,
+                                                      int64_t pool_entries,
+                                                      uint8_t* __restrict__ kv_pool,
+                                                      uint8_t* __restrict__ ik_pool,
+                                                      uint32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t j = warp0; j < E; j += nwarps) {
+    const int64_t d = dst ? dst[j] : j;
+    if (d < 0 || d >= pool_entries) {
+      if (lane == 0) flag(status, CSA2_DEV_BAD_INDEX);
+      continue;
+    }
+    // ---- main KV block `lane` -------------------------------------------------------
+    float x[16];
+    {
+      const uint4* p0 = reinterpret_cast<const uint4*>(kv + (j * ratio) * kD) + lane * 2;
+      uint4 a0 = __ldcs(p0), a1 = __ldcs(p0 + 1);
+      uint32_t w[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      if (ratio == 1) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          x[2 * i] = bf16_lo(w[i]);
+          x[2 * i + 1] = bf16_hi(w[i]);
+        }
+      } else {
+        const uint4* p1 = p0 + kD / 8;  // next token
+        uint4 b0 = __ldcs(p1), b1 = __ldcs(p1 + 1);
+        uint32_t v[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          x[2 * i] = (bf16_lo(w[i]) + bf16_lo(v[i])) * 0.5f;
+          x[2 * i + 1] = (bf16_hi(w[i]) + bf16_hi(v[i])) * 0.5f;
+        }
+      }
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    const uint32_t s = e4m3_rn_sat(__fdiv_rn(amax, 6.0f));
+    const float sd = e4m3_value(s);
+    uint32_t c0 = 0, c1 = 0;
+    if (sd != 0.0f) {
+      const float r = __frcp_rn(sd);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float q0 = refined_quot(fabsf(x[2 * i]), sd, r);
+        float q1 = refined_quot(fabsf(x[2 * i + 1]), sd, r);
+        uint32_t byte = e2m1x2_rn_sat(q0, q1);
+        byte |= ((__float_as_uint(x[2 * i]) >> 31) << 3) | ((__float_as_uint(x[2 * i + 1]) >> 31) << 7);
+        if (i < 4)
+          c0 |= byte << (8 * i);
+        else
+          c1 |= byte << (8 * (i - 4));
+      }
+    }
+    uint8_t* ek = kv_pool + d * kKvBytes;
+    __stcs(reinterpret_cast<uint2*>(ek) + lane, make_uint2(c0, c1));
+    ek[256 + lane] = (uint8_t)s;
+
+    // ---- indexer key dims 4*lane .. 4*lane+3 ------------------------------------------
+    float y[4];
+    {
+      const uint2* p0 = reinterpret_cast<const uint2*>(ik + (j * ratio) * kDI) + lane;
+      uint2 a = __ldcs(p0);
+      if (ratio == 1) {
+        y[0] = bf16_lo(a.x); y[1] = bf16_hi(a.x); y[2] = bf16_lo(a.y); y[3] = bf16_hi(a.y);
+      } else {
+        uint2 b = __ldcs(p0 + kDI / 4);
+        y[0] = (bf16_lo(a.x) + bf16_lo(b.x)) * 0.5f;
+        y[1] = (bf16_hi(a.x) + bf16_hi(b.x)) * 0.5f;
+        y[2] = (bf16_lo(a.y) + bf16_lo(b.y)) * 0.5f;
+        y[3] = (bf16_hi(a.y) + bf16_hi(b.y)) * 0.5f;
+      }
+    }
+    float im = fmaxf(fmaxf(fabsf(y[0]), fabsf(y[1])), fmaxf(fabsf(y[2]), fabsf(y[3])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) im = fmaxf(im, __shfl_xor_sync(0xffffffffu, im, o));
+    const float is = __fdiv_rn(im, 6.0f);
+    uint32_t ic = 0;
+    if (is != 0.0f) {
+      uint32_t b0 = e2m1x2_rn_sat(__fdiv_rn(fabsf(y[0]), is), __fdiv_rn(fabsf(y[1]), is));
+      uint32_t b1 = e2m1x2_rn_sat(__fdiv_rn(fabsf(y[2]), is), __fdiv_rn(fabsf(y[3]), is));
+      b0 |= ((__float_as_uint(y[0]) >> 31) << 3) | ((__float_as_uint(y[1]) >> 31) << 7);
+      b1 |= ((__float_as_uint(y[2]) >> 31) << 3) | ((__float_as_uint(y[3]) >> 31) << 7);
+      ic = b0 | (b1 << 8);
+    }
+    uint8_t* ei = ik_pool + d * kIkBytes;
+    reinterpret_cast<uint16_t*>(ei)[lane] = (uint16_t)ic;
+    if (lane == 0) *reinterpret_cast<float*>(ei + 64) = is;
+  }
+}
+
+cudaError_t launch_pack_kv(const void* kv, const void* ik, int64_t T, int ratio,
+                           const int64_t* dst, int64_t pool_entries, uint8_t* kv_pool,
+                           uint8_t* ik_pool, uint32_t* status, cudaStream_t stream, int num_sms) {
+  const int64_t E = T / ratio;
+  if (E == 0) return cudaSuccess;
+  const int threads = 256;
+  int64_t blocks = (E + 7) / 8;
+  const int64_t cap = (int64_t)num_sms * 16;  // 16 resident 256-thread blocks per SM
+  if (blocks > cap) blocks = cap;
+  pack_kv_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
+      static_cast<const uint16_t*>(kv), static_cast<const uint16_t*>(ik), E, ratio, dst,
+      pool_entries, kv_pool, ik_pool, status);
+  return cudaGetLastError();
+}
+
+}  // namespace csa2

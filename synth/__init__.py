@@ -81,19 +81,6 @@ def index_queries(seed, B, Q, HI, device="cpu", stream="qi"):
     return q, w
 
 
-def plant_keys(seed, ik_tokens, seq_base, lengths, n_plant=64, gain=4.0, stream="plant"):
-    """Scale n_plant random indexer-key tokens per sequence by `gain` (in place), so that
-    block selection has clear winners.  Returns the planted positions [B, n_plant]."""
-    g = _gen(seed, stream, "cpu")
-    pos = []
-    for b, n in enumerate(lengths):
-        p = torch.randint(0, int(n), (n_plant,), generator=g)
-        rows = (int(seq_base[b]) + p).to(ik_tokens.device)
-        ik_tokens[rows] = (ik_tokens[rows].float() * gain).to(ik_tokens.dtype)
-        pos.append(p)
-    return torch.stack(pos)
-
-
 @dataclass
 class DecodeWorkload:
     """Shapes of one decode (or verify) step; all layers share the global FP4 cache."""
@@ -165,3 +152,42 @@ def seq_bases(lengths):
         base.append(acc)
         acc += int(n)
     return torch.tensor(base, dtype=torch.int64), acc
+
+
+def seq_tokens(wl: DecodeWorkload, b: int, device="cpu", lo=0, hi=None):
+    """Raw bf16 tokens [lo, hi) of sequence b (lengths[b] * ratio tokens in all); each
+    sequence is its own stream, so any slice can be regenerated on its own.  The
+    hierarchical workload plants 64 high-norm indexer keys per sequence."""
+    T = int(wl.lengths[b]) * wl.ratio
+    hi = T if hi is None else hi
+    kv, ik = kv_tokens(wl.seed, T, device=device, recipe=wl.recipe, stream=f"seq{b}")
+    if wl.hier:
+        g = _gen(wl.seed, f"plant{b}", "cpu")
+        rows = torch.randint(0, T, (64,), generator=g).to(ik.device)
+        ik[rows] = (ik[rows].float() * 4.0).to(ik.dtype)
+    return kv[lo:hi], ik[lo:hi]
+
+
+def step_queries(wl: DecodeWorkload, device="cpu"):
+    """Per-layer queries and windows of one step.
+
+    Returns a dict: q f32 [L,B,Q,H,512]; qi f32 [L,B,Q,HI,128]; w f32 [L,B,Q,HI];
+    swa u8 [L,B,S_w,512] with S_w = window + Q - 1 (the rows the Q queries need);
+    swa_start i64 [B]; q_pos i64 [B,Q]; n_vis i32 [B,Q]."""
+    L = wl.n_layers
+    sched = layer_schedule(wl)
+    q = queries(wl.seed, L * wl.B, wl.Q, wl.H, device, stream="q").reshape(L, wl.B, wl.Q, wl.H, D)
+    qi, w = index_queries(wl.seed, L * wl.B, wl.Q, wl.HI, device, stream="qi")
+    qi = qi.reshape(L, wl.B, wl.Q, wl.HI, DI)
+    w = w.reshape(L, wl.B, wl.Q, wl.HI)
+    for l, mode in enumerate(sched):  # Reuse layers do no indexing: their rows are unused
+        if mode == "reuse":
+            qi[l].zero_()
+            w[l].zero_()
+    S_w = wl.window + wl.Q - 1
+    swa = swa_window(wl.seed, L * wl.B, S_w, device).reshape(L, wl.B, S_w, D)
+    q_pos, n_vis = query_positions(wl)
+    T = torch.tensor([int(n) * wl.ratio for n in wl.lengths], dtype=torch.int64)
+    swa_start = T - S_w
+    return dict(q=q, qi=qi, w=w, swa=swa, swa_start=swa_start.to(device), q_pos=q_pos.to(device),
+                n_vis=n_vis.to(device))

@@ -1,0 +1,99 @@
+"""CPU checks of the C-ABI library: it loads, exports every symbol include/csa2.h
+declares, sizes workspaces, maps status codes, and rejects bad arguments before
+launching anything (none of these calls reaches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_attention_fp4_pack_b200 import build as libbuild
+from sparse_attention_fp4_pack_b200 import csa2
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "csa2.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    libbuild.build()
+    return csa2.lib()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(csa2_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = header_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), f"libcsa2.so does not export {n}"
+        assert ctypes.cast(getattr(L, n), ctypes.c_void_p).value
+
+
+def test_status_strings_and_device_word(L):
+    for s in range(6):
+        assert L.csa2_status_string(s).decode().startswith(csa2.STATUS_NAMES[s])
+    assert L.csa2_status_from_device_word(0) == 0
+    assert L.csa2_status_from_device_word(csa2.DEV_BAD_INDEX) == 5
+    assert L.csa2_status_from_device_word(csa2.DEV_BAD_COUNT) == 5
+    assert L.csa2_status_from_device_word(csa2.DEV_TIMEOUT | csa2.DEV_BAD_INDEX) == 4
+    assert L.csa2_version() >= 100
+
+
+def test_workspace_sizes(L):
+    assert L.csa2_index_full_workspace_size(32, 1, 8, 512, 131072) >= 32 * 131072 * 4
+    assert L.csa2_index_full_workspace_size(32, 1, 8, 512, 131072) % 256 == 0
+    assert L.csa2_index_hier_workspace_size(4, 1, 8, 2048, 8, 1 << 20) >= 4 * (1 << 17) * 4
+    assert L.csa2_reindex_workspace_size(4, 1, 8, 2048, 8, 512) >= 4 * 16384 * 4
+    assert L.csa2_sparse_attn_workspace_size(4, 1, 64, 512, 128) > 0
+    assert L.csa2_index_full_workspace_size(0, 1, 8, 512, 10) == 0
+
+
+P = ctypes.c_void_p
+FAKE = P(0x10000)       # 16-aligned, never dereferenced: validation fails before any launch
+MIS = P(0x10004)        # misaligned
+
+
+def test_pack_rejects_bad_args(L):
+    st = ctypes.c_void_p(0)
+    assert L.csa2_pack_kv(FAKE, FAKE, 8, 3, None, 8, FAKE, FAKE, None, st) == 2   # ratio
+    assert L.csa2_pack_kv(FAKE, FAKE, 7, 2, None, 8, FAKE, FAKE, None, st) == 1   # odd T at 2:1
+    assert L.csa2_pack_kv(None, FAKE, 8, 1, None, 8, FAKE, FAKE, None, st) == 1   # null
+    assert L.csa2_pack_kv(MIS, FAKE, 8, 1, None, 8, FAKE, FAKE, None, st) == 1    # misaligned
+    assert L.csa2_pack_kv(FAKE, FAKE, 16, 1, None, 8, FAKE, FAKE, None, st) == 1  # pool too small
+    assert L.csa2_pack_kv(FAKE, FAKE, 0, 1, None, 0, None, None, None, st) == 0   # empty: no-op
+
+
+def test_index_rejects_bad_args(L):
+    st = ctypes.c_void_p(0)
+    args = lambda HI, K, ws, wsb: (FAKE, FAKE, FAKE, 100, FAKE, FAKE, 1, 1, HI, K, 100, FAKE, None, ws,
+                                   wsb, None, st)
+    assert L.csa2_index_full(*args(17, 512, FAKE, 1 << 20)) == 2   # HI > 16
+    assert L.csa2_index_full(*args(8, 2049, FAKE, 1 << 20)) == 2   # K > 2048
+    assert L.csa2_index_full(*args(8, 0, FAKE, 1 << 20)) == 2      # K = 0
+    assert L.csa2_index_full(*args(8, 512, FAKE, 16)) == 1         # workspace too small
+    assert L.csa2_index_full(*args(8, 512, None, 1 << 20)) == 1    # null workspace
+    assert L.csa2_index_full(*args(8, 512, P(0x10010), 1 << 20)) == 1  # workspace not 256-aligned
+    assert L.csa2_index_hier(FAKE, FAKE, FAKE, 100, FAKE, FAKE, 1, 1, 8, 2048, 3, 100, FAKE, None, FAKE,
+                             1 << 20, None, st) == 2                # block not a power of two
+    assert L.csa2_index_hier(FAKE, FAKE, FAKE, 100, FAKE, FAKE, 1, 1, 8, 4096, 8, 100, FAKE, None, FAKE,
+                             1 << 20, None, st) == 2                # too many blocks
+    assert L.csa2_reindex(FAKE, FAKE, FAKE, 100, FAKE, FAKE, None, 2048, 8, 1, 1, 8, 512, FAKE, None, FAKE,
+                          1 << 20, None, st) == 1                   # null blocks
+    assert L.csa2_index_full(FAKE, FAKE, FAKE, 100, FAKE, FAKE, 0, 1, 8, 512, 100, None, None, None, 0,
+                             None, st) == 0                          # no queries: no-op
+
+
+def test_attn_rejects_bad_args(L):
+    st = ctypes.c_void_p(0)
+    base = lambda H, K, win, sm, swa, S_w: (FAKE, FAKE, 100, FAKE, FAKE, K, swa, S_w, FAKE, FAKE, win, 1, 1, H,
+                                            ctypes.c_float(sm), FAKE, FAKE, FAKE, 1 << 30, None, st)
+    assert L.csa2_sparse_attn(*base(24, 512, 128, 0.04, FAKE, 128)) == 2        # H unsupported
+    assert L.csa2_sparse_attn(*base(64, 4096, 128, 0.04, FAKE, 128)) == 2       # K too large
+    assert L.csa2_sparse_attn(*base(64, 512, 4096, 0.04, FAKE, 128)) == 2       # window too large
+    assert L.csa2_sparse_attn(*base(64, 512, 128, float("nan"), FAKE, 128)) == 1  # scale
+    assert L.csa2_sparse_attn(*base(64, 512, 128, 0.04, None, 128)) == 1        # window data missing

@@ -1,0 +1,246 @@
+"""GPU parity of the indexer (flat Full scan + Top-K, hierarchical blocks, Reindex).
+
+Top-K and block sets must equal the oracle's except for entries whose oracle score lies
+within 1e-5 relative of the K-th oracle score.  Cases span several CTA chunks and ragged
+tails, sequence bases that are not 16-byte aligned, visible counts of 0, 1, < K and
+> 16,384, every supported head count, exact ties, and bad device-side counts.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from helpers import assert_topk_set, bf16_bits, np_u8
+from sparse_attention_fp4_pack_b200 import csa2
+
+pytestmark = pytest.mark.gpu
+
+
+def pools_from_tokens(orc, kv, ik):
+    """GPU pack and oracle pack of the same raw tokens (must agree byte for byte)."""
+    T = kv.shape[0]
+    kvp = torch.zeros(T, 288, dtype=torch.uint8, device="cuda")
+    ikp = torch.zeros(T, 68, dtype=torch.uint8, device="cuda")
+    csa2.csa2_pack_kv(kv, ik, 1, kvp, ikp)
+    o_kv, o_ik = orc.pack_kv(bf16_bits(kv), bf16_bits(ik), 1)
+    assert np.array_equal(np_u8(ikp), o_ik) and np.array_equal(np_u8(kvp), o_kv)
+    return kvp, ikp, o_kv, o_ik
+
+
+def run_full(q, w, ikp, seq_base, n_vis, K, max_n_vis):
+    B, Q = n_vis.shape
+    topk = torch.full((B, Q, K), -7, dtype=torch.int32, device="cuda")
+    score = torch.zeros(B, Q, K, dtype=torch.float32, device="cuda")
+    st = csa2.status_word()
+    csa2.csa2_index_full(q, w, ikp, seq_base, n_vis, K, max_n_vis, topk, score, dev_status=st)
+    torch.cuda.synchronize()
+    return topk.cpu().numpy(), score.cpu().numpy(), int(st.item())
+
+
+@pytest.mark.parametrize("HI,K", [(4, 512), (1, 7), (8, 512), (16, 2048), (3, 1)])
+def test_flat_ragged(orc, HI, K):
+    lengths = [1001, 37, 4099, 6000]           # bases 0, 1001, 1038, 5137: misaligned
+    T = sum(lengths)
+    kv, ik = synth.kv_tokens(30 + HI, T, device="cuda", recipe="clipped")
+    kvp, ikp, _, o_ik = pools_from_tokens(orc, kv, ik)
+    base = np.cumsum([0] + lengths[:-1]).astype(np.int64)
+    n_vis = np.array([[1001, 0], [37, 1], [4099, 513], [6000, 2500]], np.int32)
+    Q = 2
+    qh, wh = synth.index_queries(40 + HI, len(lengths), Q, HI)
+    topk, score, st = run_full(qh.cuda(), wh.cuda(), ikp, torch.from_numpy(base).cuda(),
+                               torch.from_numpy(n_vis).cuda(), K, 6000)
+    assert st == 0
+    o_topk, _ = orc.index_full(qh.numpy(), wh.numpy(), o_ik, base, n_vis, K)
+    for b in range(len(lengths)):
+        for i in range(Q):
+            n = n_vis[b, i]
+            s = orc.index_scores(qh[b, i].numpy(), wh[b, i].numpy(), o_ik[base[b]:base[b] + n])
+            assert_topk_set(topk[b, i], o_topk[b, i], s, K, what=f"b{b} q{i} n{n}")
+            sel = topk[b, i][topk[b, i] >= 0]
+            # reported scores are the scores of the reported entries, to fp32 accuracy on
+            # the scale sum_h |w_h| |q_h| . |k_j| of the terms that cancel inside the dots
+            if len(sel):
+                k = orc.dequant_ik(o_ik[base[b] + sel])
+                mag = np.abs(k) @ np.abs(qh[b, i].numpy().astype(np.float64)).T @ np.abs(wh[b, i].numpy())
+                assert (np.abs(score[b, i][: len(sel)] - s[sel]) <= 1e-6 * mag).all()
+
+
+def test_tiny_workload(orc):
+    """The tiny decode workload: N=4096, 4 indexer heads, Top-512."""
+    wl = synth.workload("tiny")
+    kv, ik = synth.seq_tokens(wl, 0, device="cuda")
+    _, ikp, _, o_ik = pools_from_tokens(orc, kv, ik)
+    qd = synth.step_queries(wl)
+    qi, w = qd["qi"][0], qd["w"][0]
+    n_vis = qd["n_vis"]
+    base = np.zeros(1, np.int64)
+    topk, _, st = run_full(qi.cuda(), w.cuda(), ikp, torch.zeros(1, dtype=torch.int64, device="cuda"),
+                           n_vis.cuda(), 512, 4096)
+    o_topk, _ = orc.index_full(qi.numpy(), w.numpy(), o_ik, base, n_vis.numpy(), 512)
+    s = orc.index_scores(qi[0, 0].numpy(), w[0, 0].numpy(), o_ik[:4096])
+    assert_topk_set(topk[0, 0], o_topk[0, 0], s, 512)
+
+
+def test_exact_ties_prefer_lower_index(orc):
+    """All-zero keys give score 0 everywhere: the K lowest indices, exactly."""
+    T = 3000
+    kv = torch.zeros(T, 512, dtype=torch.bfloat16, device="cuda")
+    ik = torch.zeros(T, 128, dtype=torch.bfloat16, device="cuda")
+    ik[2000:2100] = 1.0                         # 100 keys scoring > 0 for a positive query
+    _, ikp, _, o_ik = pools_from_tokens(orc, kv, ik)
+    q = torch.ones(1, 1, 2, 128)
+    w = torch.ones(1, 1, 2)
+    topk, _, _ = run_full(q.cuda(), w.cuda(), ikp, torch.zeros(1, dtype=torch.int64, device="cuda"),
+                          torch.tensor([[T]], dtype=torch.int32, device="cuda"), 300, T)
+    o_topk, _ = orc.index_full(q.numpy(), w.numpy(), o_ik, np.zeros(1, np.int64), np.array([[T]], np.int32), 300)
+    assert sorted(topk[0, 0].tolist()) == sorted(o_topk[0, 0].tolist())
+    assert sorted(topk[0, 0].tolist()) == list(range(200)) + list(range(2000, 2100))
+
+
+def test_bad_count_flags_and_empties(orc):
+    T = 500
+    kv, ik = synth.kv_tokens(50, T, device="cuda")
+    _, ikp, _, _ = pools_from_tokens(orc, kv, ik)
+    q, w = synth.index_queries(51, 1, 2, 4)
+    topk, _, st = run_full(q.cuda(), w.cuda(), ikp, torch.zeros(1, dtype=torch.int64, device="cuda"),
+                           torch.tensor([[600, 100]], dtype=torch.int32, device="cuda"), 16, 500)
+    assert st & csa2.DEV_BAD_COUNT
+    assert (topk[0, 0] == -1).all()           # the bad query selects nothing
+    assert (topk[0, 1] >= 0).all()            # the good one is unaffected
+
+
+@pytest.mark.parametrize("N,n_blocks,block", [(37, 2, 8), (5003, 64, 8), (16384, 2048, 8),
+                                              (20011, 512, 8), (3000, 100, 1), (9000, 40, 32)])
+def test_hier_blocks_and_reindex(orc, N, n_blocks, block):
+    kv, ik = synth.kv_tokens(60 + N % 97, N, device="cuda")
+    _, ikp, _, o_ik = pools_from_tokens(orc, kv, ik)
+    HI, K = 8, min(512, N)
+    q, w = synth.index_queries(61, 1, 1, HI)
+    q2, w2 = synth.index_queries(62, 1, 1, HI)
+    n_vis = torch.tensor([[N]], dtype=torch.int32)
+    base = torch.zeros(1, dtype=torch.int64)
+    blocks = torch.empty(1, 1, n_blocks, dtype=torch.int32, device="cuda")
+    bscore = torch.empty(1, 1, n_blocks, dtype=torch.float32, device="cuda")
+    st = csa2.status_word()
+    csa2.csa2_index_hier(q.cuda(), w.cuda(), ikp, base.cuda(), n_vis.cuda(), n_blocks, block, N, blocks,
+                         bscore, dev_status=st)
+    o_blocks, _ = orc.index_hier(q.numpy(), w.numpy(), o_ik, base.numpy(), n_vis.numpy(), n_blocks, block)
+    s = orc.index_scores(q[0, 0].numpy(), w[0, 0].numpy(), o_ik[:N])
+    nb = (N + block - 1) // block
+    bs = np.array([s[c * block:min(N, (c + 1) * block)].max() for c in range(nb)])
+    g_blocks = blocks.cpu().numpy()
+    assert_topk_set(g_blocks[0, 0], o_blocks[0, 0], bs, n_blocks, what="blocks")
+    # Reindex over the oracle's blocks (the same pool for both sides) with another query
+    for qq, ww in ((q, w), (q2, w2)):
+        topk = torch.empty(1, 1, K, dtype=torch.int32, device="cuda")
+        csa2.csa2_reindex(qq.cuda(), ww.cuda(), ikp, base.cuda(), n_vis.cuda(),
+                          torch.from_numpy(o_blocks).cuda(), block, K, topk, dev_status=st)
+        o_topk, _ = orc.reindex(qq.numpy(), ww.numpy(), o_ik, base.numpy(), n_vis.numpy(), o_blocks, K,
+                                block=block)
+        s2 = orc.index_scores(qq[0, 0].numpy(), ww[0, 0].numpy(), o_ik[:N])
+        cand = sorted({j for c in o_blocks[0, 0] if c >= 0 for j in range(c * block, min(N, c * block + block))})
+        assert_topk_set(topk.cpu().numpy()[0, 0], o_topk[0, 0], s2[cand], K, labels=cand, what="reindex")
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+
+
+def test_reindex_empty_slots_and_bad_ids(orc):
+    N = 300
+    kv, ik = synth.kv_tokens(70, N, device="cuda")
+    _, ikp, _, o_ik = pools_from_tokens(orc, kv, ik)
+    q, w = synth.index_queries(71, 1, 1, 4)
+    blocks = np.array([[[3, -1, 0, 37, 36, -1, 12, 30]]], np.int32)   # 37*8 >= 300: invisible; 36 ragged
+    topk = torch.empty(1, 1, 20, dtype=torch.int32, device="cuda")
+    st = csa2.status_word()
+    args = (q.cuda(), w.cuda(), ikp, torch.zeros(1, dtype=torch.int64, device="cuda"),
+            torch.tensor([[N]], dtype=torch.int32, device="cuda"))
+    csa2.csa2_reindex(*args, torch.from_numpy(blocks).cuda(), 8, 20, topk, dev_status=st)
+    o_topk, _ = orc.reindex(q.numpy(), w.numpy(), o_ik, np.zeros(1, np.int64), np.array([[N]], np.int32),
+                            blocks, 20)
+    cand = sorted({j for c in blocks[0, 0] if c >= 0 for j in range(c * 8, min(N, c * 8 + 8))})
+    s = orc.index_scores(q[0, 0].numpy(), w[0, 0].numpy(), o_ik[:N])
+    assert_topk_set(topk.cpu().numpy()[0, 0], o_topk[0, 0], s[cand], 20, labels=cand)
+    assert int(st.item()) == 0
+    bad = blocks.copy()
+    bad[0, 0, 1] = -5
+    csa2.csa2_reindex(*args, torch.from_numpy(bad).cuda(), 8, 20, topk, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & csa2.DEV_BAD_INDEX
+
+
+# ---- full-size workloads, launch as timed, sampled queries --------------------------------
+def _full_state(wl, seqs_for_oracle, orc):
+    """Device pools of the whole workload plus the oracle's own pack of some sequences."""
+    lengths = [int(n) for n in wl.lengths]
+    base = np.cumsum([0] + lengths[:-1]).astype(np.int64)
+    P = sum(lengths)
+    ikp = torch.zeros(P, 68, dtype=torch.uint8, device="cuda")
+    kvp = torch.zeros(P, 288, dtype=torch.uint8, device="cuda")
+    o_ik = {}
+    for b in range(wl.B):
+        kv, ik = synth.seq_tokens(wl, b, device="cuda")
+        d = torch.arange(base[b], base[b] + lengths[b], device="cuda")
+        csa2.csa2_pack_kv(kv, ik, wl.ratio, kvp, ikp, dst_entry=d)
+        if b in seqs_for_oracle:
+            _, o_ik[b] = orc.pack_kv(bf16_bits(kv), bf16_bits(ik), wl.ratio)
+            assert np.array_equal(np_u8(ikp[base[b]:base[b] + lengths[b]]), o_ik[b])
+        del kv, ik
+    return kvp, ikp, base, o_ik
+
+
+def test_full128k_sampled(orc):
+    wl = synth.workload("full128k")
+    sample = [0, 13, 31]
+    _, ikp, base, o_ik = _full_state(wl, sample, orc)
+    qd = synth.step_queries(wl)
+    qi, w, n_vis = qd["qi"][0], qd["w"][0], qd["n_vis"]
+    topk, _, st = run_full(qi.cuda(), w.cuda(), ikp, torch.from_numpy(base).cuda(), n_vis.cuda(), 512,
+                           max(wl.lengths))
+    assert st == 0
+    for b in sample:
+        s = orc.index_scores(qi[b, 0].numpy(), w[b, 0].numpy(), o_ik[b][: int(n_vis[b, 0])])
+        o_topk, _ = orc.topk(s, 512)
+        assert_topk_set(topk[b, 0], o_topk, s, 512, what=f"seq {b}")
+
+
+def test_verify_sampled(orc):
+    wl = synth.workload("verify")
+    _, ikp, base, o_ik = _full_state(wl, [5], orc)
+    qd = synth.step_queries(wl)
+    qi, w, n_vis = qd["qi"][0], qd["w"][0], qd["n_vis"]
+    topk, _, st = run_full(qi.cuda(), w.cuda(), ikp, torch.from_numpy(base).cuda(), n_vis.cuda(), 512,
+                           max(wl.lengths))
+    assert st == 0
+    for i in (0, 37, 63):
+        s = orc.index_scores(qi[5, i].numpy(), w[5, i].numpy(), o_ik[5][: int(n_vis[5, i])])
+        o_topk, _ = orc.topk(s, 512)
+        assert_topk_set(topk[5, i], o_topk, s, 512, what=f"query {i}")
+
+
+def test_hier1m_sampled(orc):
+    wl = synth.workload("hier1m")
+    _, ikp, base, o_ik = _full_state(wl, [2], orc)
+    qd = synth.step_queries(wl)
+    qi, w, n_vis = qd["qi"], qd["w"], qd["n_vis"]
+    N = 1 << 20
+    blocks = torch.empty(4, 1, 2048, dtype=torch.int32, device="cuda")
+    st = csa2.status_word()
+    csa2.csa2_index_hier(qi[0].cuda(), w[0].cuda(), ikp, torch.from_numpy(base).cuda(), n_vis.cuda(), 2048, 8,
+                         N, blocks, dev_status=st)
+    s = orc.index_scores(qi[0][2, 0].numpy(), w[0][2, 0].numpy(), o_ik[2])
+    bs = s.reshape(-1, 8).max(axis=1)
+    o_blocks, _ = orc.topk(bs, 2048)
+    g_blocks = blocks.cpu().numpy()
+    assert_topk_set(g_blocks[2, 0], o_blocks, bs, 2048, what="blocks")
+    # Reindex layers 0 (own query) and 1 over the GPU's blocks
+    for l in (0, 1):
+        topk = torch.empty(4, 1, 512, dtype=torch.int32, device="cuda")
+        csa2.csa2_reindex(qi[l].cuda(), w[l].cuda(), ikp, torch.from_numpy(base).cuda(), n_vis.cuda(), blocks, 8,
+                          512, topk, dev_status=st)
+        sl = orc.index_scores(qi[l][2, 0].numpy(), w[l][2, 0].numpy(), o_ik[2])
+        cand = np.sort((g_blocks[2, 0][:, None] * 8 + np.arange(8)[None, :]).reshape(-1))
+        o_topk, _ = orc.topk(sl[cand], 512)
+        o_topk = cand[o_topk]
+        assert_topk_set(topk.cpu().numpy()[2, 0], o_topk, sl[cand], 512, labels=cand, what=f"layer {l}")
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
