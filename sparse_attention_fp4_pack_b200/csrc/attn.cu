@@ -7,21 +7,27 @@
 // P3 (genexis.ai "100만 토큰을 0.9GB에…") §전역 어텐션과 지역 어텐션 — a 128-token window;
 //   §4비트로 적어도 되는 이유 — the window is kept in 8 bits.
 //
-// Split-KV.  A query's key slots are [0, K) for its Top-K entries, then [K, K+window)
-// for window tokens t-window+1 .. t.  One CTA (256 threads) owns 128 consecutive slots:
-//   1. gathers the selected 288 B entries (16 B loads) and dequantises them into a
-//      128 x 512 f16 tile in shared memory (E2M1 -> f16 by cvt, times the E4M3 block
-//      scale; every product is exact in f16), window tokens by E4M3 -> f16 cvt;
-//      empty slots become zero rows;
-//   2. S^T[128 keys x 64 heads] = Kt . Qs^T with tcgen05.mma (M=128, N=64, K=512),
-//      queries pre-scaled by sm_scale*log2(e) so the softmax works in base 2;
-//   3. per-head max / exp2 / sum across the 128 TMEM lanes (warp transpose-reductions),
-//      P^T written to shared memory as f16;
-//   4. O^T[512 dims x 64 heads] = Kt^T . P^T: the same key tile read MN-major as the A
-//      operand (4 MMAs of M=128 per K step) — the latent is both key and value;
-//   5. unnormalised O^T and (m, l) per head go to the workspace; a combine kernel merges
-//      the splits by their log-sum-exp.
-// Heads are padded to 64 (zero query rows) so every MMA has N = 64.
+// A query's key slots are [0, K) for its Top-K entries, then [K, K+window) for window
+// tokens t-window+1 .. t, cut into tiles of 128 slots.  One thread-block cluster of
+// C = min(tiles, 8) CTAs (256 threads each) handles one query; CTA r takes tiles
+// r, r+C, ...:
+//   1. the fp32 queries arrive by one bulk copy into shared memory and become f16
+//      (times sm_scale*log2 e, so the softmax works in base 2), heads padded to 64 with
+//      zero rows; meanwhile each thread gathers its half of a selected 288 B entry;
+//   2. the entries are dequantised into a 128 x 512 f16 tile in 128-byte-swizzled
+//      shared memory (E2M1 -> f16 by cvt times the E4M3 block scale, exact in f16);
+//      window tokens by E4M3 -> f16 cvt; empty slots become zero rows;
+//   3. S^T[128 keys x 64 heads] = Kt . Qs^T by tcgen05.mma (M=128, N=64, K=512) into
+//      tensor memory;
+//   4. per-head max / exp2 / sum across the 128 TMEM lanes by warp transpose
+//      reductions; a running max rescales the accumulated output when a CTA takes more
+//      than one tile; P^T goes to shared memory as f16;
+//   5. O^T[512 dims x 64 heads] += Kt^T . P^T with the same key tile read MN-major as
+//      the A operand (the latent is both key and value);
+//   6. every CTA exports its O^T and (max, sum) per head in shared memory; after a
+//      cluster barrier CTA r merges heads [r*H/C, (r+1)*H/C) of all CTAs through
+//      distributed shared memory and writes the normalised output and log-sum-exp.
+#include <cooperative_groups.h>
 #include <cuda_fp16.h>
 
 #include "csa2_device.cuh"
@@ -29,14 +35,18 @@
 
 namespace csa2 {
 
-constexpr int kTile = 128;        // key slots per CTA = UMMA M
+namespace cg = cooperative_groups;
+
+constexpr int kTile = 128;        // key slots per tile = UMMA M
 constexpr int kHeadsPad = 64;     // UMMA N
 constexpr int kAttnThreads = 256;
+constexpr int kMaxCluster = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;
-constexpr uint32_t kOffK = 0;           // 8 dim-blocks x [128 rows x 128 B]
-constexpr uint32_t kOffQ = 131072;      // 8 dim-blocks x [64 rows x 128 B]
-constexpr uint32_t kOffP = 196608;      // [128 keys x 64 heads] f16
+constexpr uint32_t kOffK = 0;           // keys: 8 dim-blocks x [128 rows x 128 B] f16; also the
+                                        // fp32 query staging and the fp32 O export [64][512]
+constexpr uint32_t kOffQ = 131072;      // queries: 8 dim-blocks x [64 rows x 128 B] f16
+constexpr uint32_t kOffP = 196608;      // P^T: [128 keys x 64 heads] f16
 constexpr uint32_t kOffMisc = 212992;
 constexpr uint32_t kSmemBytes = kOffMisc + 4096 + 1024;  // + alignment slack
 constexpr uint32_t kMaxPolls = 1u << 22;
@@ -55,9 +65,7 @@ struct AttnArgs {
   int window;
   int Q, H;
   float sm_scale;
-  int n_splits;
-  float* part_o;   // [BQ][n_splits][H][512] unnormalised
-  float* part_ml;  // [BQ][n_splits][H][2]  (max in base-2 logit units, sum)
+  int n_tiles, csize;
   float* out;
   float* lse;
   uint32_t* status;
@@ -125,46 +133,26 @@ __device__ __forceinline__ float xpose_reduce(float (&v)[32], int lane) {
   return v[0];
 }
 
-__global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* Ks = sm + kOffK;
-  uint8_t* Qs = sm + kOffQ;
-  uint8_t* Ps = sm + kOffP;
-  float* red_max = reinterpret_cast<float*>(sm + kOffMisc);  // [4][64]
-  float* red_sum = red_max + 256;                           // [4][64]
-  float* m_s = red_sum + 256;                               // [64]
-  float* l_s = m_s + 64;                                    // [64]
-  int* valid_s = reinterpret_cast<int*>(l_s + 64);          // [128]
-  uint64_t* mbar = reinterpret_cast<uint64_t*>(valid_s + 128);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mbar + 1);
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bq = blockIdx.y, split = blockIdx.x;
-  const int b = bq / a.Q;
-  const int H = a.H;
-  const int64_t base = a.seq_base[b];
-  const int64_t t = a.q_pos[bq];
-  const uint32_t mbar_a = tc::smem_u32(mbar);
+// One key slot's raw data for this thread's half of the 512 channels.
+struct SlotRaw {
+  uint4 v[16];
+  uint4 sc;
+  int kind;  // 0 empty, 1 cached entry, 2 window token
+};
 
-  if (warp == 0) tc::tmem_alloc(tc::smem_u32(tmem_slot), kTmemCols);
-  if (tid == 32) tc::mbar_init(mbar_a, 1);
-
-  // Issue the key gather first so its latency overlaps the query loads.
-  const int r = tid >> 1, hf = tid & 1;
-  const int slot = split * kTile + r;
-  int kind = 0;  // 0 empty, 1 cached entry, 2 window token
-  uint4 kraw[16];
-  uint4 ksc = make_uint4(0u, 0u, 0u, 0u);
+__device__ __forceinline__ void gather_slot(const AttnArgs& a, int bq, int b, int64_t base, int64_t t, int slot,
+                                            int hf, SlotRaw& s) {
+  s.kind = 0;
   if (slot < a.K) {
     const int32_t j = a.topk[(int64_t)bq * a.K + slot];
     if (j >= 0) {
       if (base >= 0 && base + j < a.pool_entries) {
         const uint4* e = reinterpret_cast<const uint4*>(a.kv_pool + (base + j) * kKvBytes);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) kraw[i] = e[hf * 8 + i];
-        ksc = e[16 + hf];
-        kind = 1;
+        for (int i = 0; i < 8; ++i) s.v[i] = e[hf * 8 + i];
+        s.sc = e[16 + hf];
+        s.kind = 1;
       } else if (hf == 0) {
         flag(a.status, CSA2_DEV_BAD_INDEX);
       }
@@ -175,101 +163,157 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
     if (u >= 0 && row >= 0 && row < a.S_w) {
       const uint4* src = reinterpret_cast<const uint4*>(a.swa + ((int64_t)b * a.S_w + row) * kD + hf * 256);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) kraw[i] = src[i];
-      kind = 2;
+      for (int i = 0; i < 16; ++i) s.v[i] = src[i];
+      s.kind = 2;
     }
   }
+}
 
-  // ---- queries: f16(q * sm_scale * log2 e), rows >= H are zero ---------------------------
-  // thread -> (head row tid/4, quarter tid%4 = 128 channels), two batches of 16 x 16 B
-  const float qscale = a.sm_scale * 1.4426950408889634f;
-  {
-    const int h = tid >> 2, qq = tid & 3;
-    const float4* src = reinterpret_cast<const float4*>(a.q + ((int64_t)bq * H + h) * kD + qq * 128);
-#pragma unroll
-    for (int bt = 0; bt < 2; ++bt) {
-      float4 x[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) x[i] = h < H ? src[bt * 16 + i] : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {  // 8 chunks of 8 channels
-        const float4 x0 = x[2 * i], x1 = x[2 * i + 1];
-        uint4 v;
-        v.x = half2_bits(x0.x * qscale, x0.y * qscale);
-        v.y = half2_bits(x0.z * qscale, x0.w * qscale);
-        v.z = half2_bits(x1.x * qscale, x1.y * qscale);
-        v.w = half2_bits(x1.z * qscale, x1.w * qscale);
-        const int ch = qq * 16 + bt * 8 + i, db = ch >> 3, c = ch & 7;
-        *reinterpret_cast<uint4*>(Qs + db * 8192 + tc::sw128(h, c * 16)) = v;
-      }
-    }
-  }
-
-  // ---- keys: two threads per slot, each dequantises 256 of the 512 channels -------------
-  const bool ok = kind != 0;
-  if (kind == 1) {
-    const uint32_t scw[4] = {ksc.x, ksc.y, ksc.z, ksc.w};
+// Dequantise this thread's half row (256 channels) of tile row r into the key tile.
+__device__ __forceinline__ void store_slot(uint8_t* Ks, int r, int hf, const SlotRaw& s) {
+  if (s.kind == 1) {
+    const uint32_t scw[4] = {s.sc.x, s.sc.y, s.sc.z, s.sc.w};
 #pragma unroll
     for (int dl = 0; dl < 4; ++dl) {
       uint8_t* blk = Ks + (4 * hf + dl) * 16384;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const uint4 q4 = kraw[2 * dl + (c >> 2)];
+        const uint4 q4 = s.v[2 * dl + (c >> 2)];
         const uint32_t wcode = (c & 3) == 0 ? q4.x : (c & 3) == 1 ? q4.y : (c & 3) == 2 ? q4.z : q4.w;
         const int sidx = dl * 4 + (c >> 1);  // block scale index within this half (0..15)
         const uint32_t sbyte = (scw[sidx >> 2] >> (8 * (sidx & 3))) & 0xFFu;
         *reinterpret_cast<uint4*>(blk + tc::sw128(r, c * 16)) = e2m1x8_to_f16(wcode, e4m3_scale_f16x2(sbyte));
       }
     }
-  } else if (kind == 2) {
+  } else if (s.kind == 2) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) {  // 16 channels per load: chunks 2i, 2i+1 of this half
-      const int ch = 2 * i;         // chunk of 8 channels within this half's 32 chunks
+      const int ch = 2 * i;
       uint8_t* blk = Ks + (4 * hf + (ch >> 3)) * 16384;
-      const uint2 a0 = e4m3x4_to_f16(kraw[i].x), a1 = e4m3x4_to_f16(kraw[i].y);
-      const uint2 a2 = e4m3x4_to_f16(kraw[i].z), a3 = e4m3x4_to_f16(kraw[i].w);
+      const uint2 a0 = e4m3x4_to_f16(s.v[i].x), a1 = e4m3x4_to_f16(s.v[i].y);
+      const uint2 a2 = e4m3x4_to_f16(s.v[i].z), a3 = e4m3x4_to_f16(s.v[i].w);
       *reinterpret_cast<uint4*>(blk + tc::sw128(r, (ch & 7) * 16)) = make_uint4(a0.x, a0.y, a1.x, a1.y);
       *reinterpret_cast<uint4*>(blk + tc::sw128(r, ((ch + 1) & 7) * 16)) = make_uint4(a2.x, a2.y, a3.x, a3.y);
     }
-  }
-  if (!ok) {
+  } else {
 #pragma unroll
     for (int dl = 0; dl < 4; ++dl)
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         *reinterpret_cast<uint4*>(Ks + (4 * hf + dl) * 16384 + tc::sw128(r, c * 16)) = make_uint4(0u, 0u, 0u, 0u);
   }
-  if (hf == 0) valid_s[r] = ok ? 1 : 0;
+}
 
-  tc::fence_async_smem();
+__global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* Ks = sm + kOffK;
+  uint8_t* Qs = sm + kOffQ;
+  uint8_t* Ps = sm + kOffP;
+  float* red_max = reinterpret_cast<float*>(sm + kOffMisc);  // [4][64]
+  float* red_sum = red_max + 256;                           // [4][64]
+  float* m_run = red_sum + 256;                             // [64] running max (base-2 logits)
+  float* l_run = m_run + 64;                                // [64] running sum
+  float* alpha = l_run + 64;                                // [64] rescale of this tile
+  int* valid_s = reinterpret_cast<int*>(alpha + 64);        // [128]
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(valid_s + 128);  // [0] MMA completion, [1] query copy
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mbar + 2);
+  float* Of = reinterpret_cast<float*>(Ks);                 // export [64][512] fp32
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rank = (int)cluster.block_rank();
+  const int C = a.csize;
+  const int bq = blockIdx.y;
+  const int b = bq / a.Q;
+  const int H = a.H;
+  const int64_t base = a.seq_base[b];
+  const int64_t t = a.q_pos[bq];
+  const uint32_t mbar_mma = tc::smem_u32(&mbar[0]), mbar_q = tc::smem_u32(&mbar[1]);
+
+  // Start every global read before any set-up barrier: thread 0 initialises the query
+  // barrier and issues the bulk copy of the fp32 queries into the key area, every thread
+  // gathers its half of its first key slot, then warp 0 allocates tensor memory.
+  if (tid == 0) {
+    tc::mbar_init(mbar_mma, 1);
+    tc::mbar_init(mbar_q, 1);
+    const uint32_t bytes = (uint32_t)H * kD * 4;
+    tc::mbar_arrive_expect_tx(mbar_q, bytes);
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(a.q + (int64_t)bq * H * kD);
+    for (uint32_t off = 0; off < bytes; off += 32768)
+      tc::bulk_g2s(tc::smem_u32(Ks) + off, src + off, bytes - off < 32768 ? bytes - off : 32768, mbar_q);
+  }
+  const int r = tid >> 1, hf = tid & 1;
+  const int my_tiles = rank < a.n_tiles ? (a.n_tiles - 1 - rank) / C + 1 : 0;
+  SlotRaw sr;
+  sr.kind = 0;
+  if (my_tiles > 0) gather_slot(a, bq, b, base, t, rank * kTile + r, hf, sr);
+  // phase: gather issued
+  if (warp == 0) tc::tmem_alloc(tc::smem_u32(tmem_slot), kTmemCols);
+  if (tid < kHeadsPad) {
+    m_run[tid] = -INFINITY;
+    l_run[tid] = 0.0f;
+  }
   tc::fence_before_sync();
-  const int any_valid = __syncthreads_or(ok ? 1 : 0);
+  __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const int64_t pbase = ((int64_t)bq * a.n_splits + split) * H;
+  // phase: setup
+  bool timed_out = __syncthreads_or(tc::mbar_wait(mbar_q, 0, kMaxPolls) ? 0 : 1) != 0;
+  // phase: queries landed
+  {  // fp32 staging -> f16 query tile (scaled), 8 channels per 16 B chunk
+    const float qscale = a.sm_scale * 1.4426950408889634f;
+    for (int i = tid; i < kHeadsPad * 64; i += kAttnThreads) {
+      const int h = i >> 6, ch = i & 63, db = ch >> 3, c = ch & 7;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (h < H && !timed_out) {
+        const float4 x0 = *reinterpret_cast<const float4*>(Of + h * kD + ch * 8);
+        const float4 x1 = *reinterpret_cast<const float4*>(Of + h * kD + ch * 8 + 4);
+        v.x = half2_bits(x0.x * qscale, x0.y * qscale);
+        v.y = half2_bits(x0.z * qscale, x0.w * qscale);
+        v.z = half2_bits(x1.x * qscale, x1.y * qscale);
+        v.w = half2_bits(x1.z * qscale, x1.w * qscale);
+      }
+      *reinterpret_cast<uint4*>(Qs + db * 8192 + tc::sw128(h, c * 16)) = v;
+    }
+  }
+  __syncthreads();  // staging consumed: the key area is free
+  // phase: queries converted
 
-  bool timed_out = false;
-  if (any_valid) {
-    // ---- S^T = Kt . Qs^T ----------------------------------------------------------------
+  const int q4 = warp & 3, half = warp >> 2;
+  const int key = q4 * 32 + lane;
+  const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
+  uint32_t commits = 0;
+  int processed = 0;
+  for (int it = 0; it < my_tiles && !timed_out; ++it) {
+    if (it > 0) gather_slot(a, bq, b, base, t, (rank + it * C) * kTile + r, hf, sr);
+    store_slot(Ks, r, hf, sr);
+    if (hf == 0) valid_s[r] = sr.kind != 0;
+    tc::fence_async_smem();
+    tc::fence_before_sync();
+    const int any_valid = __syncthreads_or(sr.kind != 0);
+    tc::fence_after_sync();
+  // phase: keys stored
+    if (!any_valid) continue;
+    // ---- S^T = Kt . Qs^T --------------------------------------------------------------------
     if (tid == 0) {
       constexpr uint32_t idesc = tc::idesc_f16(kTile, kHeadsPad, false, false);
-#pragma unroll 1
+#pragma unroll 4
       for (int ks = 0; ks < kD / 16; ++ks) {
         const int db = ks >> 2, kk = ks & 3;
         const uint64_t ad = tc::smem_desc_sw128(tc::smem_u32(Ks + db * 16384 + kk * 32), 16, 1024);
         const uint64_t bd = tc::smem_desc_sw128(tc::smem_u32(Qs + db * 8192 + kk * 32), 16, 1024);
         tc::mma_f16(tmem + kColS, ad, bd, idesc, ks > 0 ? 1u : 0u);
       }
-      tc::commit(mbar_a);
+      tc::commit(mbar_mma);
     }
-    timed_out = __syncthreads_or(tc::mbar_wait(mbar_a, 0, kMaxPolls) ? 0 : 1) != 0;
+    timed_out = __syncthreads_or(tc::mbar_wait(mbar_mma, commits & 1, kMaxPolls) ? 0 : 1) != 0;
+    ++commits;
     tc::fence_after_sync();
-  }
-  if (any_valid && !timed_out) {
-    const int q4 = warp & 3, half = warp >> 2;
-    const int key = q4 * 32 + lane;
+    if (timed_out) break;
+  // phase: qk done
     uint32_t raw[32];
-    tc::tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + kColS + half * 32, raw);
+    tc::tmem_ld32(lane_base + kColS + half * 32, raw);
     const bool kv = valid_s[key] != 0;
     float s[32], v[32];
 #pragma unroll
@@ -279,13 +323,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
     }
     red_max[q4 * 64 + half * 32 + lane] = xpose_reduce<true>(v, lane);
     __syncthreads();
-    if (tid < kHeadsPad)
-      m_s[tid] = fmaxf(fmaxf(red_max[tid], red_max[64 + tid]), fmaxf(red_max[128 + tid], red_max[192 + tid]));
+    if (tid < kHeadsPad) {
+      const float mt = fmaxf(fmaxf(red_max[tid], red_max[64 + tid]), fmaxf(red_max[128 + tid], red_max[192 + tid]));
+      const float mo = m_run[tid];
+      const float mn = fmaxf(mo, mt);
+      alpha[tid] = mo == -INFINITY ? 0.0f : exp2f(mo - mn);
+      m_run[tid] = mn;
+    }
     __syncthreads();
+    if (processed > 0) {  // rescale the output accumulated from earlier tiles
+#pragma unroll 1
+      for (int mt = 0; mt < 4; ++mt) {
+        uint32_t o[32];
+        const uint32_t ta = lane_base + kColO + mt * 64 + half * 32;
+        tc::tmem_ld32(ta, o);
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) o[jj] = __float_as_uint(__uint_as_float(o[jj]) * alpha[half * 32 + jj]);
+        tc::tmem_st32(ta, o);
+      }
+    }
     uint32_t ph[16];
 #pragma unroll
     for (int jj = 0; jj < 32; jj += 2) {
-      const float m0 = m_s[half * 32 + jj], m1 = m_s[half * 32 + jj + 1];
+      const float m0 = m_run[half * 32 + jj], m1 = m_run[half * 32 + jj + 1];
       const float p0 = m0 == -INFINITY ? 0.0f : exp2f(s[jj] - m0);
       const float p1 = m1 == -INFINITY ? 0.0f : exp2f(s[jj + 1] - m1);
       __half2 hp = __floats2half2_rn(p0, p1);
@@ -299,91 +359,121 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
       *reinterpret_cast<uint4*>(Ps + tc::sw128(key, half * 64 + c * 16)) =
           make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
     red_sum[q4 * 64 + half * 32 + lane] = xpose_reduce<false>(v, lane);
+  // phase: softmax done
     tc::fence_async_smem();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    // ---- O^T = Kt^T . P^T (key tile read MN-major) ---------------------------------------
+    // ---- O^T += Kt^T . P^T (key tile read MN-major) --------------------------------------
     if (tid == 0) {
       constexpr uint32_t idesc = tc::idesc_f16(kTile, kHeadsPad, true, true);
 #pragma unroll 1
       for (int mt = 0; mt < 4; ++mt)
-#pragma unroll 1
+#pragma unroll 4
         for (int ks = 0; ks < kTile / 16; ++ks) {
           const uint64_t ad = tc::smem_desc_sw128(tc::smem_u32(Ks + (2 * mt) * 16384 + ks * 2048), 16384, 1024);
           const uint64_t bd = tc::smem_desc_sw128(tc::smem_u32(Ps + ks * 2048), 8192, 1024);
-          tc::mma_f16(tmem + kColO + mt * 64, ad, bd, idesc, ks > 0 ? 1u : 0u);
+          tc::mma_f16(tmem + kColO + mt * 64, ad, bd, idesc, (ks > 0 || processed > 0) ? 1u : 0u);
         }
-      tc::commit(mbar_a);
+      tc::commit(mbar_mma);
     }
     if (tid < kHeadsPad)
-      l_s[tid] = (red_sum[tid] + red_sum[64 + tid]) + (red_sum[128 + tid] + red_sum[192 + tid]);
-    timed_out = __syncthreads_or(tc::mbar_wait(mbar_a, 1, kMaxPolls) ? 0 : 1) != 0;
+      l_run[tid] = l_run[tid] * alpha[tid] + ((red_sum[tid] + red_sum[64 + tid]) + (red_sum[128 + tid] + red_sum[192 + tid]));
+    timed_out = __syncthreads_or(tc::mbar_wait(mbar_mma, commits & 1, kMaxPolls) ? 0 : 1) != 0;
+    ++commits;
     tc::fence_after_sync();
-    if (!timed_out) {
-#pragma unroll 1
-      for (int mt = 0; mt < 4; ++mt) {
-        tc::tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + kColO + mt * 64 + half * 32, raw);
-        const int d = mt * 128 + q4 * 32 + lane;
-#pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const int h = half * 32 + jj;
-          if (h < H) a.part_o[(pbase + h) * kD + d] = __uint_as_float(raw[jj]);
-        }
-      }
-      if (tid < H) {
-        a.part_ml[(pbase + tid) * 2] = m_s[tid];
-        a.part_ml[(pbase + tid) * 2 + 1] = l_s[tid];
-      }
-    }
-  }
-  if (!any_valid && tid < H) {
-    a.part_ml[(pbase + tid) * 2] = -INFINITY;
-    a.part_ml[(pbase + tid) * 2 + 1] = 0.0f;
+    ++processed;
+  // phase: pv done
   }
   if (timed_out) {
     if (tid == 0) flag(a.status, CSA2_DEV_TIMEOUT);
-    if (tid < H) a.part_ml[(pbase + tid) * 2 + 1] = 0.0f;
-    tc::mbar_wait(mbar_a, 1, kMaxPolls);  // let any MMA still in flight drain (bounded)
+    if (tid < kHeadsPad) l_run[tid] = 0.0f;  // contribute nothing
+  }
+
+  // ---- export O^T (fp32 [head][channel]) into the key area --------------------------------
+  if (processed > 0 && !timed_out) {
+#pragma unroll 1
+    for (int mt = 0; mt < 4; ++mt) {
+      uint32_t o[32];
+      tc::tmem_ld32(lane_base + kColO + mt * 64 + half * 32, o);
+      const int d = mt * 128 + q4 * 32 + lane;
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) Of[(half * 32 + jj) * kD + d] = __uint_as_float(o[jj]);
+    }
   }
   tc::fence_before_sync();
+  cluster.sync();
+
+  // phase: exported
+  // ---- merge heads [h0, h1) across the cluster through distributed shared memory ----------
+  // Remote loads are issued together (unrolled over the largest cluster), since each one
+  // pays the cluster interconnect latency.
+  const int hpc = (H + C - 1) / C;
+  const int h0 = rank * hpc, h1 = h0 + hpc < H ? h0 + hpc : H;
+  // the P^T tile is free once the last PV product has completed
+  float* fac = reinterpret_cast<float*>(Ps);  // [kMaxCluster][64] merge factor of each CTA's partial
+  float* linv = fac + kMaxCluster * 64;       // [64] 1 / merged sum
+  if (tid < h1 - h0) {
+    const int hh = h0 + tid;
+    float mr[kMaxCluster], lr[kMaxCluster];
+#pragma unroll
+    for (int c = 0; c < kMaxCluster; ++c) {
+      mr[c] = c < C ? cluster.map_shared_rank(m_run, c)[hh] : -INFINITY;
+      lr[c] = c < C ? cluster.map_shared_rank(l_run, c)[hh] : 0.0f;
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kMaxCluster; ++c)
+      if (lr[c] > 0.0f) M = fmaxf(M, mr[c]);
+    float L = 0.0f;
+#pragma unroll
+    for (int c = 0; c < kMaxCluster; ++c) {
+      const float f = (lr[c] > 0.0f) ? exp2f(mr[c] - M) : 0.0f;
+      fac[c * 64 + tid] = f;
+      L = fmaf(lr[c], f, L);
+    }
+    linv[tid] = L > 0.0f ? 1.0f / L : 0.0f;
+    a.lse[(int64_t)bq * H + hh] = L > 0.0f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+  }
   __syncthreads();
+  // thread -> (float4 column d4, 2 heads per pass); every CTA's float4 is loaded before use
+  const int d4 = tid & 127;
+  for (int hl = tid >> 7; hl < h1 - h0; hl += 2) {
+    const int hh = h0 + hl;
+    float4 o[kMaxCluster];
+#pragma unroll
+    for (int c = 0; c < kMaxCluster; ++c)
+      o[c] = (c < C && fac[c * 64 + hl] > 0.0f)
+                 ? reinterpret_cast<const float4*>(cluster.map_shared_rank(Of, c) + hh * kD)[d4]
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < kMaxCluster; ++c) {
+      const float f = c < C ? fac[c * 64 + hl] : 0.0f;
+      acc.x = fmaf(o[c].x, f, acc.x);
+      acc.y = fmaf(o[c].y, f, acc.y);
+      acc.z = fmaf(o[c].z, f, acc.z);
+      acc.w = fmaf(o[c].w, f, acc.w);
+    }
+    const float inv = linv[hl];
+    reinterpret_cast<float4*>(a.out + ((int64_t)bq * H + hh) * kD)[d4] =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  }
+  cluster.sync();  // remote reads finished before any CTA releases its shared memory
+  // phase: merged
   if (warp == 0) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
 }
 
-// Merge the split partials of one query: grid (H, BQ), one thread per channel.
-__global__ void __launch_bounds__(kD) attn_combine_kernel(AttnArgs a) {
-  const int h = blockIdx.x, bq = blockIdx.y, c = threadIdx.x;
-  const int H = a.H;
-  float M = -INFINITY;
-  for (int s = 0; s < a.n_splits; ++s) {
-    const int64_t p = ((int64_t)bq * a.n_splits + s) * H + h;
-    if (a.part_ml[p * 2 + 1] > 0.0f) M = fmaxf(M, a.part_ml[p * 2]);
-  }
-  float L = 0.0f, o = 0.0f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < a.n_splits; ++s) {
-      const int64_t p = ((int64_t)bq * a.n_splits + s) * H + h;
-      const float l = a.part_ml[p * 2 + 1];
-      if (l > 0.0f) {
-        const float f = exp2f(a.part_ml[p * 2] - M);
-        L = fmaf(l, f, L);
-        o = fmaf(a.part_o[p * kD + c], f, o);
-      }
-    }
-  }
-  const int64_t oi = ((int64_t)bq * H + h);
-  a.out[oi * kD + c] = L > 0.0f ? o / L : 0.0f;
-  if (c == 0) a.lse[oi] = L > 0.0f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
-}
-
 size_t attn_workspace_bytes(int B, int Q, int H, int K, int window) {
-  const int64_t n_splits = (K + window + kTile - 1) / kTile;
-  const int64_t BQ = (int64_t)B * Q;
-  return (size_t)(BQ * n_splits * H * (kD + 2) * sizeof(float));
+  (void)B;
+  (void)Q;
+  (void)H;
+  (void)K;
+  (void)window;
+  return 0;  // partial results stay in distributed shared memory
 }
 
 cudaError_t launch_sparse_attn(const float* q, const uint8_t* kv_pool, int64_t pool_entries,
@@ -392,6 +482,7 @@ cudaError_t launch_sparse_attn(const float* q, const uint8_t* kv_pool, int64_t p
                                const int64_t* q_pos, int window, int B, int Q, int H,
                                float sm_scale, float* out, float* lse, void* ws,
                                uint32_t* status, cudaStream_t stream) {
+  (void)ws;
   AttnArgs a;
   a.q = q;
   a.kv_pool = kv_pool;
@@ -407,23 +498,29 @@ cudaError_t launch_sparse_attn(const float* q, const uint8_t* kv_pool, int64_t p
   a.Q = Q;
   a.H = H;
   a.sm_scale = sm_scale;
-  a.n_splits = (K + a.window + kTile - 1) / kTile;
-  const int64_t BQ = (int64_t)B * Q;
-  a.part_o = static_cast<float*>(ws);
-  a.part_ml = a.part_o + BQ * a.n_splits * H * kD;
+  a.n_tiles = (K + a.window + kTile - 1) / kTile;
+  a.csize = a.n_tiles < 1 ? 1 : (a.n_tiles > kMaxCluster ? kMaxCluster : a.n_tiles);
   a.out = out;
   a.lse = lse;
   a.status = status;
+  const int64_t BQ = (int64_t)B * Q;
   if (BQ == 0) return cudaSuccess;
-  if (a.n_splits > 0) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attn_tc_kernel<<<dim3(a.n_splits, (unsigned)BQ), kAttnThreads, kSmemBytes, stream>>>(a);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  attn_combine_kernel<<<dim3(H, (unsigned)BQ), kD, 0, stream>>>(a);
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)a.csize, (unsigned)BQ);
+  cfg.blockDim = dim3(kAttnThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)a.csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -30,6 +30,8 @@
 // uint32 key (hierarchical mode: the max over `block` neighbouring lanes).  A CTA takes
 // a group of up to G queries of one sequence (multi-query verify), so the A operand is
 // built once for the group.
+#include <cooperative_groups.h>
+
 #include "csa2_device.cuh"
 #include "tc.cuh"
 
@@ -131,9 +133,8 @@ __global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
   const int64_t left_tiles = (limit - item0 + kRows - 1) / kRows;
   const int ntiles = (int)(left_tiles < a.tiles_per_cta ? left_tiles : a.tiles_per_cta);
 
-  if (warp == 0) tc::tmem_alloc(tc::smem_u32(tmem_slot), a.tmem_cols);
-  if (tid == 32) tc::mbar_init(tc::smem_u32(mbar), 1);
   if (tid < G) nq[tid] = valid_count(a, b, b * a.Q + q0 + tid, blockIdx.x == 0);
+  const int64_t nq0 = valid_count(a, b, b * a.Q + q0, false);  // reindex: the single query's count
 
   const uint8_t* seq = a.ik_pool + base * kIkBytes;
   const int mis = (int)((reinterpret_cast<uintptr_t>(seq)) & 15u);  // same for every tile
@@ -159,7 +160,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
       }
       int cnt = 0;
       if (c >= 0) {
-        const int64_t rem = nq[0] - (int64_t)c * a.block;
+        const int64_t rem = nq0 - (int64_t)c * a.block;
         cnt = rem <= 0 ? 0 : (int)(rem < a.block ? rem : a.block);
       }
       if (cnt > 0) {
@@ -171,6 +172,10 @@ __global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
     }
     tc::cp_async_commit();
   };
+
+  load_tile(0);  // the first tile's copies overlap the set-up below
+  if (warp == 0) tc::tmem_alloc(tc::smem_u32(tmem_slot), a.tmem_cols);
+  if (tid == 32) tc::mbar_init(tc::smem_u32(mbar), 1);
 
   // ---- B operand: four int8 limbs of every (query, head), plus epilogue constants ---------
   for (int gh = warp; gh < a.G * HIPAD; gh += kScanThreads / 32) {
@@ -221,8 +226,6 @@ __global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
     if (lane == 0) wq[gh] = S > 0.f ? wv / (2.0f * S) : 0.f;
   }
 
-  __syncthreads();  // nq visible to every thread before the first gather
-  load_tile(0);
   tc::fence_async_smem();
   tc::fence_before_sync();
   __syncthreads();
@@ -251,7 +254,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
       const int s = tid / a.block, r = tid % a.block;
       const int32_t c = segc[(ti & 1) * 128 + s];
       j = (int64_t)c * a.block + r;
-      valid = c >= 0 && j < nq[0];
+      valid = c >= 0 && j < nq0;
       const int smis = c >= 0 ? (int)(reinterpret_cast<uintptr_t>(seq + (int64_t)c * a.block * kIkBytes) & 15u) : 0;
       ent = rbuf + s * seg_stride + smis + r * kIkBytes;
     }
@@ -328,32 +331,37 @@ __global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
 }
 
 // ------------------------------------------------------------------------------------
-// Top-K selection over one query's keys (one CTA of 1024 threads per query).
+// Top-K selection over one query's keys: a thread-block cluster of C CTAs (C <= 8) per
+// query, each holding a contiguous slice of the keys in registers (512 threads x 32 keys,
+// index order = thread order).
 //
-// Most-significant-digit radix select with digits of 11, 11 and 10 bits:
-//   1. histogram the current digit of every key that matches the prefix chosen so far
-//      (the first pass sees all keys) and find the bin T holding the need-th largest;
-//      keys in bins above T are selected, need shrinks by their number;
-//   2. as soon as bin T holds at most kCap keys, one ordered pass over the keys writes
-//      the selected ones to the output in index order and copies bin T's keys (with their
-//      indices, in index order) into shared memory, where the remaining digits are
-//      resolved without touching global memory again;
-//   3. keys equal to the K-th key are taken lowest index first.
-// Every output position comes from a block-wide prefix sum, so the result (contents and
-// order) is deterministic.
+// Most-significant-digit radix select with adaptive digit windows:
+//   0. the cluster reduces min / max / count of the valid (non-zero) keys; bits above the
+//      highest bit where min and max differ are common to every key, so the first
+//      11-bit digit starts right below them (keys spread over the histogram instead of
+//      piling into a few bins);
+//   1. per level: each CTA histograms the digit of the keys matching the prefix chosen
+//      so far, the histograms are summed across the cluster through distributed shared
+//      memory, and the bin holding the need-th largest key is fixed (the same in every
+//      CTA); keys in higher bins are selected;
+//   2. one ordered pass writes the selected keys in index order — positions come from
+//      block-wide prefix sums plus a prefix over the cluster's CTAs — and the keys equal
+//      to the K-th (all bits resolved) lowest index first.
+// The result (contents and order) is deterministic.
 // ------------------------------------------------------------------------------------
-constexpr int kSelThreads = 1024;
+constexpr int kSelThreads = 512;
+constexpr int kPer = 32;                         // keys per thread per register chunk
+constexpr int kSelChunk = kSelThreads * kPer;    // keys per CTA per chunk (16384)
 constexpr int kBins = 2048;
-constexpr int kCap = 8192;          // shared-memory candidates
-constexpr int kPer = 16;            // keys per thread per tile (4 x 16 B loads in flight)
-constexpr int kSelSmem = kBins * 4 + kCap * 8 + 34 * 4 + 64;
-static_assert(kSelThreads * kPer <= 65535, "packed 16-bit tile counts");
+constexpr int kMaxCluster = 8;
+constexpr int kSelSmem = 2 * kBins * 4 + 64 * 4 + 64 * 4;
 
 struct SelectArgs {
   const uint32_t* keys;
   int64_t key_stride;
   int mode;
   int Q, block, n_blocks, K;
+  int csize;                 // CTAs per query (cluster size)
   const int64_t* seq_base;
   const int32_t* n_vis;
   int64_t max_n_vis, pool_entries;
@@ -370,75 +378,58 @@ __device__ __forceinline__ int64_t item_label(const SelectArgs& a, int bq, int64
   return i;
 }
 
-// Block-wide exclusive prefix sum of one uint32 per thread (1024 threads); *total gets
-// the sum.  ws must hold 33 words.
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* ws, uint32_t* total) {
+// Block-wide exclusive prefix sum of one value per thread (kSelThreads threads) of a
+// 64-bit packed pair; ws holds kSelThreads/32 + 1 entries.
+__device__ __forceinline__ uint64_t block_excl_scan64(uint64_t v, uint64_t* ws, uint64_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t x = v;
+  constexpr int nw = kSelThreads / 32;
+  uint64_t x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
   if (lane == 31) ws[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    const uint32_t w = ws[lane];
-    uint32_t z = w;
+    const uint64_t w = lane < nw ? ws[lane] : 0ull;
+    uint64_t z = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, z, o);
+      const uint64_t y = __shfl_up_sync(0xffffffffu, z, o);
       if (lane >= o) z += y;
     }
-    ws[lane] = z - w;
-    if (lane == 31) ws[32] = z;
+    if (lane < nw) ws[lane] = z - w;
+    if (lane == nw - 1) ws[nw] = z;
   }
   __syncthreads();
-  const uint32_t r = ws[warp] + x - v;
-  *total = ws[32];
+  const uint64_t r = ws[warp] + x - v;
+  *total = ws[nw];
   __syncthreads();
   return r;
 }
 
-// Load keys [i0, i0+kPer) (zero past n); rows are 16-byte aligned and i0 % 4 == 0.
-__device__ __forceinline__ void load_keys(const uint32_t* keys, int64_t i0, int64_t n, uint32_t (&k)[kPer]) {
-  if (i0 + kPer <= n) {
-#pragma unroll
-    for (int v = 0; v < kPer / 4; ++v) {
-      const uint4 a4 = *reinterpret_cast<const uint4*>(keys + i0 + 4 * v);
-      k[4 * v] = a4.x;
-      k[4 * v + 1] = a4.y;
-      k[4 * v + 2] = a4.z;
-      k[4 * v + 3] = a4.w;
-    }
-  } else {
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) k[e] = (i0 + e < n) ? keys[i0 + e] : 0u;
-  }
-}
-
-// Find the bin T of hist[0, nb) holding the need-th largest counted key.  Executed by
-// warp 0; results in *T_out / *above_out (keys in bins above T).  Also returns the total.
+// Bin of hist[0, nb) holding the need-th largest counted key, by the whole block: each
+// thread sums a run of nb/kSelThreads bins, a block-wide prefix over the runs from the
+// top finds the run, and its thread walks it.  ws: scan scratch (kSelThreads/32 + 1).
 __device__ __forceinline__ void find_bin(const uint32_t* hist, int nb, uint32_t need, uint32_t* T_out,
-                                         uint32_t* above_out, uint32_t* total_out) {
-  const int lane = threadIdx.x & 31;
-  const int per = nb / 32;
+                                         uint32_t* above_out, uint64_t* ws) {
+  const int tid = threadIdx.x;
+  const int per = nb >= kSelThreads ? nb / kSelThreads : 1;
+  // runs are numbered from the top bins down, so an exclusive prefix counts keys above
+  const int run_id = tid;
+  const int top = nb - 1 - run_id * per;  // highest bin of this run
   uint32_t run = 0;
-  for (int i = 0; i < per; ++i) run += hist[lane * per + i];
-  uint32_t suf = run;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_down_sync(0xffffffffu, suf, o);
-    if (lane + o < 32) suf += y;
-  }
-  const uint32_t above_lane = suf - run;
-  if (lane == 0) *total_out = suf;
-  if (above_lane < need && suf >= need) {
-    uint32_t acc = above_lane;
-    for (int i = per - 1; i >= 0; --i) {
-      const uint32_t h = hist[lane * per + i];
+  if (top >= 0)
+    for (int i = 0; i < per; ++i) run += hist[top - i];
+  uint64_t total;
+  const uint32_t above = (uint32_t)block_excl_scan64(run, ws, &total);
+  if (top >= 0 && above < need && above + run >= need) {
+    uint32_t acc = above;
+    for (int i = 0; i < per; ++i) {
+      const uint32_t h = hist[top - i];
       if (acc + h >= need) {
-        *T_out = lane * per + i;
+        *T_out = top - i;
         *above_out = acc;
         break;
       }
@@ -448,15 +439,19 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, int nb, uint32_t 
 }
 
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ __align__(16) uint32_t sel_smem[];
-  uint32_t* hist = sel_smem;                  // [kBins]
-  uint32_t* cand_key = hist + kBins;          // [kCap]
-  uint32_t* cand_idx = cand_key + kCap;       // [kCap]
-  uint32_t* scan_ws = cand_idx + kCap;        // [33]
-  uint32_t* s_misc = scan_ws + 34;            // T, above, total
+  uint32_t* hist = sel_smem;                 // [kBins] this CTA's histogram
+  uint32_t* hsum = hist + kBins;             // [kBins] cluster-summed histogram
+  uint64_t* scan_ws = reinterpret_cast<uint64_t*>(hsum + kBins);  // [17]
+  uint32_t* xch = reinterpret_cast<uint32_t*>(scan_ws + 32);       // [16] values exported to the cluster
+  uint32_t* misc = xch + 16;                                        // [8]
 
   const int tid = threadIdx.x;
-  const int bq = blockIdx.x;
+  const int rank = (int)cluster.block_rank();
+  const int C = a.csize;
+  const int bq = blockIdx.y;
   const int b = bq / a.Q;
   const int K = a.K;
   int32_t* out = a.out_idx + (int64_t)bq * K;
@@ -475,150 +470,212 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
       n = (int64_t)a.n_blocks * a.block;
   }
   const uint32_t* keys = a.keys + (int64_t)bq * a.key_stride;
+  // this CTA's slice [lo, hi), a multiple of 4 keys so rows stay 16-byte aligned
+  const int64_t slice = (((n + C - 1) / C) + 3) & ~int64_t(3);
+  const int64_t lo = (int64_t)rank * slice;
+  const int64_t hi = lo + slice < n ? lo + slice : n;
+  const int nchunks = hi > lo ? (int)((hi - lo + kSelChunk - 1) / kSelChunk) : 0;
 
-  auto emit = [&](int pos, int64_t i, uint32_t k) {
-    out[pos] = (int32_t)item_label(a, bq, i);
-    if (out_s) out_s[pos] = key_score(k);
+  uint32_t k[kPer];
+  auto load_chunk = [&](int ch) {
+    const int64_t i0 = lo + (int64_t)ch * kSelChunk + (int64_t)tid * kPer;
+    if (i0 + kPer <= hi) {
+#pragma unroll
+      for (int v = 0; v < kPer / 4; ++v) {
+        const uint4 a4 = *reinterpret_cast<const uint4*>(keys + i0 + 4 * v);
+        k[4 * v] = a4.x;
+        k[4 * v + 1] = a4.y;
+        k[4 * v + 2] = a4.z;
+        k[4 * v + 3] = a4.w;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) k[e] = (i0 + e < hi) ? keys[i0 + e] : 0u;
+    }
   };
+  if (nchunks == 1) load_chunk(0);
+  // phase: keys loaded
 
-  // ---- radix levels over global memory until the threshold bin fits in shared memory ----
-  uint32_t prefix = 0, mask = 0, need = (uint32_t)K, inbin = 0;
-  int level = 0;
-  const int shifts[3] = {21, 10, 0};
-  const int widths[3] = {11, 11, 10};
-  for (;; ++level) {
-    const int sh = shifts[level];
-    const uint32_t nb = 1u << widths[level];
-    for (int i = tid; i < kBins; i += kSelThreads) hist[i] = 0;
-    __syncthreads();
-    for (int64_t i0 = (int64_t)tid * kPer; i0 < n; i0 += (int64_t)kSelThreads * kPer) {
-      uint32_t k[kPer];
-      load_keys(keys, i0, n, k);
+  // ---- 0. cluster-wide min / max / count of valid keys --------------------------------
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u, cnt = 0u;
+  for (int ch = 0; ch < nchunks; ++ch) {
+    if (nchunks > 1) load_chunk(ch);
 #pragma unroll
-      for (int e = 0; e < kPer; ++e)
-        if (k[e] != 0 && (k[e] & mask) == prefix) atomicAdd(&hist[(k[e] >> sh) & (nb - 1)], 1u);
+    for (int e = 0; e < kPer; ++e) {
+      if (k[e] != 0u) {
+        kmin = min(kmin, k[e]);
+        kmax = max(kmax, k[e]);
+        ++cnt;
+      }
     }
-    __syncthreads();
-    if (tid < 32) find_bin(hist, nb, need, &s_misc[0], &s_misc[1], &s_misc[2]);
-    __syncthreads();
-    if (level == 0 && s_misc[2] <= (uint32_t)K) break;  // everything valid is selected
-    const uint32_t T = s_misc[0];
-    need -= s_misc[1];
-    prefix |= T << sh;
-    mask |= (nb - 1) << sh;
-    inbin = hist[T];
-    __syncthreads();
-    if (inbin <= (uint32_t)kCap || level == 2) break;
   }
-  const bool all_valid = (mask == 0);
-
-  // ---- one ordered pass: selected keys to the output, threshold-bin keys to smem --------
-  // (all_valid: every non-zero key is selected; level 2 with a full-key tie: the first
-  //  `need` equal keys are taken directly)
-  const bool direct_ties = !all_valid && inbin > (uint32_t)kCap;
-  uint32_t n_gt = 0, n_eq = 0;
-  for (int64_t t0 = 0; t0 < n; t0 += (int64_t)kSelThreads * kPer) {
-    const int64_t i0 = t0 + (int64_t)tid * kPer;
-    uint32_t k[kPer];
-    load_keys(keys, i0, n, k);
-    uint32_t cg = 0, ce = 0;
 #pragma unroll
-    for (int e = 0; e < kPer; ++e) {
-      const uint32_t kp = k[e] & mask;
-      const bool valid = k[e] != 0;
-      cg += (valid && (all_valid || kp > prefix)) ? 1u : 0u;
-      ce += (valid && !all_valid && kp == prefix) ? 1u : 0u;
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  }
+  if (tid < 16) xch[tid] = (tid == 0) ? 0xFFFFFFFFu : 0u;
+  __syncthreads();
+  if ((tid & 31) == 0) {
+    atomicMin(&xch[0], kmin);
+    atomicMax(&xch[1], kmax);
+    atomicAdd(&xch[2], cnt);
+  }
+  cluster.sync();
+  uint32_t gmin = 0xFFFFFFFFu, gmax = 0u, gcnt = 0u;
+  // phase: range reduced
+  {
+    uint32_t v[kMaxCluster][3];
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) {
+      const uint32_t* rx = cluster.map_shared_rank(xch, r < C ? r : 0);
+      v[r][0] = rx[0];
+      v[r][1] = rx[1];
+      v[r][2] = r < C ? rx[2] : 0u;
     }
-    uint32_t tot;
-    const uint32_t pos = block_excl_scan(cg | (ce << 16), scan_ws, &tot);
-    uint32_t pg = n_gt + (pos & 0xFFFFu), pe = n_eq + (pos >> 16);
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) {
+      gmin = min(gmin, v[r][0]);
+      gmax = max(gmax, v[r][1]);
+      gcnt += v[r][2];
+    }
+  }
+
+  // ---- 1. radix levels ------------------------------------------------------------------
+  uint32_t prefix = 0u, mask = 0u, need = (uint32_t)K;
+  const bool all_valid = gcnt <= (uint32_t)K;
+  if (!all_valid) {
+    if (gmin == gmax) {
+      prefix = gmin;  // every valid key is equal: ties only
+      mask = 0xFFFFFFFFu;
+    } else {
+      int p = 31 - __clz(gmin ^ gmax);  // highest bit where keys differ
+      mask = p == 31 ? 0u : ~((2u << p) - 1u);
+      prefix = gmin & mask;
+      for (;;) {
+        const int sh = p >= 10 ? p - 10 : 0;
+        const int width = p - sh + 1;
+        const uint32_t nb = 1u << width;
+        for (int i = tid; i < (int)nb; i += kSelThreads) hist[i] = 0u;
+        __syncthreads();
+        for (int ch = 0; ch < nchunks; ++ch) {
+          if (nchunks > 1) load_chunk(ch);
+#pragma unroll
+          for (int e = 0; e < kPer; ++e)
+            if (k[e] != 0u && (k[e] & mask) == prefix) atomicAdd(&hist[(k[e] >> sh) & (nb - 1u)], 1u);
+        }
+        cluster.sync();  // every CTA's histogram complete
+        for (int i0 = 0; i0 < (int)nb; i0 += kSelThreads * 4) {  // 4 bins per thread per pass
+          uint32_t v[4][kMaxCluster];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u * kSelThreads + tid;
+#pragma unroll
+            for (int r = 0; r < kMaxCluster; ++r)
+              v[u][r] = (r < C && i < (int)nb) ? cluster.map_shared_rank(hist, r)[i] : 0u;
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u * kSelThreads + tid;
+            uint32_t sum = 0u;
+#pragma unroll
+            for (int r = 0; r < kMaxCluster; ++r) sum += v[u][r];
+            if (i < (int)nb) hsum[i] = sum;
+          }
+        }
+        __syncthreads();
+        find_bin(hsum, (int)nb, need, &misc[0], &misc[1], scan_ws);
+        __syncthreads();
+        const uint32_t T = misc[0];
+        need -= misc[1];
+        prefix |= T << sh;
+        mask |= (nb - 1u) << sh;
+        const uint32_t inbin = hsum[T];
+        cluster.sync();  // remote reads of `hist` done before it is reused
+        if (inbin == need) break;  // every key of the bin is selected
+        if (sh == 0) break;
+        p = sh - 1;
+      }
+    }
+  }
+
+  // ---- 2. ordered output -----------------------------------------------------------------
+  // phase: levels done
+  // per-CTA counts of selected keys (gt) and of keys equal to the threshold prefix (eq)
+  auto classify = [&](uint32_t key, bool& gt, bool& eq) {
+    const uint32_t kp = key & mask;
+    gt = key != 0u && (all_valid || kp > prefix);
+    eq = key != 0u && !all_valid && kp == prefix;
+  };
+  uint32_t my_gt = 0u, my_eq = 0u;
+  for (int ch = 0; ch < nchunks; ++ch) {
+    if (nchunks > 1) load_chunk(ch);
 #pragma unroll
     for (int e = 0; e < kPer; ++e) {
-      const uint32_t kp = k[e] & mask;
-      const bool valid = k[e] != 0;
-      if (valid && (all_valid || kp > prefix)) {
-        emit((int)pg, i0 + e, k[e]);
+      bool gt, eq;
+      classify(k[e], gt, eq);
+      my_gt += gt;
+      my_eq += eq;
+    }
+  }
+  uint64_t tot;
+  const uint64_t mine = block_excl_scan64((uint64_t)my_gt | ((uint64_t)my_eq << 32), scan_ws, &tot);
+  if (tid == 0) {
+    xch[4] = (uint32_t)tot;
+    xch[5] = (uint32_t)(tot >> 32);
+  }
+  cluster.sync();
+  uint32_t cta_gt = 0u, cta_eq = 0u, all_gt = 0u;
+  {
+    uint32_t g[kMaxCluster], q[kMaxCluster];
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) {
+      const uint32_t* rx = cluster.map_shared_rank(xch, r < C ? r : 0);
+      g[r] = r < C ? rx[4] : 0u;
+      q[r] = r < C ? rx[5] : 0u;
+    }
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) {
+      if (r < rank) {
+        cta_gt += g[r];
+        cta_eq += q[r];
+      }
+      all_gt += g[r];
+    }
+  }
+  uint32_t pg = cta_gt + (uint32_t)mine;
+  // phase: positions known
+  uint32_t pe = cta_eq + (uint32_t)(mine >> 32);
+  const uint32_t tie0 = (uint32_t)K - need;  // first slot of the equal keys
+  for (int ch = 0; ch < nchunks; ++ch) {
+    if (nchunks > 1) load_chunk(ch);
+    const int64_t i0 = lo + (int64_t)ch * kSelChunk + (int64_t)tid * kPer;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+      bool gt, eq;
+      classify(k[e], gt, eq);
+      if (gt) {
+        out[pg] = (int32_t)item_label(a, bq, i0 + e);
+        if (out_s) out_s[pg] = key_score(k[e]);
         ++pg;
-      } else if (valid && kp == prefix) {
-        if (direct_ties) {
-          if (pe < need) emit((int)(K - need + pe), i0 + e, k[e]);
-        } else {
-          cand_key[pe] = k[e];
-          cand_idx[pe] = (uint32_t)(i0 + e);
+      } else if (eq) {
+        if (pe < need) {
+          out[tie0 + pe] = (int32_t)item_label(a, bq, i0 + e);
+          if (out_s) out_s[tie0 + pe] = key_score(k[e]);
         }
         ++pe;
       }
     }
-    n_gt += tot & 0xFFFFu;
-    n_eq += tot >> 16;
   }
-  if (all_valid) {
-    for (int i = (int)n_gt + tid; i < K; i += kSelThreads) {
+  if (all_valid && rank == 0) {
+  // phase: written
+    for (int i = (int)all_gt + tid; i < K; i += kSelThreads) {
       out[i] = -1;
       if (out_s) out_s[i] = -INFINITY;
     }
-    return;
   }
-  if (direct_ties) return;
-
-  // ---- resolve the remaining digits among the shared-memory candidates -------------------
-  const int cnt = (int)n_eq;
-  __syncthreads();
-  for (int lv = level + 1; lv < 3 && (uint32_t)cnt > need; ++lv) {
-    const int sh = shifts[lv];
-    const uint32_t nb = 1u << widths[lv];
-    for (int i = tid; i < kBins; i += kSelThreads) hist[i] = 0;
-    __syncthreads();
-    for (int i = tid; i < cnt; i += kSelThreads) {
-      const uint32_t k = cand_key[i];
-      if ((k & mask) == prefix) atomicAdd(&hist[(k >> sh) & (nb - 1)], 1u);
-    }
-    __syncthreads();
-    if (tid < 32) find_bin(hist, nb, need, &s_misc[0], &s_misc[1], &s_misc[2]);
-    __syncthreads();
-    const uint32_t T = s_misc[0];
-    need -= s_misc[1];
-    prefix |= T << sh;
-    mask |= (nb - 1) << sh;
-    const uint32_t in2 = hist[T];
-    __syncthreads();
-    if (in2 == need) break;
-  }
-  // candidates above the threshold prefix, then equal ones lowest index first (cand is
-  // in index order)
-  const uint32_t base_out = (uint32_t)K - need;  // first tie slot
-  uint32_t g2 = n_gt, e2 = 0;
-  for (int c0 = 0; c0 < cnt; c0 += kSelThreads * kPer) {
-    const int i0 = c0 + tid * kPer;
-    uint32_t cg = 0, ce = 0;
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) {
-      if (i0 + e < cnt) {
-        const uint32_t kp = cand_key[i0 + e] & mask;
-        cg += kp > prefix ? 1u : 0u;
-        ce += kp == prefix ? 1u : 0u;
-      }
-    }
-    uint32_t tot;
-    const uint32_t pos = block_excl_scan(cg | (ce << 16), scan_ws, &tot);
-    uint32_t pg = g2 + (pos & 0xFFFFu), pe = e2 + (pos >> 16);
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) {
-      if (i0 + e < cnt) {
-        const uint32_t k = cand_key[i0 + e];
-        const uint32_t kp = k & mask;
-        if (kp > prefix) {
-          emit((int)pg, cand_idx[i0 + e], k);
-          ++pg;
-        } else if (kp == prefix) {
-          if (pe < need) emit((int)(base_out + pe), cand_idx[i0 + e], k);
-          ++pe;
-        }
-      }
-    }
-    g2 += tot & 0xFFFFu;
-    e2 += tot >> 16;
-  }
+  cluster.sync();  // keep every CTA's shared memory alive until remote reads are done
 }
 
 // ------------------------------------------------------------------------------------
@@ -708,9 +765,25 @@ cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t
   s.blocks = blocks;
   s.out_idx = out_idx;
   s.out_score = out_score;
-  e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelSmem);
+  const int64_t items = mode == kFlat ? max_n_vis
+                        : mode == kHier ? (max_n_vis + block - 1) / block
+                                        : (int64_t)n_blocks * block;
+  int64_t c = (items + kSelChunk - 1) / kSelChunk;  // one CTA per 16384 keys
+  s.csize = (int)(c < 1 ? 1 : (c > kMaxCluster ? kMaxCluster : c));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)s.csize, (unsigned)BQ);
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.dynamicSmemBytes = kSelSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)s.csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, select_kernel, s);
   if (e != cudaSuccess) return e;
-  select_kernel<<<BQ, kSelThreads, kSelSmem, stream>>>(s);
   return cudaGetLastError();
 }
 

@@ -150,3 +150,24 @@ def test_full128k_layer(orc):
                                    np.arange(512, dtype=np.int32).reshape(1, 1, 512), qd["swa"][0][b:b + 1].numpy(),
                                    qd["swa_start"][b:b + 1].numpy(), qd["q_pos"][b:b + 1].numpy(), SM)
         assert_attn_close(out[b:b + 1], o_ref, what=f"seq {b}")
+
+
+def test_long_list_several_tiles_per_cta(orc):
+    """K = 2048 plus the window is 17 tiles of 128 slots: the 8 CTAs of a query's cluster
+    take 2-3 tiles each and rescale their running output as the running max grows."""
+    N = 5000
+    kvp, o_kv = _pool(orc, 110, N)
+    rng = np.random.default_rng(11)
+    B, H, K = 2, 64, 2048
+    q = synth.queries(111, B, 1, H) * 3.0          # sharper softmax: the max moves between tiles
+    topk = np.stack([rng.choice(N, K, replace=False) for _ in range(B)]).astype(np.int32)[:, None]
+    topk[1, 0, 1000:1100] = -1
+    swa = synth.swa_window(112, B, 128)
+    q_pos = torch.tensor([[6000], [6001]], dtype=torch.int64)
+    start = q_pos[:, 0] - 127
+    out, lse, st = _run(q, kvp, torch.zeros(B, dtype=torch.int64), torch.from_numpy(topk), swa, start, q_pos)
+    assert st == 0
+    o_ref, l_ref = orc.sparse_attn(q.numpy(), o_kv, np.zeros(B, np.int64), topk, swa.numpy(), start.numpy(),
+                                   q_pos.numpy(), SM)
+    assert_attn_close(out, o_ref)
+    assert np.abs(lse - l_ref).max() < 1e-2
