@@ -62,13 +62,18 @@ def parse_args():
 
 # ---- distributed plumbing ------------------------------------------------------------------
 def dist_setup():
+    """One process per GPU (torchrun sets RANK / LOCAL_RANK / WORLD_SIZE); NCCL on GPUs,
+    gloo when the host has no GPU (the CPU tests of the multi-rank path)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                             device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=300)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            torch.distributed.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            torch.distributed.init_process_group("gloo", timeout=timeout)
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -80,9 +85,11 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Max of a host float over all ranks (the timing reduction: the slowest rank counts)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
