@@ -207,7 +207,7 @@ __device__ __forceinline__ void store_slot(uint8_t* Ks, int r, int hf, const Slo
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sm = tc::align_smem_1024(smem_raw);
   uint8_t* Ks = sm + kOffK;
   uint8_t* Qs = sm + kOffQ;
   uint8_t* Ps = sm + kOffP;

@@ -30,6 +30,7 @@
 // uint32 key (hierarchical mode: the max over `block` neighbouring lanes).  A CTA takes
 // a group of up to G queries of one sequence (multi-query verify), so the A operand is
 // built once for the group.
+#include <algorithm>
 #include <cooperative_groups.h>
 
 #include "csa2_device.cuh"
@@ -53,6 +54,7 @@ struct ScanArgs {
   const int32_t* n_vis;
   const int32_t* blocks;  // reindex only
   int Q, HI, hipad, G, n_groups, n_blocks, block;
+  int block_shift;        // log2(block)
   int N;                  // MMA N = G * hipad * 4
   int tmem_cols;
   int tiles_per_cta;
@@ -103,7 +105,7 @@ __device__ __forceinline__ uint2 codes_to_u8(uint32_t w) {
 template <int MODE, int HIPAD>
 __global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sm = tc::align_smem_1024(smem_raw);
   uint8_t* As = sm;                                   // [128 rows x 128 B], 128 B swizzle
   uint8_t* Bs = As + kRows * 128;                     // [N rows x 128 B]
   uint8_t* raw = Bs + a.N * 128;                      // 2 x kRawBytes
@@ -150,8 +152,8 @@ __global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
       const int cnt = (int)(limit - i0 < kRows ? limit - i0 : kRows);
       stage_async(dst + mis, seq + i0 * kIkBytes, cnt * kIkBytes, tid, kScanThreads);
     } else {
-      const int s = tid / a.block, sub = tid % a.block;  // 128/block blocks, `block` threads each
-      const int64_t slot_blk = i0 / a.block + s;
+      const int s = tid >> a.block_shift, sub = tid & (a.block - 1);  // 128/block blocks, `block` threads each
+      const int64_t slot_blk = (i0 >> a.block_shift) + s;
       int32_t c = -1;
       if (slot_blk < a.n_blocks) c = a.blocks[(int64_t)(b * a.Q + q0) * a.n_blocks + slot_blk];
       if (sub == 0) {
@@ -251,7 +253,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
       valid = j < limit;
       ent = rbuf + mis + tid * kIkBytes;
     } else {
-      const int s = tid / a.block, r = tid % a.block;
+      const int s = tid >> a.block_shift, r = tid & (a.block - 1);
       const int32_t c = segc[(ti & 1) * 128 + s];
       j = (int64_t)c * a.block + r;
       valid = c >= 0 && j < nq0;
@@ -313,7 +315,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
       uint32_t* krow = a.keys + ((int64_t)b * a.Q + q0 + g) * a.key_stride;
       if (MODE == kHier) {
         for (int o = 1; o < a.block; o <<= 1) key = max(key, __shfl_xor_sync(0xffffffffu, key, o));
-        if ((tid & (a.block - 1)) == 0 && i0 + tid < nq[g]) krow[(i0 + tid) / a.block] = key;
+        if ((tid & (a.block - 1)) == 0 && i0 + tid < nq[g]) krow[(i0 + tid) >> a.block_shift] = key;
       } else if (i0 + tid < limit) {
         krow[i0 + tid] = key;
       }
@@ -322,6 +324,299 @@ __global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
   }
   if (timed_out && tid == 0) flag(a.status, CSA2_DEV_TIMEOUT);
   tc::cp_async_wait<0>();
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, a.tmem_cols);
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// Streaming scan for the flat and hierarchical modes.  A CTA walks a contiguous run of
+// tiles of one sequence:
+//   * the copy warp (warp 4) moves each tile (128 consecutive 68 B keys) with one bulk
+//     copy into a ring of kStages raw buffers, up to kStages tiles ahead of the math; the
+//     copy starts at the 16 B boundary at or below the tile's first key (that lead,
+//     0..12 bytes, is the same for every tile of a sequence) and is rounded up to 16 B,
+//     falling back to word copies when the rounded copy would run past the pool;
+//   * the four worker warps own one tile row each: tile t's epilogue, then tile t+1's A
+//     operand, then thread 0 issues tile t+1's MMA.
+// The CTA is small (about 48 KB of shared memory, 160 threads), so four of them share an
+// SM and hide each other's MMA and copy latency.  Every wait is bounded; the workers
+// agree on giving up through a reducing barrier, and the copy warp waits for its
+// outstanding copies before the CTA exits.
+// ------------------------------------------------------------------------------------
+constexpr int kStreamWorkers = 128;                       // one tile row per thread
+constexpr int kStreamThreads = kStreamWorkers + 32;       // plus the copy warp
+constexpr int kStages = 3;                                // raw tiles in flight per CTA
+constexpr int kRawTile = kRows * kIkBytes + 16;           // one tile plus its lead, 16 B multiple
+constexpr int kWorkerBar = 1;                             // named barrier of the workers
+
+template <int MODE, int HIPAD>
+__global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = tc::align_smem_1024(smem_raw);
+  uint8_t* As = sm;                                   // [128 rows x 128 B], 128 B swizzle
+  uint8_t* Bs = As + kRows * 128;                     // [N rows x 128 B]
+  uint8_t* raw = Bs + a.N * 128;                      // kStages x kRawTile
+  int32_t* corr = reinterpret_cast<int32_t*>(raw + kStages * kRawTile);  // [N]
+  float* wq = reinterpret_cast<float*>(corr + a.N);                      // [G * HIPAD]
+  int64_t* nq = reinterpret_cast<int64_t*>(wq + a.G * HIPAD);            // [G] visible count per query
+  uint64_t* full = reinterpret_cast<uint64_t*>(nq + a.G);                // [kStages] raw tile landed
+  uint64_t* empty = full + kStages;                                      // [kStages] raw tile consumed
+  uint64_t* dfull = empty + kStages;                                     // accumulator ready
+  uint32_t* misc = reinterpret_cast<uint32_t*>(dfull + 1);               // tmem base, tiles built, issued
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = blockIdx.y / a.n_groups;
+  const int gidx = blockIdx.y % a.n_groups;
+  const int q0 = gidx * a.G;
+  const int G = min(a.G, a.Q - q0);
+
+  if (blockIdx.x == 0 && tid < G) valid_count(a, b, b * a.Q + q0 + tid, true);  // report bad counts once
+  int64_t limit = 0;
+  for (int g = 0; g < G; ++g) {
+    const int64_t n = valid_count(a, b, b * a.Q + q0 + g, false);
+    limit = n > limit ? n : limit;
+  }
+  const int64_t item0 = (int64_t)blockIdx.x * a.tiles_per_cta * kRows;
+  if (item0 >= limit) return;
+  const int64_t left_tiles = (limit - item0 + kRows - 1) / kRows;
+  const int ntiles = (int)(left_tiles < a.tiles_per_cta ? left_tiles : a.tiles_per_cta);
+  if (tid < G) nq[tid] = valid_count(a, b, b * a.Q + q0 + tid, false);
+
+  const uint8_t* seq = a.ik_pool + a.seq_base[b] * kIkBytes;
+  const uint32_t lead = (uint32_t)(reinterpret_cast<uintptr_t>(seq) & 15u);
+  const uint32_t raw_a = tc::smem_u32(raw);
+  const uint32_t full_a = tc::smem_u32(full), empty_a = tc::smem_u32(empty), dfull_a = tc::smem_u32(dfull);
+
+  if (warp == 0) tc::tmem_alloc(tc::smem_u32(misc), a.tmem_cols);
+  if (tid == 32) {
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(full_a + 8 * s, 1);
+      tc::mbar_init(empty_a + 8 * s, kStreamWorkers);
+    }
+    tc::mbar_init(dfull_a, 1);
+  }
+
+  // ---- B operand: four int8 limbs of every (query, head), plus epilogue constants ---------
+  for (int gh = warp; gh < a.G * HIPAD; gh += kStreamThreads / 32) {
+    const int g = gh / HIPAD, h = gh % HIPAD;
+    const bool live = g < G && h < a.HI;
+    float x[4] = {0.f, 0.f, 0.f, 0.f};
+    float wv = 0.f;
+    if (live) {
+      const int64_t bq = (int64_t)b * a.Q + q0 + g;
+      const float4 v = reinterpret_cast<const float4*>(a.q + (bq * a.HI + h) * kDI)[lane];
+      x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+      wv = a.w[bq * a.HI + h];
+    }
+    float m = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    // power-of-two scale S = 2^(5 - exponent(m)): x = q*S is exact and |x| < 64, so the
+    // first limb never leaves int8 and the limbs represent x to 2^-21 (heads whose max is
+    // below 1e-30 count as zero)
+    float S = 0.f;
+    if (m > 1e-30f) {
+      const int E = (int)((__float_as_uint(m) >> 23) & 0xFFu) - 127;
+      S = __uint_as_float((uint32_t)(127 + 5 - E) << 23);
+    }
+    uint32_t limb[4] = {0u, 0u, 0u, 0u};
+    int lsum[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float r = x[e] * S;
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const float L = rintf(r);
+        const int li = (int)L;
+        limb[p] |= ((uint32_t)(li & 0xFF)) << (8 * e);
+        lsum[p] += li;
+        r = (r - L) * 128.0f;
+      }
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const int n = gh * 4 + p;
+      *reinterpret_cast<uint32_t*>(Bs + tc::sw128(n, lane * 4)) = limb[p];
+      int t = lsum[p];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      if (lane == 0) corr[n] = 0x4B400000 - 12 * t;
+    }
+    if (lane == 0) wq[gh] = S > 0.f ? wv / (2.0f * S) : 0.f;
+  }
+  tc::fence_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = misc[0];
+
+  if (warp == kStreamWorkers / 32) {
+    // ---- copy warp ------------------------------------------------------------------------
+    const uint8_t* pool_end = a.ik_pool + a.pool_entries * kIkBytes;
+    int issued = 0;
+    bool ok = true;
+    for (int t = 0; t < ntiles; ++t) {
+      const int s = t % kStages;
+      if (t >= kStages) ok = tc::mbar_wait(empty_a + 8 * s, (uint32_t)((t / kStages) - 1) & 1u, kScanPolls);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      const int64_t i0 = item0 + (int64_t)t * kRows;
+      const int cnt = (int)(limit - i0 < kRows ? limit - i0 : kRows);
+      const uint8_t* src = seq + i0 * kIkBytes;
+      const uint32_t nbytes = (lead + (uint32_t)cnt * kIkBytes + 15u) & ~15u;
+      if (src - lead + nbytes <= pool_end) {
+        if (lane == 0) {
+          tc::mbar_arrive_expect_tx(full_a + 8 * s, nbytes);
+          tc::bulk_g2s(raw_a + s * kRawTile, src - lead, nbytes, full_a + 8 * s);
+        }
+      } else {  // the tile ends within 16 B of the pool's end
+        const uint32_t* sw = reinterpret_cast<const uint32_t*>(src);
+        uint32_t* dw = reinterpret_cast<uint32_t*>(raw + s * kRawTile + lead);
+        for (int k = lane; k < cnt * (kIkBytes / 4); k += 32) dw[k] = sw[k];
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(full_a + 8 * s);
+      }
+      issued = t + 1;
+    }
+    if (lane == 0) {
+      if (!ok) flag(a.status, CSA2_DEV_TIMEOUT);
+      misc[2] = (uint32_t)issued;
+    }
+  } else {
+    // ---- workers ----------------------------------------------------------------------------
+    const int row = tid;
+    const uint32_t idesc = tc::idesc_i8(kRows, a.N, false, true);
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t a_row = tc::smem_u32(As) + (uint32_t)row * 128u;  // this thread's A row
+    const uint32_t corr_a = tc::smem_u32(corr), wq_a = tc::smem_u32(wq), nq_a = tc::smem_u32(nq);
+
+    // build tile t's A row from its raw buffer; returns false if the copy never landed
+    auto build = [&](int t, float& sj, bool& valid) -> bool {
+      const int s = t % kStages;
+      const bool ok = tc::mbar_wait(full_a + 8 * s, (uint32_t)(t / kStages) & 1u, kScanPolls);
+      const int64_t j = item0 + (int64_t)t * kRows + row;
+      valid = ok && j < limit;
+      sj = 0.f;
+      if (valid) {
+        const uint32_t ea = raw_a + s * kRawTile + lead + row * kIkBytes;
+        uint32_t cw[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) cw[i] = tc::ld_shared_u32(ea + 4 * i);
+        sj = __uint_as_float(tc::ld_shared_u32(ea + 64));
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {  // 16 codes -> one 16 B chunk of the A row
+          const uint2 lo = codes_to_u8(cw[2 * c8]);
+          const uint2 hi = codes_to_u8(cw[2 * c8 + 1]);
+          tc::st_shared_v4(a_row + (((uint32_t)c8 ^ (row & 7u)) << 4), make_uint4(lo.x, lo.y, hi.x, hi.y));
+        }
+      }
+      if (ok) tc::mbar_arrive(empty_a + 8 * s);
+      tc::fence_async_smem();
+      tc::fence_before_sync();
+      return ok;
+    };
+    auto issue = [&]() {
+      if (tid == 0) {
+        tc::fence_after_sync();
+        const uint32_t ab = tc::smem_u32(As), bb = tc::smem_u32(Bs);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)  // K = 128 dims in steps of 32
+          tc::mma_i8(tmem, tc::smem_desc_sw128(ab + ks * 32, 16, 1024), tc::smem_desc_sw128(bb + ks * 32, 16, 1024),
+                     idesc, ks > 0 ? 1u : 0u);
+        tc::commit(dfull_a);
+      }
+    };
+    // limbs -> fp32 dot products -> ReLU-weighted score -> order-preserving keys of tile t
+    auto epilogue = [&](int t, float sj, bool valid) -> bool {
+      const bool ok = tc::mbar_wait(dfull_a, (uint32_t)t & 1u, kScanPolls);
+      tc::fence_after_sync();
+      const int64_t j = item0 + (int64_t)t * kRows + row;
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        if (g >= G) break;
+        uint32_t r[HIPAD * 4];
+        const uint32_t ta = lane_addr + (uint32_t)(g * HIPAD * 4);
+        if (HIPAD == 4) {
+          tc::tmem_ld16(ta, r);
+        } else {
+#pragma unroll
+          for (int c = 0; c < HIPAD * 4; c += 32) tc::tmem_ld32(ta + c, *reinterpret_cast<uint32_t(*)[32]>(r + c));
+        }
+        float tot = 0.f;
+#pragma unroll
+        for (int h4 = 0; h4 < HIPAD / 4; ++h4) {
+          const uint4 w4 = tc::ld_shared_v4(wq_a + (uint32_t)(g * HIPAD + h4 * 4) * 4u);
+          const float wh[4] = {__uint_as_float(w4.x), __uint_as_float(w4.y), __uint_as_float(w4.z),
+                               __uint_as_float(w4.w)};
+#pragma unroll
+          for (int hh = 0; hh < 4; ++hh) {
+            const int h = h4 * 4 + hh;
+            const uint4 c = tc::ld_shared_v4(corr_a + (uint32_t)(g * HIPAD + h) * 16u);
+            const float f0 = __int_as_float((int)(r[h * 4 + 0] + c.x)) - 12582912.0f;
+            const float f1 = __int_as_float((int)(r[h * 4 + 1] + c.y)) - 12582912.0f;
+            const float f2 = __int_as_float((int)(r[h * 4 + 2] + c.z)) - 12582912.0f;
+            const float f3 = __int_as_float((int)(r[h * 4 + 3] + c.w)) - 12582912.0f;
+            const float z = fmaf(fmaf(fmaf(f3, 0.0078125f, f2), 0.0078125f, f1), 0.0078125f, f0);
+            tot = fmaf(wh[hh], fmaxf(z, 0.f), tot);
+          }
+        }
+        const int64_t nqg = (int64_t)tc::ld_shared_u64(nq_a + 8u * (uint32_t)g);
+        const bool vis = valid && j < nqg;
+        uint32_t key = vis ? score_key(sj * tot) : 0u;
+        uint32_t* krow = a.keys + ((int64_t)b * a.Q + q0 + g) * a.key_stride;
+        if (MODE == kHier) {
+          for (int o = 1; o < a.block; o <<= 1) key = max(key, __shfl_xor_sync(0xffffffffu, key, o));
+          if ((row & (a.block - 1)) == 0 && j < nqg) krow[j >> a.block_shift] = key;
+        } else if (j < limit) {
+          krow[j] = key;
+        }
+      }
+      tc::fence_before_sync();
+      return ok;
+    };
+
+    float sj = 0.f, sj_nxt = 0.f;
+    bool v = false, v_nxt = false;
+    int built = 0;  // tiles whose raw buffer every worker consumed
+    bool bad = tc::named_sync_or(kWorkerBar, kStreamWorkers, !build(0, sj, v));
+    if (!bad) {
+      issue();
+      built = 1;
+    }
+    bool last_ok = true;
+    for (int t = 0; t < ntiles && !bad; ++t) {
+      bool fail = !epilogue(t, sj, v);
+      if (t + 1 < ntiles) {
+        fail |= !build(t + 1, sj_nxt, v_nxt);
+        bad = tc::named_sync_or(kWorkerBar, kStreamWorkers, fail);
+        if (!bad) {
+          issue();
+          built = t + 2;
+        }
+        sj = sj_nxt;
+        v = v_nxt;
+      } else {
+        last_ok = !fail;
+      }
+    }
+    if (tid == 0) {
+      if (bad || !last_ok) flag(a.status, CSA2_DEV_TIMEOUT);
+      if (bad && built > 0)  // let the last issued MMA finish before the accumulator goes
+        tc::mbar_wait(dfull_a, (uint32_t)(built - 1) & 1u, kScanPolls);
+      misc[1] = (uint32_t)(bad ? (built > 0 ? built - 1 : 0) : ntiles);
+    }
+  }
+  __syncthreads();
+  if (tid == kStreamWorkers) {  // copies that landed in no tile the workers consumed
+    for (int t = (int)misc[1]; t < (int)misc[2]; ++t)
+      tc::mbar_wait(full_a + 8 * (t % kStages), (uint32_t)(t / kStages) & 1u, kScanPolls);
+  }
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 0) {
@@ -361,6 +656,7 @@ struct SelectArgs {
   int64_t key_stride;
   int mode;
   int Q, block, n_blocks, K;
+  int block_shift;           // log2(block)
   int csize;                 // CTAs per query (cluster size)
   const int64_t* seq_base;
   const int32_t* n_vis;
@@ -372,8 +668,8 @@ struct SelectArgs {
 
 __device__ __forceinline__ int64_t item_label(const SelectArgs& a, int bq, int64_t i) {
   if (a.mode == kReindex) {
-    const int32_t c = a.blocks[(int64_t)bq * a.n_blocks + i / a.block];
-    return (int64_t)c * a.block + i % a.block;
+    const int32_t c = a.blocks[(int64_t)bq * a.n_blocks + (i >> a.block_shift)];
+    return ((int64_t)c << a.block_shift) + (i & (a.block - 1));
   }
   return i;
 }
@@ -465,7 +761,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
     if (a.mode == kFlat)
       n = nv;
     else if (a.mode == kHier)
-      n = (nv + a.block - 1) / a.block;
+      n = (nv + a.block - 1) >> a.block_shift;
     else
       n = (int64_t)a.n_blocks * a.block;
   }
@@ -717,6 +1013,78 @@ static cudaError_t launch_scan(ScanArgs a, int64_t items, int B, cudaStream_t st
   return cudaGetLastError();
 }
 
+// CTAs of `fn` that fit on one SM at once, from its register count, its shared memory and
+// the device's per-SM limits (registers are allocated per warp in units of 256).
+template <typename F>
+static cudaError_t resident_ctas(F fn, int dev, int threads, size_t dyn_smem, int* out) {
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, fn);
+  if (e != cudaSuccess) return e;
+  int regs_sm = 0, smem_sm = 0, reserved = 0, thr_sm = 0, blk_sm = 0;
+  if ((e = cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&thr_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&blk_sm, cudaDevAttrMaxBlocksPerMultiprocessor, dev)) != cudaSuccess)
+    return e;
+  const int warps = (threads + 31) / 32;
+  const int regs_cta = warps * (((fa.numRegs * 32) + 255) / 256) * 256;
+  int n = blk_sm;
+  n = std::min(n, thr_sm / (warps * 32));
+  if (regs_cta > 0) n = std::min(n, regs_sm / regs_cta);
+  n = std::min(n, (int)((size_t)smem_sm / (dyn_smem + fa.sharedSizeBytes + (size_t)reserved)));
+  *out = std::max(n, 1);
+  return cudaSuccess;
+}
+
+// Flat / hierarchical scan: about two waves of stream_scan_kernel CTAs, each taking a
+// contiguous run of at least 8 tiles.
+template <int MODE>
+static cudaError_t launch_stream(ScanArgs a, int64_t items, int B, cudaStream_t st) {
+  a.hipad = a.HI <= 4 ? 4 : (a.HI <= 8 ? 8 : 16);
+  a.G = max(1, min(a.Q, 256 / (a.hipad * 4)));
+  a.n_groups = (a.Q + a.G - 1) / a.G;
+  a.N = a.G * a.hipad * 4;
+  a.tmem_cols = pow2_at_least(a.N);
+  const int64_t tiles = (items + kRows - 1) / kRows;
+  const int64_t rows = (int64_t)B * a.n_groups;
+  if (tiles == 0 || rows == 0) return cudaSuccess;
+  const size_t smem = 1024 + (size_t)kRows * 128 + (size_t)a.N * 128 + (size_t)kStages * kRawTile +
+                      (size_t)a.N * 4 + (size_t)a.G * a.hipad * 4 + (size_t)a.G * 8 + (2 * kStages + 1) * 8 + 16;
+  int dev = 0, sms = 148, occ = 1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+#define CSA2_STREAM_LAUNCH(HP)                                                                          \
+  {                                                                                                     \
+    auto* fn = stream_scan_kernel<MODE, HP>;                                                            \
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);               \
+    if (e != cudaSuccess) return e;                                                                     \
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,                        \
+                             (int)cudaSharedmemCarveoutMaxShared);                                      \
+    if (e != cudaSuccess) return e;                                                                     \
+    e = resident_ctas(fn, dev, kStreamThreads, smem, &occ);                                             \
+    if (e != cudaSuccess) return e;                                                                     \
+    const int64_t slots = (int64_t)sms * (occ > 0 ? occ : 1);                                           \
+    int64_t tpc = (tiles * rows + 2 * slots - 1) / (2 * slots);                                         \
+    tpc = tpc < 8 ? 8 : tpc;                                                                            \
+    tpc = tpc > tiles ? tiles : tpc;                                                                    \
+    a.tiles_per_cta = (int)tpc;                                                                         \
+    const dim3 grid((unsigned)((tiles + tpc - 1) / tpc), (unsigned)rows);                               \
+    fn<<<grid, kStreamThreads, smem, st>>>(a);                                                          \
+  }
+  if (a.hipad == 4) {
+    CSA2_STREAM_LAUNCH(4)
+  } else if (a.hipad == 8) {
+    CSA2_STREAM_LAUNCH(8)
+  } else {
+    CSA2_STREAM_LAUNCH(16)
+  }
+#undef CSA2_STREAM_LAUNCH
+  return cudaGetLastError();
+}
+
 cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t* ik_pool,
                          int64_t pool_entries, const int64_t* seq_base, const int32_t* n_vis,
                          const int32_t* blocks, int B, int Q, int HI, int n_blocks, int block,
@@ -735,6 +1103,7 @@ cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t
   a.HI = HI;
   a.n_blocks = n_blocks;
   a.block = block;
+  a.block_shift = __builtin_ctz((unsigned)block);
   a.max_n_vis = max_n_vis;
   a.key_stride = key_stride;
   a.keys = keys;
@@ -743,9 +1112,9 @@ cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t
   if (BQ == 0) return cudaSuccess;
   cudaError_t e;
   if (mode == kFlat)
-    e = launch_scan<kFlat>(a, max_n_vis, B, stream);
+    e = launch_stream<kFlat>(a, max_n_vis, B, stream);
   else if (mode == kHier)
-    e = launch_scan<kHier>(a, max_n_vis, B, stream);
+    e = launch_stream<kHier>(a, max_n_vis, B, stream);
   else
     e = launch_scan<kReindex>(a, (int64_t)n_blocks * block, B * Q, stream);
   if (e != cudaSuccess) return e;
@@ -756,6 +1125,7 @@ cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t
   s.mode = mode;
   s.Q = Q;
   s.block = block;
+  s.block_shift = __builtin_ctz((unsigned)block);
   s.n_blocks = n_blocks;
   s.K = K;
   s.seq_base = seq_base;

@@ -23,6 +23,37 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte-aligned byte at or above `base` (dynamic shared memory), reached by
+// pointer arithmetic on `base` so the compiler still knows the result is shared memory and
+// emits shared-memory loads and stores instead of generic ones.
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* base) {
+  const uint32_t s = smem_u32(base);
+  return base + (((s + 1023u) & ~1023u) - s);
+}
+
+// Shared-memory loads and stores at 32-bit shared addresses.  volatile with a memory
+// clobber, so they stay ordered with the barrier and mbarrier waits around them.
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t saddr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(saddr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t saddr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(saddr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ uint64_t ld_shared_u64(uint32_t saddr) {
+  uint64_t v;
+  asm volatile("ld.shared.u64 %0, [%1];" : "=l"(v) : "r"(saddr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
 // Byte offset of (row, byte-in-row) in a 128-byte-swizzled tile whose rows are 128 B.
 __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t byte) {
   return row * 128u + ((((byte >> 4) ^ row) & 7u) << 4) + (byte & 15u);
@@ -144,6 +175,16 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
       : "memory");
 }
 
+// 8 consecutive 32-bit columns (32x32b shape, x8), load and wait in one statement.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+}
+
 // Asynchronous global -> shared copies (cp.async), 16 B (L2 only) and 4 B.
 __device__ __forceinline__ void cp_async16(uint32_t dst_saddr, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_saddr), "l"(src) : "memory");
@@ -178,6 +219,25 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst_saddr, const void* src, ui
                ::"r"(dst_saddr), "l"(src), "r"(bytes), "r"(mbar_saddr)
                : "memory");
 }
+// Plain arrival (release semantics at CTA scope).
+__device__ __forceinline__ void mbar_arrive(uint32_t mbar_saddr) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar_saddr) : "memory");
+}
+// Barrier among a subset of warps (named barrier `id`, `nthreads` participants) that
+// also ORs a predicate over them.
+__device__ __forceinline__ bool named_sync_or(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
 // Arrive on the mbarrier and add `bytes` to the transaction count it waits for.
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t mbar_saddr, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar_saddr), "r"(bytes) : "memory");

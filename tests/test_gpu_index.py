@@ -109,6 +109,18 @@ def test_bad_count_flags_and_empties(orc):
     assert (topk[0, 1] >= 0).all()            # the good one is unaffected
 
 
+def test_bad_count_every_query_of_a_sequence(orc):
+    """No query of the sequence has a valid count: nothing is scanned, the flag is still set."""
+    T = 500
+    kv, ik = synth.kv_tokens(52, T, device="cuda")
+    _, ikp, _, _ = pools_from_tokens(orc, kv, ik)
+    q, w = synth.index_queries(53, 1, 2, 8)
+    topk, _, st = run_full(q.cuda(), w.cuda(), ikp, torch.zeros(1, dtype=torch.int64, device="cuda"),
+                           torch.tensor([[600, -3]], dtype=torch.int32, device="cuda"), 16, 500)
+    assert st & csa2.DEV_BAD_COUNT
+    assert (topk == -1).all()
+
+
 @pytest.mark.parametrize("N,n_blocks,block", [(37, 2, 8), (5003, 64, 8), (16384, 2048, 8),
                                               (20011, 512, 8), (3000, 100, 1), (9000, 40, 32)])
 def test_hier_blocks_and_reindex(orc, N, n_blocks, block):
