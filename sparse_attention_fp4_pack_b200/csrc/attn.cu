@@ -205,6 +205,7 @@ __device__ __forceinline__ void store_slot(uint8_t* Ks, int r, int hf, const Slo
 }
 
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
+  chain_enter();
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = tc::align_smem_1024(smem_raw);
@@ -436,28 +437,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
     a.lse[(int64_t)bq * H + hh] = L > 0.0f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
   }
   __syncthreads();
-  // thread -> (float4 column d4, 2 heads per pass); every CTA's float4 is loaded before use
+  // thread -> (float4 column d4, heads hb, hb+2, hb+4, hb+6 per pass): every remote float4
+  // of a pass is loaded before any is used, so a pass costs one interconnect round trip
   const int d4 = tid & 127;
-  for (int hl = tid >> 7; hl < h1 - h0; hl += 2) {
-    const int hh = h0 + hl;
-    float4 o[kMaxCluster];
+  const int nh = h1 - h0;
+  for (int hb = tid >> 7; hb < nh; hb += 8) {
+    float4 o[4][kMaxCluster];
 #pragma unroll
-    for (int c = 0; c < kMaxCluster; ++c)
-      o[c] = (c < C && fac[c * 64 + hl] > 0.0f)
-                 ? reinterpret_cast<const float4*>(cluster.map_shared_rank(Of, c) + hh * kD)[d4]
-                 : make_float4(0.f, 0.f, 0.f, 0.f);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < 4; ++u) {
+      const int hl = hb + 2 * u;
 #pragma unroll
-    for (int c = 0; c < kMaxCluster; ++c) {
-      const float f = c < C ? fac[c * 64 + hl] : 0.0f;
-      acc.x = fmaf(o[c].x, f, acc.x);
-      acc.y = fmaf(o[c].y, f, acc.y);
-      acc.z = fmaf(o[c].z, f, acc.z);
-      acc.w = fmaf(o[c].w, f, acc.w);
+      for (int c = 0; c < kMaxCluster; ++c)
+        o[u][c] = (hl < nh && c < C && fac[c * 64 + hl] > 0.0f)
+                      ? reinterpret_cast<const float4*>(cluster.map_shared_rank(Of, c) + (h0 + hl) * kD)[d4]
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    const float inv = linv[hl];
-    reinterpret_cast<float4*>(a.out + ((int64_t)bq * H + hh) * kD)[d4] =
-        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int hl = hb + 2 * u;
+      if (hl < nh) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < kMaxCluster; ++c) {
+          const float f = c < C ? fac[c * 64 + hl] : 0.0f;
+          acc.x = fmaf(o[u][c].x, f, acc.x);
+          acc.y = fmaf(o[u][c].y, f, acc.y);
+          acc.z = fmaf(o[u][c].z, f, acc.z);
+          acc.w = fmaf(o[u][c].w, f, acc.w);
+        }
+        const float inv = linv[hl];
+        reinterpret_cast<float4*>(a.out + ((int64_t)bq * H + h0 + hl) * kD)[d4] =
+            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+      }
+    }
   }
   cluster.sync();  // remote reads finished before any CTA releases its shared memory
   // phase: merged
@@ -507,19 +519,8 @@ cudaError_t launch_sparse_attn(const float* q, const uint8_t* kv_pool, int64_t p
   if (BQ == 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)a.csize, (unsigned)BQ);
-  cfg.blockDim = dim3(kAttnThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)a.csize;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, a);
+  e = launch_chained(attn_tc_kernel, dim3((unsigned)a.csize, (unsigned)BQ), dim3(kAttnThreads), kSmemBytes, stream,
+                     (unsigned)a.csize, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -7,6 +7,7 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
 #include <cuda_runtime.h>
 
 #include "csa2.h"
@@ -17,6 +18,44 @@ constexpr int kD = CSA2_D;
 constexpr int kDI = CSA2_DI;
 constexpr int kKvBytes = CSA2_KV_ENTRY_BYTES;
 constexpr int kIkBytes = CSA2_IK_ENTRY_BYTES;
+
+// Programmatic dependent launch.  Every libcsa2 kernel is launched with programmatic
+// stream serialization, so its CTAs may be scheduled while the previous kernel in the
+// stream is still running.  Each kernel starts with chain_enter: it lets its own successor
+// begin launching, then waits until its predecessor has completed and that kernel's
+// writes are visible, before it touches global memory.  What overlaps is the launch and
+// CTA scheduling, not any data access.
+__device__ __forceinline__ void chain_enter() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Host side: launch `kernel` with programmatic stream serialization, plus a cluster of
+// cluster_x CTAs along x when cluster_x > 0.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                  cudaStream_t stream, unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 0) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 __device__ __forceinline__ void flag(uint32_t* status, uint32_t bit) {
   if (status) atomicOr(status, bit);

@@ -104,6 +104,7 @@ __device__ __forceinline__ uint2 codes_to_u8(uint32_t w) {
 
 template <int MODE, int HIPAD>
 __global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
+  chain_enter();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = tc::align_smem_1024(smem_raw);
   uint8_t* As = sm;                                   // [128 rows x 128 B], 128 B swizzle
@@ -355,6 +356,7 @@ constexpr int kWorkerBar = 1;                             // named barrier of th
 
 template <int MODE, int HIPAD>
 __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs a) {
+  chain_enter();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = tc::align_smem_1024(smem_raw);
   uint8_t* As = sm;                                   // [128 rows x 128 B], 128 B swizzle
@@ -735,6 +737,7 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, int nb, uint32_t 
 }
 
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
+  chain_enter();
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ __align__(16) uint32_t sel_smem[];
@@ -964,8 +967,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
       }
     }
   }
-  if (all_valid && rank == 0) {
   // phase: written
+  if (all_valid && rank == 0) {
     for (int i = (int)all_gt + tid; i < K; i += kSelThreads) {
       out[i] = -1;
       if (out_s) out_s[i] = -INFINITY;
@@ -1001,7 +1004,8 @@ static cudaError_t launch_scan(ScanArgs a, int64_t items, int B, cudaStream_t st
   e = cudaFuncSetAttribute(scan_tc_kernel<MODE, HP>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                            (int)smem);                                                              \
   if (e != cudaSuccess) return e;                                                                   \
-  scan_tc_kernel<MODE, HP><<<grid, kScanThreads, smem, st>>>(a);
+  e = launch_chained(scan_tc_kernel<MODE, HP>, grid, dim3(kScanThreads), smem, st, 0, a);             \
+  if (e != cudaSuccess) return e;
   if (a.hipad == 4) {
     CSA2_SCAN_LAUNCH(4)
   } else if (a.hipad == 8) {
@@ -1072,7 +1076,8 @@ static cudaError_t launch_stream(ScanArgs a, int64_t items, int B, cudaStream_t 
     tpc = tpc > tiles ? tiles : tpc;                                                                    \
     a.tiles_per_cta = (int)tpc;                                                                         \
     const dim3 grid((unsigned)((tiles + tpc - 1) / tpc), (unsigned)rows);                               \
-    fn<<<grid, kStreamThreads, smem, st>>>(a);                                                          \
+    e = launch_chained(fn, grid, dim3(kStreamThreads), smem, st, 0, a);                                 \
+    if (e != cudaSuccess) return e;                                                                     \
   }
   if (a.hipad == 4) {
     CSA2_STREAM_LAUNCH(4)
@@ -1116,7 +1121,7 @@ cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t
   else if (mode == kHier)
     e = launch_stream<kHier>(a, max_n_vis, B, stream);
   else
-    e = launch_scan<kReindex>(a, (int64_t)n_blocks * block, B * Q, stream);
+    e = launch_scan<kReindex>(a, (int64_t)n_blocks * block, B, stream);  // one CTA row per (b, query)
   if (e != cudaSuccess) return e;
 
   SelectArgs s;
@@ -1140,19 +1145,8 @@ cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t
                                         : (int64_t)n_blocks * block;
   int64_t c = (items + kSelChunk - 1) / kSelChunk;  // one CTA per 16384 keys
   s.csize = (int)(c < 1 ? 1 : (c > kMaxCluster ? kMaxCluster : c));
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)s.csize, (unsigned)BQ);
-  cfg.blockDim = dim3(kSelThreads);
-  cfg.dynamicSmemBytes = kSelSmem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)s.csize;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, select_kernel, s);
+  e = launch_chained(select_kernel, dim3((unsigned)s.csize, (unsigned)BQ), dim3(kSelThreads), kSelSmem, stream,
+                     (unsigned)s.csize, s);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

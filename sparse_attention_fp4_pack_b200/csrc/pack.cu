@@ -35,6 +35,7 @@ __global__ void __launch_bounds__(256) pack_kv_kernel(const uint16_t* __restrict
                                                       uint8_t* __restrict__ kv_pool,
                                                       uint8_t* __restrict__ ik_pool,
                                                       uint32_t* status) {
+  chain_enter();
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -133,9 +134,10 @@ cudaError_t launch_pack_kv(const void* kv, const void* ik, int64_t T, int ratio,
   int64_t blocks = (E + 7) / 8;
   const int64_t cap = (int64_t)num_sms * 16;  // 16 resident 256-thread blocks per SM
   if (blocks > cap) blocks = cap;
-  pack_kv_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
-      static_cast<const uint16_t*>(kv), static_cast<const uint16_t*>(ik), E, ratio, dst,
-      pool_entries, kv_pool, ik_pool, status);
+  cudaError_t e = launch_chained(pack_kv_kernel, dim3((unsigned)blocks), dim3(threads), 0, stream, 0,
+                                 static_cast<const uint16_t*>(kv), static_cast<const uint16_t*>(ik), E, ratio,
+                                 dst, pool_entries, kv_pool, ik_pool, status);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

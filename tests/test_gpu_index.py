@@ -156,6 +156,41 @@ def test_hier_blocks_and_reindex(orc, N, n_blocks, block):
     assert int(st.item()) == 0
 
 
+def test_reindex_several_sequences_and_queries(orc):
+    """B = 3 sequences (misaligned bases) x Q = 3 queries, each with its own block set and
+    visible count: every (sequence, query) pair scans its own candidates."""
+    lengths = [7001, 2222, 5003]
+    T = sum(lengths)
+    kv, ik = synth.kv_tokens(80, T, device="cuda")
+    _, ikp, _, o_ik = pools_from_tokens(orc, kv, ik)
+    base = np.cumsum([0] + lengths[:-1]).astype(np.int64)
+    B, Q, HI, n_blocks, block, K = 3, 3, 8, 96, 8, 300
+    n_vis = np.array([[7001, 6000, 321], [2222, 2000, 1500], [5003, 4997, 8]], np.int32)
+    rng = np.random.default_rng(81)
+    blocks = np.full((B, Q, n_blocks), -1, np.int32)
+    for b in range(B):
+        for i in range(Q):
+            nb = (int(n_vis[b, i]) + block - 1) // block
+            take = min(n_blocks - 4, nb)
+            blocks[b, i, :take] = rng.choice(nb, take, replace=False)
+    q, w = synth.index_queries(82, B, Q, HI)
+    topk = torch.full((B, Q, K), -7, dtype=torch.int32, device="cuda")
+    st = csa2.status_word()
+    csa2.csa2_reindex(q.cuda(), w.cuda(), ikp, torch.from_numpy(base).cuda(), torch.from_numpy(n_vis).cuda(),
+                      torch.from_numpy(blocks).cuda(), block, K, topk, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    o_topk, _ = orc.reindex(q.numpy(), w.numpy(), o_ik, base, n_vis, blocks, K, block=block)
+    g = topk.cpu().numpy()
+    for b in range(B):
+        n_b = lengths[b]
+        for i in range(Q):
+            n = int(n_vis[b, i])
+            s = orc.index_scores(q[b, i].numpy(), w[b, i].numpy(), o_ik[base[b]:base[b] + n_b])
+            cand = sorted({j for c in blocks[b, i] if c >= 0 for j in range(c * block, min(n, c * block + block))})
+            assert_topk_set(g[b, i], o_topk[b, i], s[cand], K, labels=cand, what=f"b{b} q{i}")
+
+
 def test_reindex_empty_slots_and_bad_ids(orc):
     N = 300
     kv, ik = synth.kv_tokens(70, N, device="cuda")
