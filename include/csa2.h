@@ -13,6 +13,8 @@
  *    returned by csa2_status_string).  The library allocates nothing, keeps no pointer
  *    after returning, holds no global mutable state and never synchronises: each call
  *    validates its host-visible arguments, enqueues its kernels on `stream` and returns.
+ *    The one exception is csa2_reindex_static (end of this file), which uses a device
+ *    array compiled into the library and caches its address per device.
  *  - On CSA2_ERR_INVALID_ARG or CSA2_ERR_UNSUPPORTED nothing has been launched.
  *    CSA2_ERR_CUDA reports a launch failure (cudaGetLastError after the launch).
  *  - Values that live on the device (sequence bases, visible counts, Top-K indices,
@@ -59,6 +61,7 @@ extern "C" {
 #define CSA2_MAX_K 2048          /* largest Top-K / block count per query */
 #define CSA2_MAX_HI 16           /* largest number of indexer heads */
 #define CSA2_MAX_WINDOW 1024     /* largest sliding window */
+#define CSA2_STATIC_SCRATCH_BYTES (4u << 20) /* device array behind csa2_reindex_static */
 
 typedef enum csa2_status {
   CSA2_OK = 0,
@@ -191,6 +194,37 @@ csa2_status csa2_sparse_attn(const float* q, const uint8_t* kv_pool, int64_t poo
                              const int64_t* q_pos, int window, int B, int Q, int H,
                              float sm_scale, float* out, float* lse, void* ws, size_t ws_bytes,
                              uint32_t* dev_status, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * csa2_reindex_static: csa2_reindex without a workspace argument.  The pages have no
+ * counterpart to this call; it is a library convenience for callers that cannot hand
+ * the library device memory: a host with no device allocator of its own, or an engine
+ * whose device memory is planned once before decoding and which must not ask for more
+ * inside the decode loop.
+ *
+ * Arguments, layouts, results and device-side checks are those of csa2_reindex.  The
+ * key scratch is a device array of CSA2_STATIC_SCRATCH_BYTES (4 MiB) compiled into the
+ * library; every GPU on which the library's device code is loaded holds it until the
+ * process exits.  Nothing is allocated by the call.
+ *  - Size limit: when csa2_reindex_workspace_size(B, Q, HI, n_blocks, block, K) exceeds
+ *    CSA2_STATIC_SCRATCH_BYTES the call returns CSA2_ERR_UNSUPPORTED before touching
+ *    the device (n_blocks * block = 16,384 candidates fit 64 queries).
+ *  - Set-up: the first call on a device, with that device current, looks up the array's
+ *    device address (cudaGetSymbolAddress) and caches it; CSA2_ERR_CUDA if that fails.
+ *    Make the first call on each device before any stream capture.
+ *  - Nothing in the array needs to start at zero: the scan writes every key the
+ *    selection reads back within the same call.
+ *  - One array per device: calls whose kernels overlap on the same device (several
+ *    streams or host threads) race on it and their results are undefined.  Issue the
+ *    calls for one device on one stream.
+ * csa2_static_scratch_bytes() returns CSA2_STATIC_SCRATCH_BYTES.
+ * --------------------------------------------------------------------------------- */
+size_t csa2_static_scratch_bytes(void);
+csa2_status csa2_reindex_static(const float* q, const float* w, const uint8_t* ik_pool,
+                                int64_t pool_entries, const int64_t* seq_base, const int32_t* n_vis,
+                                const int32_t* blocks, int n_blocks, int block, int B, int Q, int HI,
+                                int K, int32_t* topk, float* topk_score, uint32_t* dev_status,
+                                cudaStream_t stream);
 
 #ifdef __cplusplus
 }

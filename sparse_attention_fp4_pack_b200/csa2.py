@@ -57,6 +57,10 @@ def lib():
         L.csa2_reindex_workspace_size.argtypes = [I32, I32, I32, I32, I32, I32]
         L.csa2_reindex.restype = I32
         L.csa2_reindex.argtypes = [P, P, P, I64, P, P, P, I32, I32, I32, I32, I32, I32, P, P, P, SZ, P, P]
+        L.csa2_static_scratch_bytes.restype = SZ
+        L.csa2_static_scratch_bytes.argtypes = []
+        L.csa2_reindex_static.restype = I32
+        L.csa2_reindex_static.argtypes = [P, P, P, I64, P, P, P, I32, I32, I32, I32, I32, I32, P, P, P, P]
         L.csa2_sparse_attn_workspace_size.restype = SZ
         L.csa2_sparse_attn_workspace_size.argtypes = [I32, I32, I32, I32, I32]
         L.csa2_sparse_attn.restype = I32
@@ -202,6 +206,30 @@ def csa2_reindex(q, w, ik_pool, seq_base, n_vis, blocks, block, K, topk, topk_sc
                               _ptr(n_vis), _ptr(blocks), n_blocks, block, B, Q, HI, K, _ptr(topk),
                               _ptr(topk_score), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)),
            "csa2_reindex")
+
+
+def csa2_static_scratch_bytes():
+    return lib().csa2_static_scratch_bytes()
+
+
+def csa2_reindex_static(q, w, ik_pool, seq_base, n_vis, blocks, block, K, topk, topk_score=None,
+                        dev_status=None, stream=None):
+    """csa2_reindex with the library's own static device scratch instead of a workspace:
+    for callers that cannot allocate device memory for the call (see include/csa2.h)."""
+    _need(q, torch.float32, "q", 4)
+    _need(w, torch.float32, "w", 3)
+    _need(ik_pool, torch.uint8, "ik_pool", 2)
+    _need(seq_base, torch.int64, "seq_base", 1)
+    _need(n_vis, torch.int32, "n_vis", 2)
+    _need(blocks, torch.int32, "blocks", 3)
+    _need(topk, torch.int32, "topk", 3)
+    _need(topk_score, torch.float32, "topk_score", 3)
+    B, Q, HI, _ = q.shape
+    n_blocks = blocks.shape[-1]
+    _check(lib().csa2_reindex_static(_ptr(q), _ptr(w), _ptr(ik_pool), ik_pool.shape[0], _ptr(seq_base),
+                                     _ptr(n_vis), _ptr(blocks), n_blocks, block, B, Q, HI, K, _ptr(topk),
+                                     _ptr(topk_score), _ptr(dev_status), _stream(stream)),
+           "csa2_reindex_static")
 
 
 # ---- a6/a7 ------------------------------------------------------------------------------
