@@ -206,6 +206,7 @@ __device__ __forceinline__ void store_slot(uint8_t* Ks, int r, int hf, const Slo
 
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
   chain_enter();
+  // phase: started
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = tc::align_smem_1024(smem_raw);
@@ -419,8 +420,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
     float mr[kMaxCluster], lr[kMaxCluster];
 #pragma unroll
     for (int c = 0; c < kMaxCluster; ++c) {
-      mr[c] = c < C ? cluster.map_shared_rank(m_run, c)[hh] : -INFINITY;
-      lr[c] = c < C ? cluster.map_shared_rank(l_run, c)[hh] : 0.0f;
+      mr[c] = c < C ? __uint_as_float(tc::ld_cluster_u32(tc::mapa(tc::smem_u32(m_run + hh), (uint32_t)c))) : -INFINITY;
+      lr[c] = c < C ? __uint_as_float(tc::ld_cluster_u32(tc::mapa(tc::smem_u32(l_run + hh), (uint32_t)c))) : 0.0f;
     }
     float M = -INFINITY;
 #pragma unroll
@@ -441,6 +442,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
   // of a pass is loaded before any is used, so a pass costs one interconnect round trip
   const int d4 = tid & 127;
   const int nh = h1 - h0;
+  const uint32_t of_a = tc::smem_u32(Of);
   for (int hb = tid >> 7; hb < nh; hb += 8) {
     float4 o[4][kMaxCluster];
 #pragma unroll
@@ -449,7 +451,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
 #pragma unroll
       for (int c = 0; c < kMaxCluster; ++c)
         o[u][c] = (hl < nh && c < C && fac[c * 64 + hl] > 0.0f)
-                      ? reinterpret_cast<const float4*>(cluster.map_shared_rank(Of, c) + (h0 + hl) * kD)[d4]
+                      ? tc::ld_cluster_f32x4(tc::mapa(of_a + (uint32_t)(((h0 + hl) * kD + 4 * d4) * 4), (uint32_t)c))
                       : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll

@@ -649,9 +649,23 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
 constexpr int kSelThreads = 512;
 constexpr int kPer = 32;                         // keys per thread per register chunk
 constexpr int kSelChunk = kSelThreads * kPer;    // keys per CTA per chunk (16384)
-constexpr int kBins = 2048;
+constexpr int kDigitBits = 10;                   // radix digit: 1024 bins
+constexpr int kBins = 1 << kDigitBits;
 constexpr int kMaxCluster = 8;
-constexpr int kSelSmem = 2 * kBins * 4 + 64 * 4 + 64 * 4;
+constexpr int kKeyRow = kPer + 1;                // a thread's keys in shared memory, padded
+// Shared memory, in 32-bit words:
+//   sub   [kBins/2][32]: per-lane counters, two 16-bit bins per word (bin 2c in the low
+//         half of column c); once the levels are done, the selected items are staged here
+//   ks    [kSelThreads][kKeyRow]: the chunk of keys, thread t's 32 keys in row t (the pad
+//         word puts key e of consecutive threads in consecutive banks)
+//   hist  [kBins] this CTA's histogram;  hsum [kBins] the cluster's
+//   scan scratch (32 x u64), cluster exchange words (16) and misc (8), padded to 64 words
+//   blk   [CSA2_MAX_K] the query's Reindex block ids
+// A lane counts at most 32 keys per 16,384-key chunk, and a CTA holds at most 2^27 / 8 keys
+// (the host caps max_n_vis at 2^27), so a 16-bit counter holds at most 32 * 1024 = 2^15.
+constexpr int kSubWords = kBins / 2 * 32;
+constexpr int kKeyWords = kSelThreads * kKeyRow;
+constexpr int kSelSmem = (kSubWords + kKeyWords + 2 * kBins + 64 + 64 + CSA2_MAX_K) * 4;
 
 struct SelectArgs {
   const uint32_t* keys;
@@ -668,9 +682,11 @@ struct SelectArgs {
   float* out_score;
 };
 
-__device__ __forceinline__ int64_t item_label(const SelectArgs& a, int bq, int64_t i) {
+// Entry index of item i (Reindex: slot i of the candidate pool; blk = the query's block
+// ids, staged in shared memory).
+__device__ __forceinline__ int64_t item_label(const SelectArgs& a, const int32_t* blk, int64_t i) {
   if (a.mode == kReindex) {
-    const int32_t c = a.blocks[(int64_t)bq * a.n_blocks + (i >> a.block_shift)];
+    const int32_t c = blk[i >> a.block_shift];
     return ((int64_t)c << a.block_shift) + (i & (a.block - 1));
   }
   return i;
@@ -707,27 +723,34 @@ __device__ __forceinline__ uint64_t block_excl_scan64(uint64_t v, uint64_t* ws, 
   return r;
 }
 
-// Bin of hist[0, nb) holding the need-th largest counted key, by the whole block: each
-// thread sums a run of nb/kSelThreads bins, a block-wide prefix over the runs from the
-// top finds the run, and its thread walks it.  ws: scan scratch (kSelThreads/32 + 1).
-__device__ __forceinline__ void find_bin(const uint32_t* hist, int nb, uint32_t need, uint32_t* T_out,
-                                         uint32_t* above_out, uint64_t* ws) {
-  const int tid = threadIdx.x;
-  const int per = nb >= kSelThreads ? nb / kSelThreads : 1;
-  // runs are numbered from the top bins down, so an exclusive prefix counts keys above
-  const int run_id = tid;
-  const int top = nb - 1 - run_id * per;  // highest bin of this run
-  uint32_t run = 0;
-  if (top >= 0)
-    for (int i = 0; i < per; ++i) run += hist[top - i];
-  uint64_t total;
-  const uint32_t above = (uint32_t)block_excl_scan64(run, ws, &total);
-  if (top >= 0 && above < need && above + run >= need) {
+// Bin of hist[0, nb) (nb <= kBins) holding the need-th largest counted key, by one warp:
+// lane l sums the R = max(nb/32, 1) bins nb-1-lR down to nb-R-lR, an inclusive scan over
+// the lanes (top bins first) finds the lane whose run reaches need, and that lane walks
+// its run.  The caller guarantees need <= the total count.
+__device__ __forceinline__ void find_bin_warp(const uint32_t* hist, int nb, uint32_t need, uint32_t* T_out,
+                                              uint32_t* above_out) {
+  const int lane = threadIdx.x & 31;
+  const int R = nb >= 32 ? nb >> 5 : 1;
+  const int top = nb - 1 - lane * R;
+  uint32_t run = 0u;
+#pragma unroll 8
+  for (int i = 0; i < R; ++i) {  // rotated by the lane so the lanes' reads fall in different banks
+    const int ii = (i + lane) & (R - 1);
+    run += top - ii >= 0 ? hist[top - ii] : 0u;
+  }
+  uint32_t inc = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  const uint32_t above = inc - run;
+  if (above < need && inc >= need) {
     uint32_t acc = above;
-    for (int i = 0; i < per; ++i) {
+    for (int i = 0; i < R; ++i) {
       const uint32_t h = hist[top - i];
       if (acc + h >= need) {
-        *T_out = top - i;
+        *T_out = (uint32_t)(top - i);
         *above_out = acc;
         break;
       }
@@ -736,18 +759,22 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, int nb, uint32_t 
   }
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
+__global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
   chain_enter();
+  // phase: started
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ __align__(16) uint32_t sel_smem[];
-  uint32_t* hist = sel_smem;                 // [kBins] this CTA's histogram
+  uint32_t* sub = sel_smem;                  // [kBins/2][32] per-lane counters; then staging
+  uint32_t* ks = sub + kSubWords;            // [kSelThreads][kKeyRow] keys of the chunk
+  uint32_t* hist = ks + kKeyWords;           // [kBins] this CTA's histogram
   uint32_t* hsum = hist + kBins;             // [kBins] cluster-summed histogram
   uint64_t* scan_ws = reinterpret_cast<uint64_t*>(hsum + kBins);  // [17]
   uint32_t* xch = reinterpret_cast<uint32_t*>(scan_ws + 32);       // [16] values exported to the cluster
   uint32_t* misc = xch + 16;                                        // [8]
+  int32_t* blk = reinterpret_cast<int32_t*>(misc + 8);              // [n_blocks] Reindex block ids
 
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31;
   const int rank = (int)cluster.block_rank();
   const int C = a.csize;
   const int bq = blockIdx.y;
@@ -755,6 +782,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
   const int K = a.K;
   int32_t* out = a.out_idx + (int64_t)bq * K;
   float* out_s = a.out_score ? a.out_score + (int64_t)bq * K : nullptr;
+  // shared::cluster address of `src` in CTA r
+  auto remote = [&](const uint32_t* src, int r) { return tc::mapa(tc::smem_u32(src), (uint32_t)r); };
 
   int64_t n;
   {
@@ -775,22 +804,35 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
   const int64_t hi = lo + slice < n ? lo + slice : n;
   const int nchunks = hi > lo ? (int)((hi - lo + kSelChunk - 1) / kSelChunk) : 0;
 
-  uint32_t k[kPer];
+  if (a.mode == kReindex)  // read back with the labels of the selected items (barriers follow)
+    for (int i = tid; i < a.n_blocks; i += kSelThreads) blk[i] = a.blocks[(int64_t)bq * a.n_blocks + i];
+  for (int i = tid; i < kSubWords / 4; i += kSelThreads)  // counters start at zero
+    reinterpret_cast<uint4*>(sub)[i] = make_uint4(0u, 0u, 0u, 0u);
+
+  // chunk ch of the slice -> ks (item lo + ch*16384 + 32t + e is key e of thread t; 0 past hi)
+  const uint32_t* mk = ks + tid * kKeyRow;
   auto load_chunk = [&](int ch) {
-    const int64_t i0 = lo + (int64_t)ch * kSelChunk + (int64_t)tid * kPer;
-    if (i0 + kPer <= hi) {
-#pragma unroll
-      for (int v = 0; v < kPer / 4; ++v) {
-        const uint4 a4 = *reinterpret_cast<const uint4*>(keys + i0 + 4 * v);
-        k[4 * v] = a4.x;
-        k[4 * v + 1] = a4.y;
-        k[4 * v + 2] = a4.z;
-        k[4 * v + 3] = a4.w;
+    const int64_t c0 = lo + (int64_t)ch * kSelChunk;
+    const int64_t cn = hi - c0 < kSelChunk ? hi - c0 : kSelChunk;
+    __syncthreads();  // earlier readers of ks are done
+#pragma unroll 2
+    for (int i4 = tid; i4 < kSelChunk / 4; i4 += kSelThreads) {
+      const int i = 4 * i4;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (i + 4 <= cn) {
+        v = *reinterpret_cast<const uint4*>(keys + c0 + i);
+      } else if (i < cn) {
+        v.x = keys[c0 + i];
+        v.y = i + 1 < cn ? keys[c0 + i + 1] : 0u;
+        v.z = i + 2 < cn ? keys[c0 + i + 2] : 0u;
       }
-    } else {
-#pragma unroll
-      for (int e = 0; e < kPer; ++e) k[e] = (i0 + e < hi) ? keys[i0 + e] : 0u;
+      uint32_t* d = ks + (i >> 5) * kKeyRow + (i & 31);
+      d[0] = v.x;
+      d[1] = v.y;
+      d[2] = v.z;
+      d[3] = v.w;
     }
+    __syncthreads();
   };
   if (nchunks == 1) load_chunk(0);
   // phase: keys loaded
@@ -799,11 +841,12 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u, cnt = 0u;
   for (int ch = 0; ch < nchunks; ++ch) {
     if (nchunks > 1) load_chunk(ch);
-#pragma unroll
+#pragma unroll 4
     for (int e = 0; e < kPer; ++e) {
-      if (k[e] != 0u) {
-        kmin = min(kmin, k[e]);
-        kmax = max(kmax, k[e]);
+      const uint32_t key = mk[e];
+      if (key != 0u) {
+        kmin = min(kmin, key);
+        kmax = max(kmax, key);
         ++cnt;
       }
     }
@@ -816,22 +859,27 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
   }
   if (tid < 16) xch[tid] = (tid == 0) ? 0xFFFFFFFFu : 0u;
   __syncthreads();
-  if ((tid & 31) == 0) {
+  if (lane == 0) {
     atomicMin(&xch[0], kmin);
     atomicMax(&xch[1], kmax);
     atomicAdd(&xch[2], cnt);
   }
-  cluster.sync();
+  if (C == 1) __syncthreads();
+  else cluster.sync();
   uint32_t gmin = 0xFFFFFFFFu, gmax = 0u, gcnt = 0u;
   // phase: range reduced
-  {
+  if (C == 1) {
+    gmin = xch[0];
+    gmax = xch[1];
+    gcnt = xch[2];
+  } else {
     uint32_t v[kMaxCluster][3];
 #pragma unroll
     for (int r = 0; r < kMaxCluster; ++r) {
-      const uint32_t* rx = cluster.map_shared_rank(xch, r < C ? r : 0);
-      v[r][0] = rx[0];
-      v[r][1] = rx[1];
-      v[r][2] = r < C ? rx[2] : 0u;
+      const uint32_t ra = remote(xch, r < C ? r : 0);
+      v[r][0] = tc::ld_cluster_u32(ra);
+      v[r][1] = tc::ld_cluster_u32(ra + 4);
+      v[r][2] = r < C ? tc::ld_cluster_u32(ra + 8) : 0u;
     }
 #pragma unroll
     for (int r = 0; r < kMaxCluster; ++r) {
@@ -853,46 +901,63 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
       mask = p == 31 ? 0u : ~((2u << p) - 1u);
       prefix = gmin & mask;
       for (;;) {
-        const int sh = p >= 10 ? p - 10 : 0;
+        const int sh = p >= kDigitBits - 1 ? p - (kDigitBits - 1) : 0;
         const int width = p - sh + 1;
         const uint32_t nb = 1u << width;
-        for (int i = tid; i < (int)nb; i += kSelThreads) hist[i] = 0u;
-        __syncthreads();
+        // each lane counts into its own column, so a warp's increments never collide
+        // (keys of similar scores share bins)
         for (int ch = 0; ch < nchunks; ++ch) {
           if (nchunks > 1) load_chunk(ch);
-#pragma unroll
-          for (int e = 0; e < kPer; ++e)
-            if (k[e] != 0u && (k[e] & mask) == prefix) atomicAdd(&hist[(k[e] >> sh) & (nb - 1u)], 1u);
-        }
-        cluster.sync();  // every CTA's histogram complete
-        for (int i0 = 0; i0 < (int)nb; i0 += kSelThreads * 4) {  // 4 bins per thread per pass
-          uint32_t v[4][kMaxCluster];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u * kSelThreads + tid;
-#pragma unroll
-            for (int r = 0; r < kMaxCluster; ++r)
-              v[u][r] = (r < C && i < (int)nb) ? cluster.map_shared_rank(hist, r)[i] : 0u;
-          }
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u * kSelThreads + tid;
-            uint32_t sum = 0u;
-#pragma unroll
-            for (int r = 0; r < kMaxCluster; ++r) sum += v[u][r];
-            if (i < (int)nb) hsum[i] = sum;
+#pragma unroll 4
+          for (int e = 0; e < kPer; ++e) {
+            const uint32_t key = mk[e];
+            if (key != 0u && (key & mask) == prefix) {
+              const uint32_t bin = (key >> sh) & (nb - 1u);
+              atomicAdd(&sub[(bin >> 1) * 32 + lane], (bin & 1u) ? 0x10000u : 1u);
+            }
           }
         }
         __syncthreads();
-        find_bin(hsum, (int)nb, need, &misc[0], &misc[1], scan_ws);
+        // bin totals: thread c sums column c, reading word (j + c) % 32 at step j so that
+        // the 32 lanes of a warp read 32 different banks; the column is zeroed behind it
+        for (int c = tid; c < (int)(nb >> 1); c += kSelThreads) {
+          uint32_t* col = sub + c * 32;
+          uint32_t lo16 = 0u, hi16 = 0u;
+#pragma unroll 4
+          for (int j = 0; j < 32; ++j) {
+            const int w = (j + c) & 31;
+            const uint32_t x = col[w];
+            col[w] = 0u;
+            lo16 += x & 0xFFFFu;
+            hi16 += x >> 16;
+          }
+          hist[2 * c] = lo16;
+          hist[2 * c + 1] = hi16;
+        }
+        const uint32_t* hs = hist;
+        if (C > 1) {  // sum every CTA's histogram
+          cluster.sync();
+          for (int i = tid; i < (int)nb; i += kSelThreads) {
+            uint32_t v[kMaxCluster];
+#pragma unroll
+            for (int r = 0; r < kMaxCluster; ++r) v[r] = r < C ? tc::ld_cluster_u32(remote(hist, r) + 4u * i) : 0u;
+            uint32_t sum = 0u;
+#pragma unroll
+            for (int r = 0; r < kMaxCluster; ++r) sum += v[r];
+            hsum[i] = sum;
+          }
+          hs = hsum;
+        }
+        __syncthreads();
+        if (tid < 32) find_bin_warp(hs, (int)nb, need, &misc[0], &misc[1]);
         __syncthreads();
         const uint32_t T = misc[0];
         need -= misc[1];
         prefix |= T << sh;
         mask |= (nb - 1u) << sh;
-        const uint32_t inbin = hsum[T];
-        cluster.sync();  // remote reads of `hist` done before it is reused
-        if (inbin == need) break;  // every key of the bin is selected
+        const uint32_t inbin = hs[T];
+        if (C > 1) cluster.sync();  // remote reads of `hist` done before it is rewritten
+        if (inbin == need) break;   // every key of the bin is selected
         if (sh == 0) break;
         p = sh - 1;
       }
@@ -910,10 +975,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
   uint32_t my_gt = 0u, my_eq = 0u;
   for (int ch = 0; ch < nchunks; ++ch) {
     if (nchunks > 1) load_chunk(ch);
-#pragma unroll
+#pragma unroll 4
     for (int e = 0; e < kPer; ++e) {
       bool gt, eq;
-      classify(k[e], gt, eq);
+      classify(mk[e], gt, eq);
       my_gt += gt;
       my_eq += eq;
     }
@@ -924,16 +989,18 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
     xch[4] = (uint32_t)tot;
     xch[5] = (uint32_t)(tot >> 32);
   }
-  cluster.sync();
-  uint32_t cta_gt = 0u, cta_eq = 0u, all_gt = 0u;
-  {
+  if (C == 1) __syncthreads();
+  else cluster.sync();
+  uint32_t cta_gt = 0u, cta_eq = 0u, all_gt = (uint32_t)tot;
+  if (C > 1) {
     uint32_t g[kMaxCluster], q[kMaxCluster];
 #pragma unroll
     for (int r = 0; r < kMaxCluster; ++r) {
-      const uint32_t* rx = cluster.map_shared_rank(xch, r < C ? r : 0);
-      g[r] = r < C ? rx[4] : 0u;
-      q[r] = r < C ? rx[5] : 0u;
+      const uint32_t ra = remote(xch, r < C ? r : 0);
+      g[r] = r < C ? tc::ld_cluster_u32(ra + 16) : 0u;
+      q[r] = r < C ? tc::ld_cluster_u32(ra + 20) : 0u;
     }
+    all_gt = 0u;
 #pragma unroll
     for (int r = 0; r < kMaxCluster; ++r) {
       if (r < rank) {
@@ -943,29 +1010,42 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
       all_gt += g[r];
     }
   }
-  uint32_t pg = cta_gt + (uint32_t)mine;
   // phase: positions known
-  uint32_t pe = cta_eq + (uint32_t)(mine >> 32);
+  // This CTA's selected keys go to out[cta_gt, cta_gt + G) in index order, and its first
+  // e_take keys equal to the threshold to out[tie0 + cta_eq, ...): staged in shared memory
+  // in that order, then copied out with consecutive threads on consecutive slots.
+  const uint32_t G = (uint32_t)tot, E = (uint32_t)(tot >> 32);
   const uint32_t tie0 = (uint32_t)K - need;  // first slot of the equal keys
+  const uint32_t e_take = need > cta_eq ? min(E, need - cta_eq) : 0u;
+  int32_t* s_idx = reinterpret_cast<int32_t*>(sub);  // [G + e_take <= K]
+  float* s_sc = reinterpret_cast<float*>(sub + CSA2_MAX_K);
+  uint32_t lg = (uint32_t)mine, le = (uint32_t)(mine >> 32);
   for (int ch = 0; ch < nchunks; ++ch) {
     if (nchunks > 1) load_chunk(ch);
     const int64_t i0 = lo + (int64_t)ch * kSelChunk + (int64_t)tid * kPer;
-#pragma unroll
+#pragma unroll 2
     for (int e = 0; e < kPer; ++e) {
+      const uint32_t key = mk[e];
       bool gt, eq;
-      classify(k[e], gt, eq);
+      classify(key, gt, eq);
       if (gt) {
-        out[pg] = (int32_t)item_label(a, bq, i0 + e);
-        if (out_s) out_s[pg] = key_score(k[e]);
-        ++pg;
+        s_idx[lg] = (int32_t)item_label(a, blk, i0 + e);
+        s_sc[lg] = key_score(key);
+        ++lg;
       } else if (eq) {
-        if (pe < need) {
-          out[tie0 + pe] = (int32_t)item_label(a, bq, i0 + e);
-          if (out_s) out_s[tie0 + pe] = key_score(k[e]);
+        if (le < e_take) {
+          s_idx[G + le] = (int32_t)item_label(a, blk, i0 + e);
+          s_sc[G + le] = key_score(key);
         }
-        ++pe;
+        ++le;
       }
     }
+  }
+  __syncthreads();
+  for (uint32_t i = tid; i < G + e_take; i += kSelThreads) {
+    const uint32_t slot = i < G ? cta_gt + i : tie0 + cta_eq + (i - G);
+    out[slot] = s_idx[i];
+    if (out_s) out_s[slot] = s_sc[i];
   }
   // phase: written
   if (all_valid && rank == 0) {
@@ -974,7 +1054,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
       if (out_s) out_s[i] = -INFINITY;
     }
   }
-  cluster.sync();  // keep every CTA's shared memory alive until remote reads are done
+  if (C > 1) cluster.sync();  // keep every CTA's shared memory alive until remote reads are done
 }
 
 // ------------------------------------------------------------------------------------
@@ -1145,6 +1225,8 @@ cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t
                                         : (int64_t)n_blocks * block;
   int64_t c = (items + kSelChunk - 1) / kSelChunk;  // one CTA per 16384 keys
   s.csize = (int)(c < 1 ? 1 : (c > kMaxCluster ? kMaxCluster : c));
+  e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelSmem);
+  if (e != cudaSuccess) return e;
   e = launch_chained(select_kernel, dim3((unsigned)s.csize, (unsigned)BQ), dim3(kSelThreads), kSelSmem, stream,
                      (unsigned)s.csize, s);
   if (e != cudaSuccess) return e;
