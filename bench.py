@@ -295,6 +295,12 @@ def run_ours(args, world, rank, local):
     return line, wl, x
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the call's
+# dominant kernel, from an ncu capture of that kernel as it is now, per workload; a kernel
+# that changes drops out of this table until it is captured again.
+NCU_DRAM_BYTES_PER_LAUNCH = {("hier1m", "attn"): 1642240}
+
+
 def roofline(wl, per_call, counts, steps):
     peaks = load_peaks()
     dom = max(per_call, key=lambda k: per_call[k])
@@ -309,6 +315,7 @@ def roofline(wl, per_call, counts, steps):
         achieved = flops / (avg_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16"], "unit": "TFLOP/s",
                 "frac": round(achieved / peaks["bf16"], 4), "traffic": None}
+    roof["traffic"] = NCU_DRAM_BYTES_PER_LAUNCH.get((wl.name, dom))
     roof.update({"kernel": kernel_info["kernel"], "call": dom, "avg_launch_ms": round(avg_ms, 4),
                  "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
                  "peak_src": peaks["src"] + (" (bf16 sustained; f16 has the same nominal rate)"
@@ -318,8 +325,8 @@ def roofline(wl, per_call, counts, steps):
 
 def dominant_kernel_info(call):
     return {
-        "index_hier": {"kernel": "scan_tc_kernel<hier> + select_kernel", "bound": "hbm"},
-        "index_full": {"kernel": "scan_tc_kernel<flat> + select_kernel", "bound": "hbm"},
+        "index_hier": {"kernel": "stream_scan_kernel<hier> + select_kernel", "bound": "hbm"},
+        "index_full": {"kernel": "stream_scan_kernel<flat> + select_kernel", "bound": "hbm"},
         "reindex": {"kernel": "scan_tc_kernel<reindex> + select_kernel", "bound": "hbm"},
         "attn": {"kernel": "attn_tc_kernel", "bound": "tensor"},
         "pack": {"kernel": "pack_kv_kernel", "bound": "hbm"},
