@@ -116,7 +116,7 @@ csa2_status csa2_pack_kv(const void* kv, const void* ik, int64_t T, int ratio,
  *   q    fp32 [B][Q][HI][128]  indexer queries;  w  fp32 [B][Q][HI]  head weights
  *   ik_pool u8 [pool_entries][68];  seq_base int64 [B];  n_vis int32 [B][Q]
  *   max_n_vis  host-side upper bound on every n_vis (sizes the grid and workspace),
- *              at most 2^27
+ *              at most 2^23
  *   topk int32 [B][Q][K]  out: the K best visible entries (indices relative to
  *        seq_base), -1 in unused slots; topk_score fp32 [B][Q][K] (may be NULL)
  *

@@ -265,6 +265,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
   // phase: queries landed
   {  // fp32 staging -> f16 query tile (scaled), 8 channels per 16 B chunk
     const float qscale = a.sm_scale * 1.4426950408889634f;
+#pragma unroll 4
     for (int i = tid; i < kHeadsPad * 64; i += kAttnThreads) {
       const int h = i >> 6, ch = i & 63, db = ch >> 3, c = ch & 7;
       uint4 v = make_uint4(0u, 0u, 0u, 0u);

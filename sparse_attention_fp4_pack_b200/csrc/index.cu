@@ -646,8 +646,9 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
 //      to the K-th (all bits resolved) lowest index first.
 // The result (contents and order) is deterministic.
 // ------------------------------------------------------------------------------------
-constexpr int kSelThreads = 512;
-constexpr int kPer = 32;                         // keys per thread per register chunk
+constexpr int kSelThreads = 1024;
+constexpr int kPerShift = 4;
+constexpr int kPer = 1 << kPerShift;             // keys per thread per chunk
 constexpr int kSelChunk = kSelThreads * kPer;    // keys per CTA per chunk (16384)
 constexpr int kDigitBits = 10;                   // radix digit: 1024 bins
 constexpr int kBins = 1 << kDigitBits;
@@ -656,16 +657,18 @@ constexpr int kKeyRow = kPer + 1;                // a thread's keys in shared me
 // Shared memory, in 32-bit words:
 //   sub   [kBins/2][32]: per-lane counters, two 16-bit bins per word (bin 2c in the low
 //         half of column c); once the levels are done, the selected items are staged here
-//   ks    [kSelThreads][kKeyRow]: the chunk of keys, thread t's 32 keys in row t (the pad
+//   ks    [kSelThreads][kKeyRow]: the chunk of keys, thread t's kPer keys in row t (the pad
 //         word puts key e of consecutive threads in consecutive banks)
 //   hist  [kBins] this CTA's histogram;  hsum [kBins] the cluster's
 //   scan scratch (32 x u64), cluster exchange words (16) and misc (8), padded to 64 words
 //   blk   [CSA2_MAX_K] the query's Reindex block ids
-// A lane counts at most 32 keys per 16,384-key chunk, and a CTA holds at most 2^27 / 8 keys
-// (the host caps max_n_vis at 2^27), so a 16-bit counter holds at most 32 * 1024 = 2^15.
+// Column l collects lane l of every warp: at most 32 warps x 16 keys = 512 increments per
+// 16,384-key chunk.  launch_index gives a query one CTA per 16,384 keys, up to 8, and the
+// host caps max_n_vis at 2^23, so a CTA holds at most 2^20 keys (64 chunks) and a 16-bit
+// counter reaches at most 64 x 512 = 2^15.
 constexpr int kSubWords = kBins / 2 * 32;
 constexpr int kKeyWords = kSelThreads * kKeyRow;
-constexpr int kSelSmem = (kSubWords + kKeyWords + 2 * kBins + 64 + 64 + CSA2_MAX_K) * 4;
+constexpr int kSelSmem = (kSubWords + kKeyWords + 2 * kBins + 128 + 64 + CSA2_MAX_K) * 4;
 
 struct SelectArgs {
   const uint32_t* keys;
@@ -769,8 +772,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
   uint32_t* ks = sub + kSubWords;            // [kSelThreads][kKeyRow] keys of the chunk
   uint32_t* hist = ks + kKeyWords;           // [kBins] this CTA's histogram
   uint32_t* hsum = hist + kBins;             // [kBins] cluster-summed histogram
-  uint64_t* scan_ws = reinterpret_cast<uint64_t*>(hsum + kBins);  // [17]
-  uint32_t* xch = reinterpret_cast<uint32_t*>(scan_ws + 32);       // [16] values exported to the cluster
+  uint64_t* scan_ws = reinterpret_cast<uint64_t*>(hsum + kBins);  // [kSelThreads/32 + 1]
+  uint32_t* xch = reinterpret_cast<uint32_t*>(scan_ws + 64);       // [16] values exported to the cluster
   uint32_t* misc = xch + 16;                                        // [8]
   int32_t* blk = reinterpret_cast<int32_t*>(misc + 8);              // [n_blocks] Reindex block ids
 
@@ -811,7 +814,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
 
   // chunk ch of the slice -> ks (item lo + ch*16384 + 32t + e is key e of thread t; 0 past hi)
   const uint32_t* mk = ks + tid * kKeyRow;
-  auto load_chunk = [&](int ch) {
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u, cnt = 0u;  // over the valid (non-zero) keys
+  auto load_chunk = [&](int ch, bool range) {
     const int64_t c0 = lo + (int64_t)ch * kSelChunk;
     const int64_t cn = hi - c0 < kSelChunk ? hi - c0 : kSelChunk;
     __syncthreads();  // earlier readers of ks are done
@@ -826,7 +830,18 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
         v.y = i + 1 < cn ? keys[c0 + i + 1] : 0u;
         v.z = i + 2 < cn ? keys[c0 + i + 2] : 0u;
       }
-      uint32_t* d = ks + (i >> 5) * kKeyRow + (i & 31);
+      if (range) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (w[u] != 0u) {
+            kmin = min(kmin, w[u]);
+            kmax = max(kmax, w[u]);
+            ++cnt;
+          }
+        }
+      }
+      uint32_t* d = ks + (i >> kPerShift) * kKeyRow + (i & (kPer - 1));
       d[0] = v.x;
       d[1] = v.y;
       d[2] = v.z;
@@ -834,23 +849,9 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
     }
     __syncthreads();
   };
-  if (nchunks == 1) load_chunk(0);
+  // ---- 0. cluster-wide min / max / count of valid keys, taken while loading -------------
+  for (int ch = 0; ch < nchunks; ++ch) load_chunk(ch, true);  // a single chunk stays loaded
   // phase: keys loaded
-
-  // ---- 0. cluster-wide min / max / count of valid keys --------------------------------
-  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u, cnt = 0u;
-  for (int ch = 0; ch < nchunks; ++ch) {
-    if (nchunks > 1) load_chunk(ch);
-#pragma unroll 4
-    for (int e = 0; e < kPer; ++e) {
-      const uint32_t key = mk[e];
-      if (key != 0u) {
-        kmin = min(kmin, key);
-        kmax = max(kmax, key);
-        ++cnt;
-      }
-    }
-  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
@@ -907,7 +908,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
         // each lane counts into its own column, so a warp's increments never collide
         // (keys of similar scores share bins)
         for (int ch = 0; ch < nchunks; ++ch) {
-          if (nchunks > 1) load_chunk(ch);
+          if (nchunks > 1) load_chunk(ch, false);
 #pragma unroll 4
           for (int e = 0; e < kPer; ++e) {
             const uint32_t key = mk[e];
@@ -974,7 +975,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
   };
   uint32_t my_gt = 0u, my_eq = 0u;
   for (int ch = 0; ch < nchunks; ++ch) {
-    if (nchunks > 1) load_chunk(ch);
+    if (nchunks > 1) load_chunk(ch, false);
 #pragma unroll 4
     for (int e = 0; e < kPer; ++e) {
       bool gt, eq;
@@ -1021,7 +1022,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
   float* s_sc = reinterpret_cast<float*>(sub + CSA2_MAX_K);
   uint32_t lg = (uint32_t)mine, le = (uint32_t)(mine >> 32);
   for (int ch = 0; ch < nchunks; ++ch) {
-    if (nchunks > 1) load_chunk(ch);
+    if (nchunks > 1) load_chunk(ch, false);
     const int64_t i0 = lo + (int64_t)ch * kSelChunk + (int64_t)tid * kPer;
 #pragma unroll 2
     for (int e = 0; e < kPer; ++e) {

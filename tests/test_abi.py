@@ -78,8 +78,8 @@ def test_index_rejects_bad_args(L):
     assert L.csa2_index_full(*args(8, 512, FAKE, 16)) == 1         # workspace too small
     assert L.csa2_index_full(*args(8, 512, None, 1 << 20)) == 1    # null workspace
     assert L.csa2_index_full(*args(8, 512, P(0x10010), 1 << 20)) == 1  # workspace not 256-aligned
-    big = (FAKE, FAKE, FAKE, 1 << 28, FAKE, FAKE, 1, 1, 8, 512, (1 << 27) + 1, FAKE, None, FAKE, 1 << 40, None, st)
-    assert L.csa2_index_full(*big) == 2                              # max_n_vis above 2^27
+    big = (FAKE, FAKE, FAKE, 1 << 28, FAKE, FAKE, 1, 1, 8, 512, (1 << 23) + 1, FAKE, None, FAKE, 1 << 40, None, st)
+    assert L.csa2_index_full(*big) == 2                              # max_n_vis above 2^23
     assert L.csa2_index_hier(FAKE, FAKE, FAKE, 100, FAKE, FAKE, 1, 1, 8, 2048, 3, 100, FAKE, None, FAKE,
                              1 << 20, None, st) == 2                # block not a power of two
     assert L.csa2_index_hier(FAKE, FAKE, FAKE, 100, FAKE, FAKE, 1, 1, 8, 4096, 8, 100, FAKE, None, FAKE,
