@@ -727,9 +727,10 @@ __device__ __forceinline__ uint64_t block_excl_scan64(uint64_t v, uint64_t* ws, 
 }
 
 // Bin of hist[0, nb) (nb <= kBins) holding the need-th largest counted key, by one warp:
-// lane l sums the R = max(nb/32, 1) bins nb-1-lR down to nb-R-lR, an inclusive scan over
-// the lanes (top bins first) finds the lane whose run reaches need, and that lane walks
-// its run.  The caller guarantees need <= the total count.
+// lane l sums the R = max(nb/32, 1) bins nb-1-lR down to nb-R-lR; an inclusive scan over
+// the lanes (top bins first) finds the lane whose run reaches need; then the whole warp
+// scans that run (lane i takes its i-th bin from the top) and a ballot finds the bin.  The
+// caller guarantees 1 <= need <= the total count.
 __device__ __forceinline__ void find_bin_warp(const uint32_t* hist, int nb, uint32_t need, uint32_t* T_out,
                                               uint32_t* above_out) {
   const int lane = threadIdx.x & 31;
@@ -748,17 +749,25 @@ __device__ __forceinline__ void find_bin_warp(const uint32_t* hist, int nb, uint
     if (lane >= o) inc += y;
   }
   const uint32_t above = inc - run;
-  if (above < need && inc >= need) {
-    uint32_t acc = above;
-    for (int i = 0; i < R; ++i) {
-      const uint32_t h = hist[top - i];
-      if (acc + h >= need) {
-        *T_out = (uint32_t)(top - i);
-        *above_out = acc;
-        break;
-      }
-      acc += h;
-    }
+  // the lane whose run reaches need, and the count above its run
+  const uint32_t hit = __ballot_sync(0xffffffffu, above < need && inc >= need);
+  const int wl = __ffs(hit) - 1;
+  const uint32_t w_above = __shfl_sync(0xffffffffu, above, wl);
+  const int w_top = nb - 1 - wl * R;
+  // lane i: i-th bin of that run from the top (R <= 32)
+  const int b = w_top - lane;
+  const uint32_t h = (lane < R && b >= 0) ? hist[b] : 0u;
+  uint32_t hinc = h;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, hinc, o);
+    if (lane >= o) hinc += y;
+  }
+  const uint32_t reach = __ballot_sync(0xffffffffu, lane < R && w_above + hinc >= need);
+  const int fl = __ffs(reach) - 1;
+  if (lane == fl) {
+    *T_out = (uint32_t)b;
+    *above_out = w_above + hinc - h;
   }
 }
 
@@ -935,6 +944,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
           hist[2 * c] = lo16;
           hist[2 * c + 1] = hi16;
         }
+  // phase: level counted
         const uint32_t* hs = hist;
         if (C > 1) {  // sum every CTA's histogram
           cluster.sync();
@@ -952,6 +962,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
         __syncthreads();
         if (tid < 32) find_bin_warp(hs, (int)nb, need, &misc[0], &misc[1]);
         __syncthreads();
+  // phase: level found
         const uint32_t T = misc[0];
         need -= misc[1];
         prefix |= T << sh;
