@@ -66,6 +66,7 @@ struct AttnArgs {
   int Q, H;
   float sm_scale;
   int n_tiles, csize;
+  int hgroups, hg_size;  // a query's heads in hgroups groups of hg_size, one cluster each
   float* out;
   float* lse;
   uint32_t* status;
@@ -226,9 +227,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rank = (int)cluster.block_rank();
   const int C = a.csize;
-  const int bq = blockIdx.y;
+  const int bq = blockIdx.y / a.hgroups;
   const int b = bq / a.Q;
-  const int H = a.H;
+  const int H = a.H;                                 // heads of the query (output layout)
+  const int h_base = (blockIdx.y % a.hgroups) * a.hg_size;
+  const int NH = min(a.hg_size, H - h_base);         // heads of this cluster, rows 0..NH-1
   const int64_t base = a.seq_base[b];
   const int64_t t = a.q_pos[bq];
   const uint32_t mbar_mma = tc::smem_u32(&mbar[0]), mbar_q = tc::smem_u32(&mbar[1]);
@@ -239,9 +242,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
   if (tid == 0) {
     tc::mbar_init(mbar_mma, 1);
     tc::mbar_init(mbar_q, 1);
-    const uint32_t bytes = (uint32_t)H * kD * 4;
+    const uint32_t bytes = (uint32_t)NH * kD * 4;
     tc::mbar_arrive_expect_tx(mbar_q, bytes);
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(a.q + (int64_t)bq * H * kD);
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(a.q + ((int64_t)bq * H + h_base) * kD);
     for (uint32_t off = 0; off < bytes; off += 32768)
       tc::bulk_g2s(tc::smem_u32(Ks) + off, src + off, bytes - off < 32768 ? bytes - off : 32768, mbar_q);
   }
@@ -269,7 +272,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
     for (int i = tid; i < kHeadsPad * 64; i += kAttnThreads) {
       const int h = i >> 6, ch = i & 63, db = ch >> 3, c = ch & 7;
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (h < H && !timed_out) {
+      if (h < NH && !timed_out) {
         const float4 x0 = *reinterpret_cast<const float4*>(Of + h * kD + ch * 8);
         const float4 x1 = *reinterpret_cast<const float4*>(Of + h * kD + ch * 8 + 4);
         v.x = half2_bits(x0.x * qscale, x0.y * qscale);
@@ -321,7 +324,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
     float s[32], v[32];
 #pragma unroll
     for (int jj = 0; jj < 32; ++jj) {
-      s[jj] = kv ? __uint_as_float(raw[jj]) : -INFINITY;
+      s[jj] = (kv && half * 32 + jj < NH) ? __uint_as_float(raw[jj]) : -INFINITY;  // pad heads: no keys
       v[jj] = s[jj];
     }
     red_max[q4 * 64 + half * 32 + lane] = xpose_reduce<true>(v, lane);
@@ -394,14 +397,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
   }
 
   // ---- export O^T (fp32 [head][channel]) into the key area --------------------------------
-  if (processed > 0 && !timed_out) {
+  if (processed > 0 && !timed_out && half * 32 < NH) {
 #pragma unroll 1
     for (int mt = 0; mt < 4; ++mt) {
       uint32_t o[32];
       tc::tmem_ld32(lane_base + kColO + mt * 64 + half * 32, o);
       const int d = mt * 128 + q4 * 32 + lane;
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) Of[(half * 32 + jj) * kD + d] = __uint_as_float(o[jj]);
+      for (int jj = 0; jj < 32; ++jj)
+        if (half * 32 + jj < NH) Of[(half * 32 + jj) * kD + d] = __uint_as_float(o[jj]);
     }
   }
   tc::fence_before_sync();
@@ -411,8 +415,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
   // ---- merge heads [h0, h1) across the cluster through distributed shared memory ----------
   // Remote loads are issued together (unrolled over the largest cluster), since each one
   // pays the cluster interconnect latency.
-  const int hpc = (H + C - 1) / C;
-  const int h0 = rank * hpc, h1 = h0 + hpc < H ? h0 + hpc : H;
+  const int hpc = (NH + C - 1) / C;
+  const int h0 = rank * hpc, h1 = h0 + hpc < NH ? h0 + hpc : NH;  // this cluster's head rows
   // the P^T tile is free once the last PV product has completed
   float* fac = reinterpret_cast<float*>(Ps);  // [kMaxCluster][64] merge factor of each CTA's partial
   float* linv = fac + kMaxCluster * 64;       // [64] 1 / merged sum
@@ -436,7 +440,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
       L = fmaf(lr[c], f, L);
     }
     linv[tid] = L > 0.0f ? 1.0f / L : 0.0f;
-    a.lse[(int64_t)bq * H + hh] = L > 0.0f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+    a.lse[(int64_t)bq * H + h_base + hh] = L > 0.0f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
   }
   __syncthreads();
   // thread -> (float4 column d4, heads hb, hb+2, hb+4, hb+6 per pass): every remote float4
@@ -469,7 +473,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
           acc.w = fmaf(o[u][c].w, f, acc.w);
         }
         const float inv = linv[hl];
-        reinterpret_cast<float4*>(a.out + ((int64_t)bq * H + h0 + hl) * kD)[d4] =
+        reinterpret_cast<float4*>(a.out + ((int64_t)bq * H + h_base + h0 + hl) * kD)[d4] =
             make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
       }
     }
@@ -520,9 +524,20 @@ cudaError_t launch_sparse_attn(const float* q, const uint8_t* kv_pool, int64_t p
   a.status = status;
   const int64_t BQ = (int64_t)B * Q;
   if (BQ == 0) return cudaSuccess;
+  // When the clusters do not fill the GPU, split each query's heads into groups of 16 or 32,
+  // one cluster per group: a CTA then converts, exports and merges only its group's heads.
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  a.hgroups = 1;
+  for (int g = 4; g >= 2; g >>= 1)
+    if (H % (16 * g) == 0 && BQ * a.csize * g <= sms) {
+      a.hgroups = g;
+      break;
+    }
+  a.hg_size = H / a.hgroups;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  e = launch_chained(attn_tc_kernel, dim3((unsigned)a.csize, (unsigned)BQ), dim3(kAttnThreads), kSmemBytes, stream,
+  e = launch_chained(attn_tc_kernel, dim3((unsigned)a.csize, (unsigned)(BQ * a.hgroups)), dim3(kAttnThreads), kSmemBytes, stream,
                      (unsigned)a.csize, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
