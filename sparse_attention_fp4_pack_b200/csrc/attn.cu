@@ -303,7 +303,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
     if (!any_valid) continue;
     // ---- S^T = Kt . Qs^T --------------------------------------------------------------------
     if (tid == 0) {
-      constexpr uint32_t idesc = tc::idesc_f16(kTile, kHeadsPad, false, false);
+      // N covers this cluster's heads only (rows past NH of the query tile are zero and the
+      // softmax masks those columns)
+      const uint32_t idesc = tc::idesc_f16(kTile, NH <= 16 ? 16 : (NH <= 32 ? 32 : kHeadsPad), false, false);
 #pragma unroll 4
       for (int ks = 0; ks < kD / 16; ++ks) {
         const int db = ks >> 2, kk = ks & 3;
