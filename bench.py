@@ -55,6 +55,8 @@ def parse_args():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--cpu-seqs", type=int, default=1, help="sequences in the oracle's timed sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-pack-throughput", action="store_true",
+                   help="skip the separate FP4 pack throughput measurement (2^20 tokens)")
     p.add_argument("--no-call-timing", action="store_true",
                    help="time the step without the per-call events (no breakdown or roofline)")
     return p.parse_args()
@@ -395,6 +397,39 @@ def oracle_step(wl, st):
                            sm, window=wl.window)
 
 
+def time_pack(steps, warmup, device):
+    """FP4 pack throughput on 2^20 new tokens (512-channel main KV + 128-dim indexer key,
+    bf16, resident in HBM) at 1:1 and 2:1: (bytes read + bytes written) / device time, L2
+    flushed between launches.  Inputs follow the pack workload's value recipe."""
+    import synth
+    from sparse_attention_fp4_pack_b200 import csa2
+    T = 1 << 20
+    kv, ik = synth.kv_tokens(1, T, device=device, recipe="rmsnorm")
+    kvp = torch.empty(T, 288, dtype=torch.uint8, device=device)
+    ikp = torch.empty(T, 68, dtype=torch.uint8, device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    res = {}
+    for ratio in (1, 2):
+        ms = 0.0
+        for i in range(warmup + steps):
+            flush.fill_(i)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            csa2.csa2_pack_kv(kv, ik, ratio, kvp, ikp)
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= warmup:
+                ms += e0.elapsed_time(e1)
+        ms /= steps
+        nbytes = T * 1280 + (T // ratio) * 356
+        res[f"{ratio}:1"] = {"GB/s": round(nbytes / (ms * 1e-3) / 1e9, 1), "us": round(ms * 1e3, 1),
+                             "bytes": nbytes}
+    del kv, ik, kvp, ikp, flush
+    torch.cuda.empty_cache()
+    return res
+
+
 def time_oracle(wl, nseq, steps, warmup, device):
     import oracle
     st = oracle_sample_state(wl, nseq, device)
@@ -432,9 +467,14 @@ def main():
             torch.distributed.destroy_process_group()
         return
     line, wl, x = run_ours(args, world, rank, local)
+    del x
+    torch.cuda.empty_cache()
+    if not args.no_pack_throughput:
+        pk = time_pack(5, 3, "cuda")
+        peak = load_peaks()["hbm"]
+        line["pack_throughput"] = {"tokens": 1 << 20, "unit": "GB/s", "peak": peak,
+                                   **{k: dict(v, frac=round(v["GB/s"] / peak, 3)) for k, v in pk.items()}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        del x
-        torch.cuda.empty_cache()
         v, cores, sample = time_oracle(wl, args.cpu_seqs, 1, 0, "cuda")
         line["cpu_baseline"] = {"value": round(v, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
                                 "sample": sample}

@@ -45,6 +45,10 @@ __global__ void __launch_bounds__(256) pack_kv_kernel(const uint16_t* __restrict
       if (lane == 0) flag(status, CSA2_DEV_BAD_INDEX);
       continue;
     }
+    // every load of the entry is issued before any arithmetic: one memory round trip
+    const uint2* pi = reinterpret_cast<const uint2*>(ik + (j * ratio) * kDI) + lane;
+    const uint2 ia = __ldcs(pi);
+    const uint2 ib = ratio == 1 ? make_uint2(0u, 0u) : __ldcs(pi + kDI / 4);
     // ---- main KV block `lane` -------------------------------------------------------
     float x[16];
     {
@@ -95,12 +99,11 @@ __global__ void __launch_bounds__(256) pack_kv_kernel(const uint16_t* __restrict
     // ---- indexer key dims 4*lane .. 4*lane+3 ------------------------------------------
     float y[4];
     {
-      const uint2* p0 = reinterpret_cast<const uint2*>(ik + (j * ratio) * kDI) + lane;
-      uint2 a = __ldcs(p0);
+      const uint2 a = ia;
       if (ratio == 1) {
         y[0] = bf16_lo(a.x); y[1] = bf16_hi(a.x); y[2] = bf16_lo(a.y); y[3] = bf16_hi(a.y);
       } else {
-        uint2 b = __ldcs(p0 + kDI / 4);
+        const uint2 b = ib;
         y[0] = (bf16_lo(a.x) + bf16_lo(b.x)) * 0.5f;
         y[1] = (bf16_hi(a.x) + bf16_hi(b.x)) * 0.5f;
         y[2] = (bf16_lo(a.y) + bf16_lo(b.y)) * 0.5f;
