@@ -145,3 +145,49 @@ def test_graph_replay_matches_eager():
     # selection output order is deterministic, so replay reproduces the eager step exactly
     assert torch.equal(step.topk[0], ref_topk[0])
     assert torch.equal(step.out, ref_out)
+
+
+def test_hier1m_step_graph_sampled(orc):
+    """The hier1m step at full size (4 x 2^20 entries, 20 layers) in the launch configuration
+    the benchmark times (captured CUDA graph, replayed), checked on sequence 2 against the
+    oracle: its packed pool, the layer-0 block set, every layer's Top-512 and every layer's
+    attention output (the oracle attending with the GPU's list)."""
+    wl = synth.workload("hier1m")
+    sched = synth.layer_schedule(wl)
+    qd = synth.step_queries(wl)
+    x = build_state(wl, lambda b: synth.seq_tokens(wl, b, device="cuda"), qd)
+    step = DecodeStep(B=wl.B, Q=wl.Q, H=wl.H, HI=wl.HI, K=wl.K, window=wl.window, ratio=wl.ratio,
+                      schedule=sched, hier=True, max_n_vis=max(wl.lengths), n_blocks=2048, block=wl.block)
+    step.capture(x)
+    step.replay()
+    torch.cuda.synchronize()
+    step.check_status()
+    b = 2
+    N = int(wl.lengths[b])
+    base = int(x.seq_base[b])
+    kv, ik = synth.seq_tokens(wl, b, device="cuda")
+    o_kv, o_ik = orc.pack_kv(bf16_bits(kv), bf16_bits(ik), wl.ratio)
+    del kv, ik
+    assert np.array_equal(np_u8(x.kv_pool[base:base + N]), o_kv)
+    assert np.array_equal(np_u8(x.ik_pool[base:base + N]), o_ik)
+    one = lambda t: t[b:b + 1].numpy()
+    n_vis = int(qd["n_vis"][b, 0])
+    g_blocks = step.blocks.cpu().numpy()[b, 0]
+    cand = np.sort((g_blocks[:, None] * wl.block + np.arange(wl.block)[None, :]).reshape(-1))
+    cand = cand[cand < n_vis]
+    for l, mode in enumerate(sched):
+        if mode == "full":
+            s = orc.index_scores(qd["qi"][l][b, 0].numpy(), qd["w"][l][b, 0].numpy(), o_ik[:n_vis])
+            bs = s.reshape(-1, wl.block).max(axis=1)
+            o_blocks, _ = orc.topk(bs, 2048)
+            assert_topk_set(g_blocks, o_blocks, bs, 2048, what="blocks")
+        if mode in ("full", "reindex"):
+            sl = orc.index_scores(qd["qi"][l][b, 0].numpy(), qd["w"][l][b, 0].numpy(), o_ik[cand])
+            o_sel, _ = orc.topk(sl, wl.K)
+            assert_topk_set(step.topk[l].cpu().numpy()[b, 0], cand[o_sel], sl, wl.K, labels=cand,
+                            what=f"layer {l}")
+        g_topk = step.layer_topk(l).cpu().numpy()[b:b + 1]
+        o_out, o_lse = orc.sparse_attn(one(qd["q"][l]), o_kv, np.zeros(1, np.int64), g_topk, one(qd["swa"][l]),
+                                       one(qd["swa_start"]), one(qd["q_pos"]), SM, window=wl.window)
+        assert_attn_close(step.out[l].cpu().numpy()[b:b + 1], o_out, what=f"layer {l} ({mode})")
+        assert np.abs(step.lse[l].cpu().numpy()[b:b + 1] - o_lse).max() < 1e-2
