@@ -142,11 +142,17 @@ struct SlotRaw {
   int kind;  // 0 empty, 1 cached entry, 2 window token
 };
 
-__device__ __forceinline__ void gather_slot(const AttnArgs& a, int bq, int b, int64_t base, int64_t t, int slot,
-                                            int hf, SlotRaw& s) {
+// Entry index of Top-K slot `slot` (-1 for an empty slot or a window slot).
+__device__ __forceinline__ int32_t slot_entry(const AttnArgs& a, int bq, int slot) {
+  return slot < a.K ? a.topk[(int64_t)bq * a.K + slot] : -1;
+}
+
+// Issue the loads of this thread's half of key slot `slot`: j = slot_entry(...) and
+// sws = swa_start[b] are passed in, so a caller can load them early.
+__device__ __forceinline__ void gather_slot(const AttnArgs& a, int b, int64_t base, int64_t t, int slot, int hf,
+                                            int32_t j, int64_t sws, SlotRaw& s) {
   s.kind = 0;
   if (slot < a.K) {
-    const int32_t j = a.topk[(int64_t)bq * a.K + slot];
     if (j >= 0) {
       if (base >= 0 && base + j < a.pool_entries) {
         const uint4* e = reinterpret_cast<const uint4*>(a.kv_pool + (base + j) * kKvBytes);
@@ -160,7 +166,7 @@ __device__ __forceinline__ void gather_slot(const AttnArgs& a, int bq, int b, in
     }
   } else if (slot < a.K + a.window && a.S_w > 0) {
     const int64_t u = t - a.window + 1 + (slot - a.K);
-    const int64_t row = u - a.swa_start[b];
+    const int64_t row = u - sws;
     if (u >= 0 && row >= 0 && row < a.S_w) {
       const uint4* src = reinterpret_cast<const uint4*>(a.swa + ((int64_t)b * a.S_w + row) * kD + hf * 256);
 #pragma unroll
@@ -232,8 +238,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
   const int H = a.H;                                 // heads of the query (output layout)
   const int h_base = (blockIdx.y % a.hgroups) * a.hg_size;
   const int NH = min(a.hg_size, H - h_base);         // heads of this cluster, rows 0..NH-1
+  const int r = tid >> 1, hf = tid & 1;
+  const int my_tiles = rank < a.n_tiles ? (a.n_tiles - 1 - rank) / C + 1 : 0;
+  // every load the first gather depends on, issued together
   const int64_t base = a.seq_base[b];
   const int64_t t = a.q_pos[bq];
+  const int32_t j0 = my_tiles > 0 ? slot_entry(a, bq, rank * kTile + r) : -1;
+  const int64_t sws = a.S_w > 0 ? a.swa_start[b] : 0;
   const uint32_t mbar_mma = tc::smem_u32(&mbar[0]), mbar_q = tc::smem_u32(&mbar[1]);
 
   // Start every global read before any set-up barrier: thread 0 initialises the query
@@ -248,11 +259,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
     for (uint32_t off = 0; off < bytes; off += 32768)
       tc::bulk_g2s(tc::smem_u32(Ks) + off, src + off, bytes - off < 32768 ? bytes - off : 32768, mbar_q);
   }
-  const int r = tid >> 1, hf = tid & 1;
-  const int my_tiles = rank < a.n_tiles ? (a.n_tiles - 1 - rank) / C + 1 : 0;
   SlotRaw sr;
   sr.kind = 0;
-  if (my_tiles > 0) gather_slot(a, bq, b, base, t, rank * kTile + r, hf, sr);
+  if (my_tiles > 0) gather_slot(a, b, base, t, rank * kTile + r, hf, j0, sws, sr);
   // phase: gather issued
   if (warp == 0) tc::tmem_alloc(tc::smem_u32(tmem_slot), kTmemCols);
   if (tid < kHeadsPad) {
@@ -292,7 +301,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
   uint32_t commits = 0;
   int processed = 0;
   for (int it = 0; it < my_tiles && !timed_out; ++it) {
-    if (it > 0) gather_slot(a, bq, b, base, t, (rank + it * C) * kTile + r, hf, sr);
+    if (it > 0) {
+      const int slot = (rank + it * C) * kTile + r;
+      gather_slot(a, b, base, t, slot, hf, slot_entry(a, bq, slot), sws, sr);
+    }
     store_slot(Ks, r, hf, sr);
     if (hf == 0) valid_s[r] = sr.kind != 0;
     tc::fence_async_smem();

@@ -176,22 +176,35 @@ __global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
     tc::cp_async_commit();
   };
 
+  // The B operand's query rows and weights are loaded first, so their latency overlaps the
+  // block-id loads the first tile's gather waits for.  Reindex runs one query per CTA
+  // (G = 1), so a warp takes at most 16 / 4 = 4 (query, head) rows.
+  constexpr int kGhPerWarp = 4;
+  float4 qpre[kGhPerWarp];
+  float wpre[kGhPerWarp];
+#pragma unroll
+  for (int k = 0; k < kGhPerWarp; ++k) {
+    const int gh = warp + k * (kScanThreads / 32);
+    const int g = gh / HIPAD, h = gh % HIPAD;
+    qpre[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    wpre[k] = 0.f;
+    if (gh < a.G * HIPAD && g < G && h < a.HI) {
+      const int64_t bq = (int64_t)b * a.Q + q0 + g;
+      qpre[k] = reinterpret_cast<const float4*>(a.q + (bq * a.HI + h) * kDI)[lane];
+      wpre[k] = a.w[bq * a.HI + h];
+    }
+  }
   load_tile(0);  // the first tile's copies overlap the set-up below
   if (warp == 0) tc::tmem_alloc(tc::smem_u32(tmem_slot), a.tmem_cols);
   if (tid == 32) tc::mbar_init(tc::smem_u32(mbar), 1);
 
   // ---- B operand: four int8 limbs of every (query, head), plus epilogue constants ---------
-  for (int gh = warp; gh < a.G * HIPAD; gh += kScanThreads / 32) {
-    const int g = gh / HIPAD, h = gh % HIPAD;
-    const bool live = g < G && h < a.HI;
-    float x[4] = {0.f, 0.f, 0.f, 0.f};
-    float wv = 0.f;
-    if (live) {
-      const int64_t bq = (int64_t)b * a.Q + q0 + g;
-      const float4 v = reinterpret_cast<const float4*>(a.q + (bq * a.HI + h) * kDI)[lane];
-      x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-      wv = a.w[bq * a.HI + h];
-    }
+#pragma unroll
+  for (int k = 0; k < kGhPerWarp; ++k) {
+    const int gh = warp + k * (kScanThreads / 32);
+    if (gh >= a.G * HIPAD) break;
+    float x[4] = {qpre[k].x, qpre[k].y, qpre[k].z, qpre[k].w};
+    const float wv = wpre[k];
     float m = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
