@@ -12,24 +12,23 @@
 // Score of entry j for one query:  score_j = s_j * sum_h w_h * max(0, q_h . c_j)
 // (c_j the key's E2M1 values, s_j >= 0 its fp32 scale, so the ReLU commutes with s_j).
 //
-// scan_tc_kernel computes the dot products exactly on the tensor cores (tcgen05.mma
-// kind::i8, int32 accumulation):
+// Both scan kernels (stream_scan_kernel for the flat and hierarchical scans,
+// reindex_scan_kernel for Reindex) compute the dot products exactly on the tensor cores
+// (tcgen05.mma kind::i8, int32 accumulation):
 //   * A (128 entries x 128 dims, u8): u = 2c + 12 in [0, 24] — the E2M1 value doubled and
 //     offset to be non-negative; two byte-permutes per 4 codes build it (sign-replicate
 //     selects the positive or negative table).
-//   * B (N rows x 128 dims, s8): each query head h is scaled by S_h = 127 / max|q_h| and
-//     split into four int8 limbs, x = q*S_h = L0 + L1/128 + L2/128^2 + L3/128^3 with an
-//     error below 0.5/128^3 (about 2e-9 of max|q_h|).
+//   * B (N rows x 128 dims, s8): each query head h is scaled by the power of two
+//     S_h = 2^(5 - exponent(max|q_h|)), so x = q*S_h is exact with |x| < 64, and split into
+//     four int8 limbs x = L0 + L1/128 + L2/128^2 + L3/128^3 (error below 2^-22).
 //   * D (128 x N, s32): acc_p = sum_d u_d L_p,d, so sum_d c_d L_p,d = (acc_p - 12 T_p)/2
-//     with T_p = sum_d L_p,d; the epilogue combines the limbs in fp32:
-//     q_h . c_j = (sum_p 128^-p (acc_p - 12 T_p)) / (2 S_h).
-// The raw 68 B keys reach shared memory through cp.async (16 B copies, ragged ends with
-// 4 B copies, one tile ahead); Reindex tiles are 16 gathered blocks of 8 entries.  Each
-// of the 128 threads owns one tile row (entry) end to end: it builds the row's A operand,
-// and after the MMA reads the same TMEM lane and writes the entry's order-preserving
-// uint32 key (hierarchical mode: the max over `block` neighbouring lanes).  A CTA takes
-// a group of up to G queries of one sequence (multi-query verify), so the A operand is
-// built once for the group.
+//     with T_p = sum_d L_p,d; the epilogue removes the offset exactly in integers and
+//     combines the limbs in fp32: q_h . c_j = (sum_p 128^-p (acc_p - 12 T_p)) / (2 S_h).
+// One thread owns one tile row (entry) end to end: it builds the row's A operand, and
+// after the MMA reads the same TMEM lane and writes the entry's order-preserving uint32
+// key (hierarchical mode: the max over `block` neighbouring lanes).  The streaming scan
+// takes a group of up to 8 queries of one sequence per CTA (multi-query verify), so the A
+// operand is built once for the group.
 #include <algorithm>
 #include <cooperative_groups.h>
 
@@ -102,8 +101,11 @@ __device__ __forceinline__ uint2 codes_to_u8(uint32_t w) {
   return make_uint2(p0 | n0, p1 | n1);
 }
 
-template <int MODE, int HIPAD>
-__global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
+// Reindex scan: one CTA row per (sequence, query), each CTA scoring kRows-candidate tiles
+// gathered from the query's block list (128 / block blocks of `block` consecutive keys per
+// tile, staged by cp.async one tile ahead).
+template <int HIPAD>
+__global__ void __launch_bounds__(kScanThreads) reindex_scan_kernel(ScanArgs a) {
   chain_enter();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = tc::align_smem_1024(smem_raw);
@@ -111,100 +113,76 @@ __global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
   uint8_t* Bs = As + kRows * 128;                     // [N rows x 128 B]
   uint8_t* raw = Bs + a.N * 128;                      // 2 x kRawBytes
   int32_t* corr = reinterpret_cast<int32_t*>(raw + 2 * kRawBytes);  // [N]
-  float* wq = reinterpret_cast<float*>(corr + a.N);                 // [G * HIPAD]
-  int64_t* nq = reinterpret_cast<int64_t*>(wq + a.G * HIPAD);       // [G] visible count per query
-  int32_t* segc = reinterpret_cast<int32_t*>(nq + a.G);             // [2][128] gathered block ids
+  float* wq = reinterpret_cast<float*>(corr + a.N);                 // [HIPAD]
+  int32_t* segc = reinterpret_cast<int32_t*>(wq + HIPAD);           // [2][128] gathered block ids
   uint64_t* mbar = reinterpret_cast<uint64_t*>(segc + 256);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mbar + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int b = blockIdx.y / a.n_groups;
-  const int gidx = blockIdx.y % a.n_groups;
-  const int q0 = gidx * a.G;
-  const int G = min(a.G, a.Q - q0);
-  const int64_t base = a.seq_base[b];
-
-  // items of this CTA's query group: entries (flat/hier) or candidate slots (reindex)
-  int64_t limit = 0;
-  for (int g = 0; g < G; ++g) {
-    const int64_t n = valid_count(a, b, b * a.Q + q0 + g, false);
-    limit = n > limit ? n : limit;
-  }
-  if (MODE == kReindex) limit = (int64_t)a.n_blocks * a.block;
+  const int bq = blockIdx.y;  // (sequence, query) of this CTA row
+  const int b = bq / a.Q;
+  const int64_t limit = (int64_t)a.n_blocks * a.block;  // candidate slots
   const int64_t item0 = (int64_t)blockIdx.x * a.tiles_per_cta * kRows;
   if (item0 >= limit) return;
   const int64_t left_tiles = (limit - item0 + kRows - 1) / kRows;
   const int ntiles = (int)(left_tiles < a.tiles_per_cta ? left_tiles : a.tiles_per_cta);
+  const int64_t nvis = valid_count(a, b, bq, blockIdx.x == 0);  // 0 if the count is bad
 
-  if (tid < G) nq[tid] = valid_count(a, b, b * a.Q + q0 + tid, blockIdx.x == 0);
-  const int64_t nq0 = valid_count(a, b, b * a.Q + q0, false);  // reindex: the single query's count
-
-  const uint8_t* seq = a.ik_pool + base * kIkBytes;
-  const int mis = (int)((reinterpret_cast<uintptr_t>(seq)) & 15u);  // same for every tile
+  const uint8_t* seq = a.ik_pool + a.seq_base[b] * kIkBytes;
   const uint32_t raw_a = tc::smem_u32(raw);
-  // reindex tiles: 128 / block gathered blocks, each staged at seg_stride (16 B multiple)
+  // a tile's 128 / block gathered blocks, each staged at seg_stride (a 16 B multiple)
   const int seg_stride = ((a.block * kIkBytes + 16) + 15) & ~15;
 
-  // raw tile loader: tile index ti into buffer ti & 1
+  // gathered tile loader: tile ti into buffer ti & 1; `block` threads copy each block
   auto load_tile = [&](int ti) {
     const int64_t i0 = item0 + (int64_t)ti * kRows;
     const uint32_t dst = raw_a + (ti & 1) * kRawBytes;
-    if (MODE != kReindex) {
-      const int cnt = (int)(limit - i0 < kRows ? limit - i0 : kRows);
-      stage_async(dst + mis, seq + i0 * kIkBytes, cnt * kIkBytes, tid, kScanThreads);
-    } else {
-      const int s = tid >> a.block_shift, sub = tid & (a.block - 1);  // 128/block blocks, `block` threads each
-      const int64_t slot_blk = (i0 >> a.block_shift) + s;
-      int32_t c = -1;
-      if (slot_blk < a.n_blocks) c = a.blocks[(int64_t)(b * a.Q + q0) * a.n_blocks + slot_blk];
-      if (sub == 0) {
-        segc[(ti & 1) * 128 + s] = c;
-        if (c < -1) flag(a.status, CSA2_DEV_BAD_INDEX);
-      }
-      int cnt = 0;
-      if (c >= 0) {
-        const int64_t rem = nq0 - (int64_t)c * a.block;
-        cnt = rem <= 0 ? 0 : (int)(rem < a.block ? rem : a.block);
-      }
-      if (cnt > 0) {
-        // a block starts at its own address residue mod 16 unless block*68 is a 16 B multiple
-        const uint8_t* src = seq + (int64_t)c * a.block * kIkBytes;
-        const int smis = (int)(reinterpret_cast<uintptr_t>(src) & 15u);
-        stage_async(dst + s * seg_stride + smis, src, cnt * kIkBytes, sub, a.block);
-      }
+    const int s = tid >> a.block_shift, sub = tid & (a.block - 1);
+    const int64_t slot_blk = (i0 >> a.block_shift) + s;
+    int32_t c = -1;
+    if (slot_blk < a.n_blocks) c = a.blocks[(int64_t)bq * a.n_blocks + slot_blk];
+    if (sub == 0) {
+      segc[(ti & 1) * 128 + s] = c;
+      if (c < -1) flag(a.status, CSA2_DEV_BAD_INDEX);
+    }
+    int cnt = 0;
+    if (c >= 0) {
+      const int64_t rem = nvis - (int64_t)c * a.block;
+      cnt = rem <= 0 ? 0 : (int)(rem < a.block ? rem : a.block);
+    }
+    if (cnt > 0) {
+      // a block starts at its own address residue mod 16 unless block*68 is a 16 B multiple
+      const uint8_t* src = seq + (int64_t)c * a.block * kIkBytes;
+      const int smis = (int)(reinterpret_cast<uintptr_t>(src) & 15u);
+      stage_async(dst + s * seg_stride + smis, src, cnt * kIkBytes, sub, a.block);
     }
     tc::cp_async_commit();
   };
 
   // The B operand's query rows and weights are loaded first, so their latency overlaps the
-  // block-id loads the first tile's gather waits for.  Reindex runs one query per CTA
-  // (G = 1), so a warp takes at most 16 / 4 = 4 (query, head) rows.
-  constexpr int kGhPerWarp = 4;
-  float4 qpre[kGhPerWarp];
-  float wpre[kGhPerWarp];
+  // block-id loads the first tile's gather waits for; a warp takes HIPAD / 4 heads.
+  constexpr int kHeadsPerWarp = HIPAD / (kScanThreads / 32);
+  float4 qpre[kHeadsPerWarp];
+  float wpre[kHeadsPerWarp];
 #pragma unroll
-  for (int k = 0; k < kGhPerWarp; ++k) {
-    const int gh = warp + k * (kScanThreads / 32);
-    const int g = gh / HIPAD, h = gh % HIPAD;
+  for (int k = 0; k < kHeadsPerWarp; ++k) {
+    const int h = warp + k * (kScanThreads / 32);
     qpre[k] = make_float4(0.f, 0.f, 0.f, 0.f);
     wpre[k] = 0.f;
-    if (gh < a.G * HIPAD && g < G && h < a.HI) {
-      const int64_t bq = (int64_t)b * a.Q + q0 + g;
-      qpre[k] = reinterpret_cast<const float4*>(a.q + (bq * a.HI + h) * kDI)[lane];
-      wpre[k] = a.w[bq * a.HI + h];
+    if (h < a.HI) {
+      qpre[k] = reinterpret_cast<const float4*>(a.q + ((int64_t)bq * a.HI + h) * kDI)[lane];
+      wpre[k] = a.w[(int64_t)bq * a.HI + h];
     }
   }
   load_tile(0);  // the first tile's copies overlap the set-up below
   if (warp == 0) tc::tmem_alloc(tc::smem_u32(tmem_slot), a.tmem_cols);
   if (tid == 32) tc::mbar_init(tc::smem_u32(mbar), 1);
 
-  // ---- B operand: four int8 limbs of every (query, head), plus epilogue constants ---------
+  // ---- B operand: four int8 limbs of every head, plus epilogue constants ----------------
 #pragma unroll
-  for (int k = 0; k < kGhPerWarp; ++k) {
-    const int gh = warp + k * (kScanThreads / 32);
-    if (gh >= a.G * HIPAD) break;
-    float x[4] = {qpre[k].x, qpre[k].y, qpre[k].z, qpre[k].w};
-    const float wv = wpre[k];
+  for (int k = 0; k < kHeadsPerWarp; ++k) {
+    const int h = warp + k * (kScanThreads / 32);
+    const float x[4] = {qpre[k].x, qpre[k].y, qpre[k].z, qpre[k].w};
     float m = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -232,16 +210,15 @@ __global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
     }
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-      const int n = gh * 4 + p;
+      const int n = h * 4 + p;
       *reinterpret_cast<uint32_t*>(Bs + tc::sw128(n, lane * 4)) = limb[p];
       int t = lsum[p];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
       if (lane == 0) corr[n] = 0x4B400000 - 12 * t;
     }
-    if (lane == 0) wq[gh] = S > 0.f ? wv / (2.0f * S) : 0.f;
+    if (lane == 0) wq[h] = S > 0.f ? wpre[k] / (2.0f * S) : 0.f;
   }
-
   tc::fence_async_smem();
   tc::fence_before_sync();
   __syncthreads();
@@ -249,6 +226,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
   const uint32_t tmem = *tmem_slot;
   const uint32_t idesc = tc::idesc_i8(kRows, a.N, false, true);
   const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+  uint32_t* krow = a.keys + (int64_t)bq * a.key_stride;
   bool timed_out = false;
 
   for (int ti = 0; ti < ntiles; ++ti) {
@@ -257,26 +235,16 @@ __global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
     tc::cp_async_wait<1>();
     __syncthreads();
     const int64_t i0 = item0 + (int64_t)ti * kRows;
-    // ---- this thread's row: locate the entry, build the A row --------------------------
-    const uint8_t* rbuf = raw + (ti & 1) * kRawBytes;
-    const uint8_t* ent;
-    bool valid;
-    int64_t j;  // entry index within the sequence
-    if (MODE != kReindex) {
-      j = i0 + tid;
-      valid = j < limit;
-      ent = rbuf + mis + tid * kIkBytes;
-    } else {
-      const int s = tid >> a.block_shift, r = tid & (a.block - 1);
-      const int32_t c = segc[(ti & 1) * 128 + s];
-      j = (int64_t)c * a.block + r;
-      valid = c >= 0 && j < nq0;
-      const int smis = c >= 0 ? (int)(reinterpret_cast<uintptr_t>(seq + (int64_t)c * a.block * kIkBytes) & 15u) : 0;
-      ent = rbuf + s * seg_stride + smis + r * kIkBytes;
-    }
+    // ---- this thread's row: locate the candidate, build the A row ------------------------
+    const int s = tid >> a.block_shift, r = tid & (a.block - 1);
+    const int32_t c = segc[(ti & 1) * 128 + s];
+    const int64_t j = (int64_t)c * a.block + r;  // entry index within the sequence
+    const bool valid = c >= 0 && j < nvis;
     float sj = 0.f;
     if (valid) {
-      const uint32_t* ew = reinterpret_cast<const uint32_t*>(ent);
+      const int smis = (int)(reinterpret_cast<uintptr_t>(seq + (int64_t)c * a.block * kIkBytes) & 15u);
+      const uint32_t* ew =
+          reinterpret_cast<const uint32_t*>(raw + (ti & 1) * kRawBytes + s * seg_stride + smis + r * kIkBytes);
       uint32_t cw[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) cw[i] = ew[i];
@@ -305,35 +273,24 @@ __global__ void __launch_bounds__(kScanThreads) scan_tc_kernel(ScanArgs a) {
     tc::fence_after_sync();
     if (timed_out) break;
     // ---- epilogue: limbs -> fp32 dot products -> ReLU-weighted score -> key --------------
-    for (int g = 0; g < G; ++g) {
-      uint32_t r[HIPAD * 4];
-      if (HIPAD == 4) {
-        tc::tmem_ld16(lane_addr + g * 16, r);
-      } else {
+    uint32_t acc[HIPAD * 4];
+    if (HIPAD == 4) {
+      tc::tmem_ld16(lane_addr, acc);
+    } else {
 #pragma unroll
-        for (int c = 0; c < HIPAD / 8; ++c) tc::tmem_ld32(lane_addr + g * HIPAD * 4 + c * 32,
-                                                         *reinterpret_cast<uint32_t(*)[32]>(r + 32 * c));
-      }
-      float tot = 0.f;
-#pragma unroll
-      for (int h = 0; h < HIPAD; ++h) {
-        const int nb = (g * HIPAD + h) * 4;
-        float f[4];
-#pragma unroll
-        for (int p = 0; p < 4; ++p) f[p] = __int_as_float((int)r[h * 4 + p] + corr[nb + p]) - 12582912.0f;
-        const float z = fmaf(fmaf(fmaf(f[3], 0.0078125f, f[2]), 0.0078125f, f[1]), 0.0078125f, f[0]);
-        tot = fmaf(wq[g * HIPAD + h], fmaxf(z, 0.f), tot);
-      }
-      const bool vis = valid && j < nq[g];
-      uint32_t key = vis ? score_key(sj * tot) : 0u;
-      uint32_t* krow = a.keys + ((int64_t)b * a.Q + q0 + g) * a.key_stride;
-      if (MODE == kHier) {
-        for (int o = 1; o < a.block; o <<= 1) key = max(key, __shfl_xor_sync(0xffffffffu, key, o));
-        if ((tid & (a.block - 1)) == 0 && i0 + tid < nq[g]) krow[(i0 + tid) >> a.block_shift] = key;
-      } else if (i0 + tid < limit) {
-        krow[i0 + tid] = key;
-      }
+      for (int c32 = 0; c32 < HIPAD / 8; ++c32)
+        tc::tmem_ld32(lane_addr + c32 * 32, *reinterpret_cast<uint32_t(*)[32]>(acc + 32 * c32));
     }
+    float tot = 0.f;
+#pragma unroll
+    for (int h = 0; h < HIPAD; ++h) {
+      float f[4];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) f[p] = __int_as_float((int)acc[h * 4 + p] + corr[h * 4 + p]) - 12582912.0f;
+      const float z = fmaf(fmaf(fmaf(f[3], 0.0078125f, f[2]), 0.0078125f, f[1]), 0.0078125f, f[0]);
+      tot = fmaf(wq[h], fmaxf(z, 0.f), tot);
+    }
+    if (i0 + tid < limit) krow[i0 + tid] = valid ? score_key(sj * tot) : 0u;
     tc::fence_before_sync();
   }
   if (timed_out && tid == 0) flag(a.status, CSA2_DEV_TIMEOUT);
@@ -1091,34 +1048,34 @@ static int pow2_at_least(int x) {
   return p;
 }
 
-template <int MODE>
-static cudaError_t launch_scan(ScanArgs a, int64_t items, int B, cudaStream_t st) {
+// Reindex scan: one CTA row per (sequence, query), two 128-candidate tiles per CTA.
+static cudaError_t launch_reindex_scan(ScanArgs a, int64_t items, int BQ, cudaStream_t st) {
   a.hipad = a.HI <= 4 ? 4 : (a.HI <= 8 ? 8 : 16);
-  a.G = MODE == kReindex ? 1 : max(1, min(a.Q, 256 / (a.hipad * 4)));
-  a.n_groups = (a.Q + a.G - 1) / a.G;
-  a.N = a.G * a.hipad * 4;
+  a.G = 1;
+  a.n_groups = a.Q;
+  a.N = a.hipad * 4;
   a.tmem_cols = pow2_at_least(a.N);
-  a.tiles_per_cta = MODE == kReindex ? 2 : 8;
+  a.tiles_per_cta = 2;
   const int64_t per_cta = (int64_t)a.tiles_per_cta * kRows;
-  const dim3 grid((unsigned)((items + per_cta - 1) / per_cta), (unsigned)(B * a.n_groups));
+  const dim3 grid((unsigned)((items + per_cta - 1) / per_cta), (unsigned)BQ);
   if (grid.x == 0 || grid.y == 0) return cudaSuccess;
-  const size_t smem = 1024 + (size_t)kRows * 128 + (size_t)a.N * 128 + 2 * kRawBytes + (size_t)a.N * 4 +
-                      (size_t)a.G * a.hipad * 4 + (size_t)a.G * 8 + 256 * 4 + 16;
+  const size_t smem = 1024 + (size_t)kRows * 128 + (size_t)a.N * 128 + 2 * (size_t)kRawBytes + (size_t)a.N * 4 +
+                      (size_t)a.hipad * 4 + 256 * 4 + 16;
   cudaError_t e;
-#define CSA2_SCAN_LAUNCH(HP)                                                                        \
-  e = cudaFuncSetAttribute(scan_tc_kernel<MODE, HP>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+#define CSA2_REINDEX_LAUNCH(HP)                                                                     \
+  e = cudaFuncSetAttribute(reindex_scan_kernel<HP>, cudaFuncAttributeMaxDynamicSharedMemorySize,    \
                            (int)smem);                                                              \
   if (e != cudaSuccess) return e;                                                                   \
-  e = launch_chained(scan_tc_kernel<MODE, HP>, grid, dim3(kScanThreads), smem, st, 0, a);             \
+  e = launch_chained(reindex_scan_kernel<HP>, grid, dim3(kScanThreads), smem, st, 0, a);            \
   if (e != cudaSuccess) return e;
   if (a.hipad == 4) {
-    CSA2_SCAN_LAUNCH(4)
+    CSA2_REINDEX_LAUNCH(4)
   } else if (a.hipad == 8) {
-    CSA2_SCAN_LAUNCH(8)
+    CSA2_REINDEX_LAUNCH(8)
   } else {
-    CSA2_SCAN_LAUNCH(16)
+    CSA2_REINDEX_LAUNCH(16)
   }
-#undef CSA2_SCAN_LAUNCH
+#undef CSA2_REINDEX_LAUNCH
   return cudaGetLastError();
 }
 
@@ -1226,7 +1183,7 @@ cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t
   else if (mode == kHier)
     e = launch_stream<kHier>(a, max_n_vis, B, stream);
   else
-    e = launch_scan<kReindex>(a, (int64_t)n_blocks * block, B, stream);  // one CTA row per (b, query)
+    e = launch_reindex_scan(a, (int64_t)n_blocks * block, BQ, stream);
   if (e != cudaSuccess) return e;
 
   SelectArgs s;
