@@ -532,16 +532,33 @@ cudaError_t launch_sparse_attn(const float* q, const uint8_t* kv_pool, int64_t p
   a.H = H;
   a.sm_scale = sm_scale;
   a.n_tiles = (K + a.window + kTile - 1) / kTile;
-  a.csize = a.n_tiles < 1 ? 1 : (a.n_tiles > kMaxCluster ? kMaxCluster : a.n_tiles);
   a.out = out;
   a.lse = lse;
   a.status = status;
   const int64_t BQ = (int64_t)B * Q;
   if (BQ == 0) return cudaSuccess;
-  // When the clusters do not fill the GPU, split each query's heads into groups of 16 or 32,
-  // one cluster per group: a CTA then converts, exports and merges only its group's heads.
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // Key split: the C CTAs of a query's cluster take its tiles round-robin.  Few queries want
+  // a wide split (more SMs at work), many queries want none (no merge, fewer waves).  C
+  // minimises waves x (set-up + tiles per CTA x per-tile time + merge when split), with one
+  // CTA per SM and costs in microseconds measured on the kernel's phases.
+  {
+    constexpr double kSetup = 5.0, kPerTile = 7.0, kMerge = 5.0;
+    const int cmax = a.n_tiles < 1 ? 1 : (a.n_tiles > kMaxCluster ? kMaxCluster : a.n_tiles);
+    double best = 0.0;
+    a.csize = 1;
+    for (int c = 1; c <= cmax; ++c) {
+      const double waves = (double)((BQ * c + sms - 1) / sms);
+      const double per_cta = kSetup + (double)((a.n_tiles + c - 1) / c) * kPerTile + (c > 1 ? kMerge : 0.0);
+      if (c == 1 || waves * per_cta < best) {
+        best = waves * per_cta;
+        a.csize = c;
+      }
+    }
+  }
+  // When the clusters do not fill the GPU, split each query's heads into groups of 16 or 32,
+  // one cluster per group: a CTA then converts, exports and merges only its group's heads.
   a.hgroups = 1;
   for (int g = 4; g >= 2; g >>= 1)
     if (H % (16 * g) == 0 && BQ * a.csize * g <= sms) {
