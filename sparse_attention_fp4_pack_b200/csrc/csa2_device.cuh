@@ -91,14 +91,6 @@ __device__ __forceinline__ float e4m3_value(uint32_t s) {
   return __uint_as_float(((e + 120u) << 23) | (m << 20));
 }
 
-// E2M1 magnitude code (0..7) -> fp32.
-__device__ __forceinline__ float e2m1_mag(uint32_t m) {
-  // 0, 0.5, 1, 1.5, 2, 3, 4, 6 : for m >= 2 the fp32 exponent is 126 + (m >> 1) and the
-  // top mantissa bit is m & 1; m = 1 is the subnormal 0.5.
-  float v = __uint_as_float(((126u + (m >> 1)) << 23) | ((m & 1u) << 22));
-  return m >= 2 ? v : (m == 1 ? 0.5f : 0.0f);
-}
-
 // Order-preserving map of an fp32 score onto uint32 (larger score -> larger key).
 // Key 0 is reserved for "no candidate" (it is the image of a negative NaN only).
 __device__ __forceinline__ uint32_t score_key(float s) {

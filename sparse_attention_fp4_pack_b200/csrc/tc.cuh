@@ -1,6 +1,7 @@
-// sm_100a tensor-core primitives used by libcsa2: shared-memory matrix descriptors,
-// tcgen05.mma instruction descriptors, TMEM allocation and loads, tcgen05.commit to an
-// mbarrier, and bounded mbarrier waits.
+// sm_100a primitives used by libcsa2: shared-memory matrix descriptors, tcgen05.mma
+// instruction descriptors, TMEM allocation, loads and stores, tcgen05.commit to an
+// mbarrier, bounded mbarrier waits, cp.async and bulk copies, explicit shared-memory and
+// cluster shared-memory accesses, and a reducing named barrier.
 //
 // Descriptor layouts (Blackwell UMMA):
 //   shared-memory descriptor (64 bit): start address >> 4 in bits [0,14), leading byte
@@ -48,19 +49,6 @@ __device__ __forceinline__ uint64_t ld_shared_u64(uint32_t saddr) {
   uint64_t v;
   asm volatile("ld.shared.u64 %0, [%1];" : "=l"(v) : "r"(saddr) : "memory");
   return v;
-}
-__device__ __forceinline__ float ld_shared_f32(uint32_t saddr) {
-  float v;
-  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(saddr) : "memory");
-  return v;
-}
-__device__ __forceinline__ uint16_t ld_shared_u16(uint32_t saddr) {
-  uint16_t v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(saddr) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_shared_u16(uint32_t saddr, uint16_t v) {
-  asm volatile("st.shared.u16 [%0], %1;" ::"r"(saddr), "h"(v) : "memory");
 }
 __device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
@@ -188,16 +176,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
       : "memory");
 }
 
-// 8 consecutive 32-bit columns (32x32b shape, x8), load and wait in one statement.
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-      : "r"(taddr)
-      : "memory");
-}
-
 // Asynchronous global -> shared copies (cp.async), 16 B (L2 only) and 4 B.
 __device__ __forceinline__ void cp_async16(uint32_t dst_saddr, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_saddr), "l"(src) : "memory");
@@ -251,22 +229,6 @@ __device__ __forceinline__ bool named_sync_or(int id, int nthreads, bool pred) {
   return r != 0;
 }
 
-// Bulk copy from this CTA's shared memory into shared memory of a CTA of the cluster
-// (dst and mbar are shared::cluster addresses from mapa); the bytes count toward the
-// destination mbarrier's transaction count.  Addresses and size are 16-byte multiples.
-__device__ __forceinline__ void bulk_s2cluster(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t mbar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-      "r"(src), "r"(bytes), "r"(mbar)
-      : "memory");
-}
-// Bulk-copy completion groups of this thread: commit, then wait until every committed
-// copy has finished reading its source.
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read_all() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-
 // Shared-memory address of the same variable in CTA `rank` of this cluster.
 __device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
   uint32_t r;
@@ -285,14 +247,6 @@ __device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t caddr) {
                : "r"(caddr)
                : "memory");
   return v;
-}
-
-// Asynchronous 4-byte store into (possibly another CTA's) shared memory; its bytes count
-// toward the transaction count of the mbarrier at rmbar in the same CTA as the target.
-__device__ __forceinline__ void st_async_b32(uint32_t raddr, uint32_t v, uint32_t rmbar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(raddr), "r"(v),
-               "r"(rmbar)
-               : "memory");
 }
 
 // Arrive on the mbarrier and add `bytes` to the transaction count it waits for.
