@@ -98,6 +98,7 @@ class DecodeStep:
         self.lse = torch.empty(L, B, Q, H, dtype=torch.float32, device=device)
         self.status = csa2.status_word(device)
         self.graph = None
+        self.graph_io = None
         self.timer: Optional[CallTimer] = None
 
     def launches_per_step(self) -> int:
@@ -119,7 +120,9 @@ class DecodeStep:
         if self.timer is not None:
             self.timer.end()
 
-    def run(self, x: StepInputs):
+    def run(self, x: StepInputs, before_layer=None, after_layer=None):
+        """Enqueue the step on the current stream; before_layer(l) / after_layer(l), when
+        given, run (on the host, while enqueueing) around layer l's calls."""
         if self.timer is not None:
             self.timer.rewind()
         self._begin("pack")
@@ -128,6 +131,8 @@ class DecodeStep:
         self._end()
         cur = None
         for l, mode in enumerate(self.schedule):
+            if before_layer is not None:
+                before_layer(l)
             if mode == "full":
                 if self.hier:
                     self._begin("index_hier")
@@ -159,6 +164,57 @@ class DecodeStep:
                                   self.out[l], self.lse[l], window=self.window, ws=self.ws,
                                   dev_status=self.status)
             self._end()
+            if after_layer is not None:
+                after_layer(l)
+
+    def run_io(self, x: StepInputs, h_in: dict, h_out: dict, s_in: torch.cuda.Stream,
+               s_out: torch.cuda.Stream):
+        """The step with its per-step inputs copied from pinned host memory and its results
+        read back, overlapped with the work: s_in copies the new tokens, then the layers'
+        queries, indexer queries, weights and windows in layer order, in chunks that double
+        in length (layers 0, 1, 2-3, 4-7, ...); the first layer of a chunk starts once the
+        chunk has landed (later layers keep their launches chained to the previous kernel);
+        s_out copies layer l's output, log-sum-exp and Top-K list to the host as soon as the
+        layer has finished.  The current stream joins both at the end.
+        h_in: pinned tensors named like the StepInputs fields new_kv, new_ik, q, qi, w, swa;
+        h_out: pinned tensors out, lse, topk shaped like this step's buffers."""
+        comp = torch.cuda.current_stream()
+        s_in.wait_stream(comp)
+        s_out.wait_stream(comp)
+        L = len(self.schedule)
+        with torch.cuda.stream(s_in):
+            x.new_kv.copy_(h_in["new_kv"], non_blocking=True)
+            x.new_ik.copy_(h_in["new_ik"], non_blocking=True)
+            new_ready = torch.cuda.Event()
+            new_ready.record(s_in)
+            chunk_ready = {}
+            l0, n = 0, 1
+            while l0 < L:
+                l1 = min(L, l0 + n)
+                for k in ("q", "qi", "w", "swa"):
+                    getattr(x, k)[l0:l1].copy_(h_in[k][l0:l1], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(s_in)
+                chunk_ready[l0] = ev
+                l0, n = l1, (n if l0 == 0 else 2 * n)
+        comp.wait_event(new_ready)
+
+        def before(l):
+            if l in chunk_ready:
+                comp.wait_event(chunk_ready[l])
+
+        def after(l):
+            done = torch.cuda.Event()
+            done.record(comp)
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                h_out["out"][l].copy_(self.out[l], non_blocking=True)
+                h_out["lse"][l].copy_(self.lse[l], non_blocking=True)
+                h_out["topk"][l].copy_(self.topk[l], non_blocking=True)
+
+        self.run(x, before_layer=before, after_layer=after)
+        comp.wait_stream(s_in)
+        comp.wait_stream(s_out)
 
     def layer_topk(self, l: int) -> torch.Tensor:
         """The Top-K list layer l attended with (a Reuse layer's is its source's)."""
@@ -179,8 +235,25 @@ class DecodeStep:
         self.graph = g
         return g
 
+    def capture_io(self, x: StepInputs, h_in: dict, h_out: dict):
+        """Capture run_io in a CUDA graph (host and device buffers must stay in place)."""
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.run_io(x, h_in, h_out, s_in, s_out)  # warm-up outside the graph
+        torch.cuda.current_stream().wait_stream(s)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.run_io(x, h_in, h_out, s_in, s_out)
+        self.graph_io = g
+        return g
+
     def replay(self):
         self.graph.replay()
+
+    def replay_io(self):
+        self.graph_io.replay()
 
     def check_status(self):
         word = int(self.status.item())

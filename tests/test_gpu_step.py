@@ -191,3 +191,33 @@ def test_hier1m_step_graph_sampled(orc):
                                        one(qd["swa_start"]), one(qd["q_pos"]), SM, window=wl.window)
         assert_attn_close(step.out[l].cpu().numpy()[b:b + 1], o_out, what=f"layer {l} ({mode})")
         assert np.abs(step.lse[l].cpu().numpy()[b:b + 1] - o_lse).max() < 1e-2
+
+
+def test_io_step_matches_device_step():
+    """run_io (pinned host inputs in, results out, copies overlapped with the layers) in a
+    captured graph gives exactly the device step's results, on the hierarchical schedule."""
+    wl = synth.DecodeWorkload("hier-io", 13, B=2, Q=1, H=32, HI=8, K=128, window=128, ratio=1,
+                              lengths=[9000, 7001], hier=True, n_layers=5)
+    step, x, qd, toks, sched = _step(wl, n_blocks=64)
+    step.run(x)
+    torch.cuda.synchronize()
+    step.check_status()
+    ref = {"out": step.out.clone(), "lse": step.lse.clone(), "topk": step.topk.clone()}
+    h_in = {k: getattr(x, k).cpu().pin_memory() for k in ("new_kv", "new_ik", "q", "qi", "w", "swa")}
+    h_out = {k: torch.full_like(v, 7, device="cpu").pin_memory() for k, v in ref.items()}
+    for k in ("q", "qi", "w", "swa"):
+        getattr(x, k).zero_()                      # the graph must bring them in itself
+    step.out.zero_()
+    step.capture_io(x, h_in, h_out)
+    for k in ("q", "qi", "w", "swa"):
+        getattr(x, k).zero_()
+    for t in h_out.values():
+        t.fill_(7)
+    step.replay_io()
+    torch.cuda.synchronize()
+    step.check_status()
+    for k in ("out", "lse"):
+        assert torch.equal(h_out[k], ref[k].cpu()), k
+    for l, mode in enumerate(sched):
+        if mode != "reuse":
+            assert torch.equal(h_out["topk"][l], ref["topk"][l].cpu()), f"topk layer {l}"
