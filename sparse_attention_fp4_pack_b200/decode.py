@@ -102,14 +102,15 @@ class DecodeStep:
         self.timer: Optional[CallTimer] = None
 
     def launches_per_step(self) -> int:
-        """Kernel launches one run() issues (pack 1; each index/reindex call 2; each attention 2)."""
+        """Kernel launches one run() issues: the pack 1; each index, hierarchical-index and
+        Reindex call 2 (scan, select); each attention call 1 (its merge runs inside)."""
         n = 1
         for mode in self.schedule:
             if mode == "full":
-                n += 4 if self.hier else 2
+                n += 4 if self.hier else 2   # hierarchical: block select, then the layer's own Reindex
             elif mode == "reindex":
                 n += 2
-            n += 2
+            n += 1
         return n
 
     def _begin(self, name):

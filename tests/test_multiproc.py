@@ -68,3 +68,18 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["unit"] == "µs/token"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_launch_count_matches_the_schedule():
+    """gpu_launches in the bench line comes from launches_per_step: 45 kernels per hier1m
+    step (pack 1, hierarchical scan + select 2, 11 Reindex scans + selects 22, 20
+    attention launches), as the ncu launch list of one step shows."""
+    import synth
+    from sparse_attention_fp4_pack_b200.decode import DecodeStep
+    wl = synth.workload("hier1m")
+    sched = synth.layer_schedule(wl)
+    step = DecodeStep.__new__(DecodeStep)  # the count needs only the schedule
+    step.schedule, step.hier = sched, True
+    assert step.launches_per_step() == 45
+    step.schedule, step.hier = ["full", "reuse"], False
+    assert step.launches_per_step() == 1 + 2 + 1 + 1
