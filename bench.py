@@ -97,18 +97,59 @@ def max_over_ranks(x, world):
 
 
 # ---- clocks during the timed region ---------------------------------------------------------
+# Separate process (no share of this process's interpreter lock): read-only NVML queries of
+# one GPU every 2 ms, one "time,sm_mhz,reasons_bitmask" line each, until terminated.
+_NVML_POLL = """
+import sys, time, pynvml
+pynvml.nvmlInit()
+h = pynvml.nvmlDeviceGetHandleByPciBusId(sys.argv[1])
+with open(sys.argv[2], "w", buffering=1) as f:
+    f.write("max,%f\\n" % pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+    while True:
+        f.write("%.6f,%d,%d\\n" % (time.time(), pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                   pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)))
+        time.sleep(0.002)
+"""
+
+
 class ClockSampler:
+    """SM clock and clock-event (throttle) reasons of this rank's GPU during the timed steps.
+    A separate process polls NVML every 2 ms from construction on (so it is running before
+    the timed region starts) and the samples time-stamped inside [start, stop] are kept; with
+    no NVML, `nvidia-smi -lms 200` runs over the same window."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
 
     def __init__(self, device):
         p = torch.cuda.get_device_properties(device)
         self.bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
         self.proc = None
         self.path = None
+        self.poller = None
+        try:
+            import pynvml  # noqa: F401  (the poller needs it)
+            fd, self.poll_path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.poller = subprocess.Popen([sys.executable, "-c", _NVML_POLL, self.bus, self.poll_path],
+                                           stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.poller = None
 
     def start(self):
+        if self.poller is not None:
+            # wait (at most 10 s) for the poller's first sample so the window is covered
+            for _ in range(1000):
+                with open(self.poll_path) as f:
+                    if f.read().count("\n") >= 2:
+                        break
+                if self.poller.poll() is not None:
+                    break
+                time.sleep(0.01)
+            self.t0 = time.time()
+            return
+        self.t0 = time.time()
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
@@ -119,6 +160,31 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
+        t1 = time.time()
+        if self.poller is not None:
+            time.sleep(0.005)
+            self.poller.terminate()
+            try:
+                self.poller.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.poller.kill()
+            mx, rows = None, []
+            with open(self.poll_path) as f:
+                for line in f:
+                    parts = line.strip().split(",")
+                    if parts[0] == "max" and len(parts) == 2:
+                        mx = float(parts[1])
+                    elif len(parts) == 3:
+                        rows.append((float(parts[0]), float(parts[1]), int(parts[2])))
+            os.unlink(self.poll_path)
+            inside = [r for r in rows if self.t0 <= r[0] <= t1]
+            if not inside and rows:  # a window shorter than the poll interval: nearest samples
+                inside = sorted(rows, key=lambda r: abs(r[0] - (self.t0 + t1) / 2))[:2]
+            if not inside:
+                return None
+            reasons = sorted(n for n, bit in self.REASONS.items() if any(r[2] & bit for r in inside))
+            return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": mx, "reasons": reasons,
+                    "samples": len(inside), "source": "nvml every 2 ms, samples inside the timed steps"}
         if self.proc is None:
             return None
         time.sleep(0.25)
@@ -141,7 +207,7 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "source": "nvidia-smi every 200 ms"}
 
 
 # ---- roofline bookkeeping -------------------------------------------------------------------
@@ -228,10 +294,10 @@ def run_ours(args, world, rank, local):
         del probe
     step.capture(x)
 
+    clocks = ClockSampler(dev)  # its poller starts now and is running by the timed steps
     for _ in range(args.warmup):
         one(step)
     step.check_status()
-    clocks = ClockSampler(dev)
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
