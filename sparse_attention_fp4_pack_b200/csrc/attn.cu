@@ -12,18 +12,20 @@
 // C = min(tiles, 8) CTAs (256 threads each) handles one query; CTA r takes tiles
 // r, r+C, ...:
 //   1. the fp32 queries arrive by one bulk copy into shared memory and become f16
-//      (times sm_scale*log2 e, so the softmax works in base 2), heads padded to 64 with
-//      zero rows; meanwhile each thread gathers its half of a selected 288 B entry;
+//      (times sm_scale*log2 e, so the softmax works in base 2), heads padded with zero
+//      rows up to the products' N; meanwhile each thread gathers its half of a selected
+//      288 B entry;
 //   2. the entries are dequantised into a 128 x 512 f16 tile in 128-byte-swizzled
 //      shared memory (E2M1 -> f16 by cvt times the E4M3 block scale, exact in f16);
 //      window tokens by E4M3 -> f16 cvt; empty slots become zero rows;
-//   3. S^T[128 keys x 64 heads] = Kt . Qs^T by tcgen05.mma (M=128, N=64, K=512) into
+//   3. S^T[128 keys x N heads] = Kt . Qs^T by tcgen05.mma (M=128, K=512) into
 //      tensor memory;
 //   4. per-head max / exp2 / sum across the 128 TMEM lanes by warp transpose
 //      reductions; a running max rescales the accumulated output when a CTA takes more
 //      than one tile; P^T goes to shared memory as f16;
-//   5. O^T[512 dims x 64 heads] += Kt^T . P^T with the same key tile read MN-major as
-//      the A operand (the latent is both key and value);
+//   5. O^T[512 dims x heads] += Kt^T . P^T with the same key tile read MN-major as
+//      the A operand (the latent is both key and value); both products take N = the
+//      cluster's heads rounded up to 16, 32 or 64, P^T in rows of that width;
 //   6. every CTA exports its O^T and (max, sum) per head in shared memory; after a
 //      cluster barrier CTA r merges heads [r*H/C, (r+1)*H/C) of all CTAs through
 //      distributed shared memory and writes the normalised output and log-sum-exp.
@@ -38,7 +40,7 @@ namespace csa2 {
 namespace cg = cooperative_groups;
 
 constexpr int kTile = 128;        // key slots per tile = UMMA M
-constexpr int kHeadsPad = 64;     // UMMA N
+constexpr int kHeadsPad = 64;     // most heads per cluster (largest UMMA N used)
 constexpr int kAttnThreads = 256;
 constexpr int kMaxCluster = 8;
 constexpr uint32_t kTmemCols = 512;
@@ -134,6 +136,24 @@ __device__ __forceinline__ float xpose_reduce(float (&v)[32], int lane) {
   return v[0];
 }
 
+// The same for 16 values: 4 exchange steps within each half-warp leave lane i with value
+// i mod 16 reduced over its 16 lanes; one more exchange adds the other half-warp.
+template <bool kMax>
+__device__ __forceinline__ float xpose_reduce16(float (&v)[16], int lane) {
+#pragma unroll
+  for (int n = 8; n >= 1; n >>= 1) {
+    const bool upper = (lane & n) != 0;
+#pragma unroll
+    for (int j = 0; j < n; ++j) {
+      const float send = upper ? v[j] : v[j + n];
+      const float keep = upper ? v[j + n] : v[j];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, n);
+      v[j] = kMax ? fmaxf(keep, recv) : keep + recv;
+    }
+  }
+  const float other = __shfl_xor_sync(0xffffffffu, v[0], 16);
+  return kMax ? fmaxf(v[0], other) : v[0] + other;
+}
 
 // One key slot's raw data for this thread's half of the 512 channels.
 struct SlotRaw {
@@ -275,10 +295,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
   // phase: setup
   bool timed_out = __syncthreads_or(tc::mbar_wait(mbar_q, 0, kMaxPolls) ? 0 : 1) != 0;
   // phase: queries landed
+  // The S product's N: this cluster's heads rounded up to 16, 32 or 64.  Query rows past NH
+  // up to NQ are zero; rows past NQ are never read.
+  const int NQ = NH <= 16 ? 16 : (NH <= 32 ? 32 : kHeadsPad);
   {  // fp32 staging -> f16 query tile (scaled), 8 channels per 16 B chunk
     const float qscale = a.sm_scale * 1.4426950408889634f;
 #pragma unroll 4
-    for (int i = tid; i < kHeadsPad * 64; i += kAttnThreads) {
+    for (int i = tid; i < NQ * 64; i += kAttnThreads) {
       const int h = i >> 6, ch = i & 63, db = ch >> 3, c = ch & 7;
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
       if (h < NH && !timed_out) {
@@ -317,7 +340,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
     if (tid == 0) {
       // N covers this cluster's heads only (rows past NH of the query tile are zero and the
       // softmax masks those columns)
-      const uint32_t idesc = tc::idesc_f16(kTile, NH <= 16 ? 16 : (NH <= 32 ? 32 : kHeadsPad), false, false);
+      const uint32_t idesc = tc::idesc_f16(kTile, NQ, false, false);
 #pragma unroll 4
       for (int ks = 0; ks < kD / 16; ++ks) {
         const int db = ks >> 2, kk = ks & 3;
@@ -332,18 +355,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
     tc::fence_after_sync();
     if (timed_out) break;
   // phase: qk done
-    uint32_t raw[32];
-    tc::tmem_ld32(lane_base + kColS + half * 32, raw);
     const bool kv = valid_s[key] != 0;
     float s[32], v[32];
+    if (NQ == 16) {  // heads 0..15 only: warps 0-3 take them, warps 4-7 have no columns
+      if (half == 0) {
+        uint32_t raw[16];
+        tc::tmem_ld16(lane_base + kColS, raw);
+        float v16[16];
 #pragma unroll
-    for (int jj = 0; jj < 32; ++jj) {
-      s[jj] = (kv && half * 32 + jj < NH) ? __uint_as_float(raw[jj]) : -INFINITY;  // pad heads: no keys
-      v[jj] = s[jj];
+        for (int jj = 0; jj < 16; ++jj) {
+          s[jj] = (kv && jj < NH) ? __uint_as_float(raw[jj]) : -INFINITY;
+          v16[jj] = s[jj];
+        }
+        const float m16 = xpose_reduce16<true>(v16, lane);
+        if (lane < 16) red_max[q4 * 64 + lane] = m16;
+      }
+    } else {
+      uint32_t raw[32];
+      tc::tmem_ld32(lane_base + kColS + half * 32, raw);
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) {
+        s[jj] = (kv && half * 32 + jj < NH) ? __uint_as_float(raw[jj]) : -INFINITY;  // pad heads: no keys
+        v[jj] = s[jj];
+      }
+      red_max[q4 * 64 + half * 32 + lane] = xpose_reduce<true>(v, lane);
     }
-    red_max[q4 * 64 + half * 32 + lane] = xpose_reduce<true>(v, lane);
     __syncthreads();
-    if (tid < kHeadsPad) {
+    if (tid < NQ) {
       const float mt = fmaxf(fmaxf(red_max[tid], red_max[64 + tid]), fmaxf(red_max[128 + tid], red_max[192 + tid]));
       const float mo = m_run[tid];
       const float mn = fmaxf(mo, mt);
@@ -351,7 +389,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
       m_run[tid] = mn;
     }
     __syncthreads();
-    if (processed > 0) {  // rescale the output accumulated from earlier tiles
+    if (processed > 0 && half * 32 < NQ) {  // rescale the output accumulated from earlier tiles
 #pragma unroll 1
       for (int mt = 0; mt < 4; ++mt) {
         uint32_t o[32];
@@ -362,23 +400,55 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
         tc::tmem_st32(ta, o);
       }
     }
-    uint32_t ph[16];
+    if (NQ == 16) {
+      if (half == 0) {
+        uint32_t ph[8];
+        float v16[16];
 #pragma unroll
-    for (int jj = 0; jj < 32; jj += 2) {
-      const float m0 = m_run[half * 32 + jj], m1 = m_run[half * 32 + jj + 1];
-      const float p0 = m0 == -INFINITY ? 0.0f : exp2f(s[jj] - m0);
-      const float p1 = m1 == -INFINITY ? 0.0f : exp2f(s[jj + 1] - m1);
-      __half2 hp = __floats2half2_rn(p0, p1);
-      ph[jj >> 1] = *reinterpret_cast<uint32_t*>(&hp);
-      const float2 back = __half22float2(hp);
-      v[jj] = back.x;  // the sum uses exactly the f16 values the PV product sees
-      v[jj + 1] = back.y;
+        for (int jj = 0; jj < 16; jj += 2) {
+          const float m0 = m_run[jj], m1 = m_run[jj + 1];
+          const float p0 = m0 == -INFINITY ? 0.0f : exp2f(s[jj] - m0);
+          const float p1 = m1 == -INFINITY ? 0.0f : exp2f(s[jj + 1] - m1);
+          __half2 hp = __floats2half2_rn(p0, p1);
+          ph[jj >> 1] = *reinterpret_cast<uint32_t*>(&hp);
+          const float2 back = __half22float2(hp);
+          v16[jj] = back.x;  // the sum uses exactly the f16 values the PV product sees
+          v16[jj + 1] = back.y;
+        }
+        // P^T rows of 16 heads (32 B, 32-byte swizzle)
+        *reinterpret_cast<uint4*>(Ps + tc::swz(key, 0, 32)) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+        *reinterpret_cast<uint4*>(Ps + tc::swz(key, 16, 32)) = make_uint4(ph[4], ph[5], ph[6], ph[7]);
+        const float s16 = xpose_reduce16<false>(v16, lane);
+        if (lane < 16) red_sum[q4 * 64 + lane] = s16;
+      }
+    } else {
+      uint32_t ph[16];
+#pragma unroll
+      for (int jj = 0; jj < 32; jj += 2) {
+        const float m0 = m_run[half * 32 + jj], m1 = m_run[half * 32 + jj + 1];
+        const float p0 = m0 == -INFINITY ? 0.0f : exp2f(s[jj] - m0);
+        const float p1 = m1 == -INFINITY ? 0.0f : exp2f(s[jj + 1] - m1);
+        __half2 hp = __floats2half2_rn(p0, p1);
+        ph[jj >> 1] = *reinterpret_cast<uint32_t*>(&hp);
+        const float2 back = __half22float2(hp);
+        v[jj] = back.x;  // the sum uses exactly the f16 values the PV product sees
+        v[jj + 1] = back.y;
+      }
+      // P^T rows of NQ heads (NQ * 2 bytes, swizzle of that width); with NQ = 32 the upper
+      // warps hold no heads of the product
+      if (NQ == kHeadsPad) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(Ps + tc::swz(key, half * 64 + c * 16, 128)) =
+              make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
+      } else if (half == 0) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(Ps + tc::swz(key, c * 16, 64)) =
+              make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
+      }
+      red_sum[q4 * 64 + half * 32 + lane] = xpose_reduce<false>(v, lane);
     }
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-      *reinterpret_cast<uint4*>(Ps + tc::sw128(key, half * 64 + c * 16)) =
-          make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
-    red_sum[q4 * 64 + half * 32 + lane] = xpose_reduce<false>(v, lane);
   // phase: softmax done
     tc::fence_async_smem();
     tc::fence_before_sync();
@@ -386,18 +456,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
     tc::fence_after_sync();
     // ---- O^T += Kt^T . P^T (key tile read MN-major) --------------------------------------
     if (tid == 0) {
-      constexpr uint32_t idesc = tc::idesc_f16(kTile, kHeadsPad, true, true);
+      // B = P^T [128 keys x NQ heads], MN-major, rows of rb = 2 NQ bytes: 8-row groups at
+      // 8 rb, 16 keys (one K step) at 16 rb
+      const uint32_t idesc = tc::idesc_f16(kTile, NQ, true, true);
+      const uint32_t rb = 2u * (uint32_t)NQ, pcode = tc::swizzle_code(rb);
 #pragma unroll 1
       for (int mt = 0; mt < 4; ++mt)
 #pragma unroll 4
         for (int ks = 0; ks < kTile / 16; ++ks) {
           const uint64_t ad = tc::smem_desc_sw128(tc::smem_u32(Ks + (2 * mt) * 16384 + ks * 2048), 16384, 1024);
-          const uint64_t bd = tc::smem_desc_sw128(tc::smem_u32(Ps + ks * 2048), 8192, 1024);
+          const uint64_t bd = tc::smem_desc(tc::smem_u32(Ps + ks * 16 * rb), 64u * rb, 8u * rb, pcode);
           tc::mma_f16(tmem + kColO + mt * 64, ad, bd, idesc, (ks > 0 || processed > 0) ? 1u : 0u);
         }
       tc::commit(mbar_mma);
     }
-    if (tid < kHeadsPad)
+    if (tid < NQ)
       l_run[tid] = l_run[tid] * alpha[tid] + ((red_sum[tid] + red_sum[64 + tid]) + (red_sum[128 + tid] + red_sum[192 + tid]));
     timed_out = __syncthreads_or(tc::mbar_wait(mbar_mma, commits & 1, kMaxPolls) ? 0 : 1) != 0;
     ++commits;
@@ -411,15 +484,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_tc_kernel(AttnArgs a) {
   }
 
   // ---- export O^T (fp32 [head][channel]) into the key area --------------------------------
-  if (processed > 0 && !timed_out && half * 32 < NH) {
+  // Items (dim block mt, column group g of cw heads) are shared by the two warp halves.
+  if (processed > 0 && !timed_out) {
+    const int cw = NQ == 16 ? 16 : 32;
+    const int ngroups = (NH + cw - 1) / cw;
 #pragma unroll 1
-    for (int mt = 0; mt < 4; ++mt) {
-      uint32_t o[32];
-      tc::tmem_ld32(lane_base + kColO + mt * 64 + half * 32, o);
+    for (int item = half; item < 4 * ngroups; item += 2) {
+      const int mt = item / ngroups, g = item - mt * ngroups;
+      const uint32_t ta = lane_base + kColO + mt * 64 + g * cw;
       const int d = mt * 128 + q4 * 32 + lane;
+      if (cw == 16) {
+        uint32_t o[16];
+        tc::tmem_ld16(ta, o);
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj)
-        if (half * 32 + jj < NH) Of[(half * 32 + jj) * kD + d] = __uint_as_float(o[jj]);
+        for (int jj = 0; jj < 16; ++jj)
+          if (jj < NH) Of[jj * kD + d] = __uint_as_float(o[jj]);
+      } else {
+        uint32_t o[32];
+        tc::tmem_ld32(ta, o);
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj)
+          if (g * 32 + jj < NH) Of[(g * 32 + jj) * kD + d] = __uint_as_float(o[jj]);
+      }
     }
   }
   tc::fence_before_sync();

@@ -599,13 +599,13 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
 
 // ------------------------------------------------------------------------------------
 // Top-K selection over one query's keys: a thread-block cluster of C CTAs (C <= 8) per
-// query, each holding a contiguous slice of the keys in registers (512 threads x 32 keys,
-// index order = thread order).
+// query, each holding a contiguous slice of the keys in shared memory (1024 threads x
+// 2^PS keys, index order = thread order).
 //
 // Most-significant-digit radix select with adaptive digit windows:
 //   0. the cluster reduces min / max / count of the valid (non-zero) keys; bits above the
 //      highest bit where min and max differ are common to every key, so the first
-//      11-bit digit starts right below them (keys spread over the histogram instead of
+//      10-bit digit starts right below them (keys spread over the histogram instead of
 //      piling into a few bins);
 //   1. per level: each CTA histograms the digit of the keys matching the prefix chosen
 //      so far, the histograms are summed across the cluster through distributed shared
@@ -614,16 +614,14 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
 //   2. one ordered pass writes the selected keys in index order — positions come from
 //      block-wide prefix sums plus a prefix over the cluster's CTAs — and the keys equal
 //      to the K-th (all bits resolved) lowest index first.
-// The result (contents and order) is deterministic.
+// The result (contents and order) is deterministic.  PS = 4 (16 keys per thread) serves
+// long key lists; PS = 2 (4 keys per thread) a list of at most 4,096 keys, which then
+// takes a quarter of the per-key work.
 // ------------------------------------------------------------------------------------
 constexpr int kSelThreads = 1024;
-constexpr int kPerShift = 4;
-constexpr int kPer = 1 << kPerShift;             // keys per thread per chunk
-constexpr int kSelChunk = kSelThreads * kPer;    // keys per CTA per chunk (16384)
 constexpr int kDigitBits = 10;                   // radix digit: 1024 bins
 constexpr int kBins = 1 << kDigitBits;
 constexpr int kMaxCluster = 8;
-constexpr int kKeyRow = kPer + 1;                // a thread's keys in shared memory, padded
 // Shared memory, in 32-bit words:
 //   sub   [kBins/2][32]: per-lane counters, two 16-bit bins per word (bin 2c in the low
 //         half of column c); once the levels are done, the selected items are staged here
@@ -633,12 +631,19 @@ constexpr int kKeyRow = kPer + 1;                // a thread's keys in shared me
 //   scan scratch (32 x u64), cluster exchange words (16) and misc (8), padded to 64 words
 //   blk   [CSA2_MAX_K] the query's Reindex block ids
 // Column l collects lane l of every warp: at most 32 warps x 16 keys = 512 increments per
-// 16,384-key chunk.  launch_index gives a query one CTA per 16,384 keys, up to 8, and the
-// host caps max_n_vis at 2^23, so a CTA holds at most 2^20 keys (64 chunks) and a 16-bit
+// chunk.  The launcher gives a query one CTA per chunk, up to 8, and the host caps
+// max_n_vis at 2^23, so a CTA holds at most 2^20 keys (64 chunks of 16,384) and a 16-bit
 // counter reaches at most 64 x 512 = 2^15.
 constexpr int kSubWords = kBins / 2 * 32;
-constexpr int kKeyWords = kSelThreads * kKeyRow;
-constexpr int kSelSmem = (kSubWords + kKeyWords + 2 * kBins + 128 + 64 + CSA2_MAX_K) * 4;
+template <int PS>
+struct SelShape {
+  static constexpr int kPer = 1 << PS;                  // keys per thread per chunk
+  static constexpr int kChunk = kSelThreads * kPer;     // keys per CTA per chunk
+  static constexpr int kKeyRow = kPer + 1;              // a thread's keys in shared memory, padded
+  static constexpr int kKeyWords = kSelThreads * kKeyRow;
+  static constexpr int kSmem = (kSubWords + kKeyWords + 2 * kBins + 128 + 64 + CSA2_MAX_K) * 4;
+};
+static_assert(2 * CSA2_MAX_K <= kSubWords, "selected items are staged in the counter area");
 
 struct SelectArgs {
   const uint32_t* keys;
@@ -741,7 +746,13 @@ __device__ __forceinline__ void find_bin_warp(const uint32_t* hist, int nb, uint
   }
 }
 
+template <int PS>
 __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
+  constexpr int kPerShift = PS;
+  constexpr int kPer = SelShape<PS>::kPer;
+  constexpr int kSelChunk = SelShape<PS>::kChunk;
+  constexpr int kKeyRow = SelShape<PS>::kKeyRow;
+  constexpr int kKeyWords = SelShape<PS>::kKeyWords;
   chain_enter();
   // phase: started
   namespace cg = cooperative_groups;
@@ -791,40 +802,46 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
   for (int i = tid; i < kSubWords / 4; i += kSelThreads)  // counters start at zero
     reinterpret_cast<uint4*>(sub)[i] = make_uint4(0u, 0u, 0u, 0u);
 
-  // chunk ch of the slice -> ks (item lo + ch*16384 + 32t + e is key e of thread t; 0 past hi)
+  // chunk ch of the slice -> ks (item lo + ch*kSelChunk + kPer*t + e is key e of thread t; 0 past hi)
   const uint32_t* mk = ks + tid * kKeyRow;
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u, cnt = 0u;  // over the valid (non-zero) keys
   auto load_chunk = [&](int ch, bool range) {
     const int64_t c0 = lo + (int64_t)ch * kSelChunk;
     const int64_t cn = hi - c0 < kSelChunk ? hi - c0 : kSelChunk;
     __syncthreads();  // earlier readers of ks are done
-#pragma unroll 2
-    for (int i4 = tid; i4 < kSelChunk / 4; i4 += kSelThreads) {
-      const int i = 4 * i4;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (i + 4 <= cn) {
-        v = *reinterpret_cast<const uint4*>(keys + c0 + i);
-      } else if (i < cn) {
-        v.x = keys[c0 + i];
-        v.y = i + 1 < cn ? keys[c0 + i + 1] : 0u;
-        v.z = i + 2 < cn ? keys[c0 + i + 2] : 0u;
-      }
-      if (range) {
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    constexpr int kLoads = kSelChunk / 4 / kSelThreads;  // 16 B loads per thread, all in flight
+    uint4 v[kLoads];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (w[u] != 0u) {
-            kmin = min(kmin, w[u]);
-            kmax = max(kmax, w[u]);
+    for (int u = 0; u < kLoads; ++u) {
+      const int i = 4 * (tid + u * kSelThreads);
+      v[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (i + 4 <= cn) {
+        v[u] = *reinterpret_cast<const uint4*>(keys + c0 + i);
+      } else if (i < cn) {
+        v[u].x = keys[c0 + i];
+        v[u].y = i + 1 < cn ? keys[c0 + i + 1] : 0u;
+        v[u].z = i + 2 < cn ? keys[c0 + i + 2] : 0u;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kLoads; ++u) {
+      const int i = 4 * (tid + u * kSelThreads);
+      if (range) {
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (w[e] != 0u) {
+            kmin = min(kmin, w[e]);
+            kmax = max(kmax, w[e]);
             ++cnt;
           }
         }
       }
       uint32_t* d = ks + (i >> kPerShift) * kKeyRow + (i & (kPer - 1));
-      d[0] = v.x;
-      d[1] = v.y;
-      d[2] = v.z;
-      d[3] = v.w;
+      d[0] = v[u].x;
+      d[1] = v[u].y;
+      d[2] = v[u].z;
+      d[3] = v[u].w;
     }
     __syncthreads();
   };
@@ -1205,12 +1222,24 @@ cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t
   const int64_t items = mode == kFlat ? max_n_vis
                         : mode == kHier ? (max_n_vis + block - 1) / block
                                         : (int64_t)n_blocks * block;
-  int64_t c = (items + kSelChunk - 1) / kSelChunk;  // one CTA per 16384 keys
-  s.csize = (int)(c < 1 ? 1 : (c > kMaxCluster ? kMaxCluster : c));
-  e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelSmem);
-  if (e != cudaSuccess) return e;
-  e = launch_chained(select_kernel, dim3((unsigned)s.csize, (unsigned)BQ), dim3(kSelThreads), kSelSmem, stream,
-                     (unsigned)s.csize, s);
+  // At most 4,096 keys: one CTA with 4 keys per thread.  Otherwise one CTA per 16,384 keys
+  // (16 per thread), up to 8.  (Splitting a 16,384-key list over a cluster of 4-key CTAs
+  // measured no faster: each radix level then waits on two cluster barriers and a
+  // remote histogram sum, which cost what the shorter count saves.)
+  if (items <= SelShape<2>::kChunk) {
+    s.csize = 1;
+    e = cudaFuncSetAttribute(select_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, SelShape<2>::kSmem);
+    if (e != cudaSuccess) return e;
+    e = launch_chained(select_kernel<2>, dim3((unsigned)s.csize, (unsigned)BQ), dim3(kSelThreads),
+                       SelShape<2>::kSmem, stream, (unsigned)s.csize, s);
+  } else {
+    const int64_t c = (items + SelShape<4>::kChunk - 1) / SelShape<4>::kChunk;
+    s.csize = (int)(c < 1 ? 1 : (c > kMaxCluster ? kMaxCluster : c));
+    e = cudaFuncSetAttribute(select_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, SelShape<4>::kSmem);
+    if (e != cudaSuccess) return e;
+    e = launch_chained(select_kernel<4>, dim3((unsigned)s.csize, (unsigned)BQ), dim3(kSelThreads),
+                       SelShape<4>::kSmem, stream, (unsigned)s.csize, s);
+  }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -60,9 +60,26 @@ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t byte) {
   return row * 128u + ((((byte >> 4) ^ row) & 7u) << 4) + (byte & 15u);
 }
 
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+// Byte offset of (row, byte-in-row) in a tile of rb-byte rows, rb = 32, 64 or 128, under the
+// swizzle of that width (the 16-byte chunk index is XORed with address bits 7 and up, i.e.
+// with row / (128 / rb)).
+__device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t byte, uint32_t rb) {
+  const uint32_t shift = rb == 128u ? 0u : (rb == 64u ? 1u : 2u);
+  return row * rb + ((((byte >> 4) ^ (row >> shift)) & ((rb >> 4) - 1u)) << 4) + (byte & 15u);
+}
+
+// Shared-memory matrix descriptor (sm_100 form): start address, leading and stride byte
+// offsets, swizzle layout code (2: 128 B, 4: 64 B, 6: 32 B).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                              uint32_t layout) {
   return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+         ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)(layout & 7u) << 61);
+}
+// Swizzle layout code of rb-byte rows.
+__host__ __device__ constexpr uint32_t swizzle_code(uint32_t rb) { return rb == 128u ? 2u : (rb == 64u ? 4u : 6u); }
+
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return smem_desc(saddr, lbo_bytes, sbo_bytes, 2u);
 }
 
 // kind::f16 with f16 A/B and f32 accumulation.

@@ -64,6 +64,30 @@ def test_heads_and_lists(orc, H):
     assert np.abs(lse - l_ref).max() < 1e-2
 
 
+@pytest.mark.parametrize("H,B,Q", [(64, 2, 5), (32, 4, 4)])
+def test_head_groups_of_32(orc, H, B, Q):
+    """Enough queries that a query's heads go to clusters of 32 (64 heads in two groups, or
+    32 heads in one): both products then run with N = 32 and 64-byte P^T rows."""
+    N, K = 3000, 512
+    kvp, o_kv = _pool(orc, 120 + H, N)
+    rng = np.random.default_rng(120 + Q)
+    base = torch.tensor([0, 1400, 100, 2000][:B], dtype=torch.int64)
+    topk = np.stack([np.stack([rng.choice(1000, K, replace=False) for _ in range(Q)]) for _ in range(B)])
+    topk = topk.astype(np.int32)
+    topk[0, 1, 200:] = -1
+    q = synth.queries(121 + H, B, Q, H)
+    S_w = 128 + Q - 1
+    swa = synth.swa_window(122, B, S_w)
+    q_pos = torch.tensor([[3000 + 10 * b + i for i in range(Q)] for b in range(B)], dtype=torch.int64)
+    swa_start = q_pos[:, -1] - S_w + 1
+    out, lse, st = _run(q, kvp, base, torch.from_numpy(topk), swa, swa_start, q_pos)
+    assert st == 0
+    o_ref, l_ref = orc.sparse_attn(q.numpy(), o_kv, base.numpy(), topk, swa.numpy(), swa_start.numpy(),
+                                   q_pos.numpy(), SM)
+    assert_attn_close(out, o_ref)
+    assert np.abs(lse - l_ref).max() < 1e-2
+
+
 def test_tiny_workload_layer(orc):
     wl = synth.workload("tiny")
     kv, ik = synth.seq_tokens(wl, 0, device="cuda")
