@@ -28,7 +28,8 @@ cudaError_t launch_sparse_attn(const float* q, const uint8_t* kv_pool, int64_t p
 namespace {
 
 constexpr int64_t kMaxQueries = 65535;  // grid.y limit of the per-query kernels
-constexpr int64_t kMaxNVis = (int64_t)1 << 23;  // keeps the selection's 16-bit counters in range
+constexpr int64_t kMaxNVis = (int64_t)1 << 23;  // largest accepted visible count: a selection CTA then
+                                                // holds at most 2^20 keys (64 reloaded chunks)
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 

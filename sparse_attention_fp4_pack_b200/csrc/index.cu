@@ -623,18 +623,18 @@ constexpr int kDigitBits = 10;                   // radix digit: 1024 bins
 constexpr int kBins = 1 << kDigitBits;
 constexpr int kMaxCluster = 8;
 // Shared memory, in 32-bit words:
-//   sub   [kBins/2][32]: per-lane counters, two 16-bit bins per word (bin 2c in the low
-//         half of column c); once the levels are done, the selected items are staged here
+//   sub   [kBins] one 32-bit counter per bin, counted by shared-memory atomics (lanes of a
+//         warp that hit the same bin are serialised by the hardware; that measured cheaper
+//         than lane-private counters, whose per-bin sums cost more than the collisions);
+//         once the levels are done, the selected items are staged here
 //   ks    [kSelThreads][kKeyRow]: the chunk of keys, thread t's kPer keys in row t (the pad
 //         word puts key e of consecutive threads in consecutive banks)
 //   hist  [kBins] this CTA's histogram;  hsum [kBins] the cluster's
 //   scan scratch (32 x u64), cluster exchange words (16) and misc (8), padded to 64 words
 //   blk   [CSA2_MAX_K] the query's Reindex block ids
-// Column l collects lane l of every warp: at most 32 warps x 16 keys = 512 increments per
-// chunk.  The launcher gives a query one CTA per chunk, up to 8, and the host caps
-// max_n_vis at 2^23, so a CTA holds at most 2^20 keys (64 chunks of 16,384) and a 16-bit
-// counter reaches at most 64 x 512 = 2^15.
-constexpr int kSubWords = kBins / 2 * 32;
+// A CTA holds at most 2^20 keys (the host caps max_n_vis at 2^23, a query gets up to 8
+// CTAs), so no 32-bit counter can overflow.
+constexpr int kSubWords = kBins > 2 * CSA2_MAX_K ? kBins : 2 * CSA2_MAX_K;
 template <int PS>
 struct SelShape {
   static constexpr int kPer = 1 << PS;                  // keys per thread per chunk
@@ -901,8 +901,6 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
         const int sh = p >= kDigitBits - 1 ? p - (kDigitBits - 1) : 0;
         const int width = p - sh + 1;
         const uint32_t nb = 1u << width;
-        // each lane counts into its own column, so a warp's increments never collide
-        // (keys of similar scores share bins)
         for (int ch = 0; ch < nchunks; ++ch) {
           if (nchunks > 1) load_chunk(ch, false);
 #pragma unroll 4
@@ -910,26 +908,15 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
             const uint32_t key = mk[e];
             if (key != 0u && (key & mask) == prefix) {
               const uint32_t bin = (key >> sh) & (nb - 1u);
-              atomicAdd(&sub[(bin >> 1) * 32 + lane], (bin & 1u) ? 0x10000u : 1u);
+              atomicAdd(&sub[bin], 1u);
             }
           }
         }
         __syncthreads();
-        // bin totals: thread c sums column c, reading word (j + c) % 32 at step j so that
-        // the 32 lanes of a warp read 32 different banks; the column is zeroed behind it
-        for (int c = tid; c < (int)(nb >> 1); c += kSelThreads) {
-          uint32_t* col = sub + c * 32;
-          uint32_t lo16 = 0u, hi16 = 0u;
-#pragma unroll 4
-          for (int j = 0; j < 32; ++j) {
-            const int w = (j + c) & 31;
-            const uint32_t x = col[w];
-            col[w] = 0u;
-            lo16 += x & 0xFFFFu;
-            hi16 += x >> 16;
-          }
-          hist[2 * c] = lo16;
-          hist[2 * c + 1] = hi16;
+        // bin totals to hist; the counters are zeroed for the next level
+        for (int c = tid; c < (int)nb; c += kSelThreads) {
+          hist[c] = sub[c];
+          sub[c] = 0u;
         }
   // phase: level counted
         const uint32_t* hs = hist;
