@@ -19,9 +19,11 @@ _lib = None
 
 
 def lib():
+    """The oracle's shared library.  CSA2_ORACLE_LIB, when set, names another build of
+    ``csa2_oracle.c`` to load instead (the mutation test loads planted-mistake builds)."""
     global _lib
     if _lib is None:
-        path = _build.build()
+        path = os.environ.get("CSA2_ORACLE_LIB") or _build.build()
         L = ctypes.CDLL(path)
         c_p = ctypes.c_void_p
         i64, i32, dbl, flt = ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_float

@@ -12,17 +12,21 @@ SRC = os.path.join(HERE, "csa2_oracle.c")
 LIB = os.path.join(HERE, "liboracle.so")
 
 
+# IEEE semantics: no contraction of a*b+c into fma, no fast-math
+CFLAGS = ["-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math"]
+
+
+def compile_to(src: str, out: str) -> str:
+    """Compile one oracle source file into the shared library `out`."""
+    subprocess.run(["gcc", *CFLAGS, "-o", out, src, "-lm"], check=True)
+    return out
+
+
 def build(force: bool = False) -> str:
     """Build liboracle.so if it is missing or older than its source; return its path."""
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
         return LIB
-    cmd = [
-        "gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
-        # IEEE semantics: no contraction of a*b+c into fma, no fast-math
-        "-ffp-contract=off", "-fno-fast-math",
-        "-o", LIB + ".tmp", SRC, "-lm",
-    ]
-    subprocess.run(cmd, check=True)
+    compile_to(SRC, LIB + ".tmp")
     os.replace(LIB + ".tmp", LIB)
     return LIB
 
