@@ -97,6 +97,31 @@ def max_over_ranks(x, world):
 
 
 # ---- clocks during the timed region ---------------------------------------------------------
+def step_stats(ms_list):
+    """Median, 10th and 90th percentile (nearest rank) of per-step device times in ms."""
+    if not ms_list:
+        return None
+    s = sorted(ms_list)
+
+    def pct(p):
+        return s[min(len(s) - 1, max(0, math.ceil(p / 100.0 * len(s)) - 1))]
+
+    return {"median": round(statistics.median(s), 4), "p10": round(pct(10), 4), "p90": round(pct(90), 4),
+            "n": len(s)}
+
+
+def cpu_model():
+    """The host CPU's model name (first 'model name' of /proc/cpuinfo), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 # Separate process (no share of this process's interpreter lock): read-only NVML queries of
 # one GPU every 2 ms, one "time,sm_mhz,reasons_bitmask" line each, until terminated.
 _NVML_POLL = """
@@ -302,9 +327,11 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     clocks.start()
     total_ms = 0.0
+    step_ms = []
     for _ in range(args.steps):
         ms, _ = one(step)
         total_ms += ms
+        step_ms.append(ms)
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
@@ -346,6 +373,7 @@ def run_ours(args, world, rank, local):
     line = {
         "metric": METRIC, "value": round(us_per_token, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 4),
+        "ms_per_step_rank0": step_stats(step_ms),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": DTYPE,
         "data": "synthetic (seeded)",
         "config": {"workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}", "B": wl.B, "Q": wl.Q,
@@ -525,7 +553,7 @@ def main():
                     "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
                     "config": {"workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}"},
                     "cpu_baseline": {"value": round(v, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
-                                     "sample": sample},
+                                     "sample": sample, "cpu_model": cpu_model()},
                     "e2e": {"value": round(v, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
             print(json.dumps(line, ensure_ascii=False), flush=True)
         if world > 1:
@@ -542,7 +570,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample = time_oracle(wl, args.cpu_seqs, 1, 0, "cuda")
         line["cpu_baseline"] = {"value": round(v, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": sample}
+                                "sample": sample, "cpu_model": cpu_model()}
     if rank == 0:
         print(json.dumps(line, ensure_ascii=False), flush=True)
     if world > 1:

@@ -67,6 +67,7 @@ def test_reference_arm_under_torchrun_two_ranks():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["unit"] == "µs/token"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["value"] > 0
+    assert "cpu_model" in d["cpu_baseline"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0
 
 
@@ -83,3 +84,14 @@ def test_launch_count_matches_the_schedule():
     assert step.launches_per_step() == 45
     step.schedule, step.hier = ["full", "reuse"], False
     assert step.launches_per_step() == 1 + 2 + 1 + 1
+
+
+def test_step_stats_nearest_rank():
+    """ms_per_step_rank0 in the bench line: median and nearest-rank 10th / 90th percentiles."""
+    import bench
+    assert bench.step_stats([]) is None
+    st = bench.step_stats([float(v) for v in (7, 1, 9, 3, 5, 2, 8, 4, 10, 6)])
+    assert st == {"median": 5.5, "p10": 1.0, "p90": 9.0, "n": 10}
+    st = bench.step_stats([0.25, 0.75, 0.5])
+    assert st["median"] == 0.5 and st["p10"] == 0.25 and st["p90"] == 0.75 and st["n"] == 3
+    assert isinstance(bench.cpu_model(), (str, type(None)))
