@@ -1,8 +1,10 @@
 """Thin ctypes binding of libcsa2 (C ABI in include/csa2.h).
 
-Argument marshalling only: every function checks tensor devices/dtypes/shapes, passes
-raw device pointers and the current CUDA stream to the C entry point of the same name,
-and raises CSA2Error on a non-OK status.  All compute runs in libcsa2's kernels; there
+Argument marshalling only: every function checks that its tensors' shapes agree with the
+sizes it passes (the C entry points take sizes and cannot see a buffer's extent, so a
+smaller buffer would be accessed out of bounds), then their devices, dtypes and layout,
+passes raw device pointers and the current CUDA stream to the C entry point of the same
+name, and raises CSA2Error on a non-OK status.  All compute runs in libcsa2's kernels; there
 is no other code path.  Workspaces are plain uint8 device tensors from torch's
 allocator (``workspace``).
 """
@@ -97,6 +99,28 @@ def _need(t, dtype, name, ndim=None):
         raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
 
 
+def _shape(t, shape, name):
+    """Raise unless `t` (when given) has exactly `shape`; None in `shape` matches any size.
+    The C entry points take sizes, not buffers, and cannot check a buffer's extent: a
+    tensor smaller than the sizes say would be read or written out of bounds."""
+    if t is None:
+        return
+    if t.dim() != len(shape) or any(e is not None and d != e for d, e in zip(t.shape, shape)):
+        want = ", ".join("*" if e is None else str(e) for e in shape)
+        raise ValueError(f"{name} must have shape ({want}), got {tuple(t.shape)}")
+
+
+def _rows(t, n, name):
+    """Raise unless the 1-D `t` (when given) has at least n entries (per-sequence arrays)."""
+    if t is not None and (t.dim() != 1 or t.shape[0] < n):
+        raise ValueError(f"{name} must be 1-D with at least {n} entries, got {tuple(t.shape)}")
+
+
+def _status(t):
+    if t is not None and (t.dtype != torch.int32 or t.numel() < 1 or not t.is_cuda):
+        raise ValueError("dev_status must be a CUDA int32 tensor with at least one element")
+
+
 def workspace(nbytes: int, device=None) -> torch.Tensor:
     """A uint8 device buffer usable as csa2 workspace (torch's allocator aligns to 512 B)."""
     return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device or "cuda")
@@ -119,19 +143,33 @@ def version() -> int:
 def csa2_pack_kv(kv, ik, ratio, kv_pool, ik_pool, dst_entry=None, dev_status=None, stream=None):
     """kv bf16 [T,512], ik bf16 [T,128] -> entries written into kv_pool u8 [P,288] and
     ik_pool u8 [P,68] (slots dst_entry int64 [T/ratio], or 0..T/ratio-1)."""
+    _shape(kv, (None, D), "kv")
+    T = kv.shape[0]
+    _shape(ik, (T, DI), "ik")
+    _shape(kv_pool, (None, KV_BYTES), "kv_pool")
+    _shape(ik_pool, (kv_pool.shape[0], IK_BYTES), "ik_pool")
+    if dst_entry is not None and (dst_entry.dim() != 1 or dst_entry.numel() != T // max(int(ratio), 1)):
+        raise ValueError("dst_entry must hold one slot per new entry (T // ratio)")
     _need(kv, torch.bfloat16, "kv", 2)
     _need(ik, torch.bfloat16, "ik", 2)
     _need(kv_pool, torch.uint8, "kv_pool", 2)
     _need(ik_pool, torch.uint8, "ik_pool", 2)
     _need(dst_entry, torch.int64, "dst_entry", 1)
-    T = kv.shape[0]
-    assert kv.shape == (T, D) and ik.shape == (T, DI)
-    assert kv_pool.shape[1] == KV_BYTES and ik_pool.shape[1] == IK_BYTES and kv_pool.shape[0] == ik_pool.shape[0]
-    if dst_entry is not None and dst_entry.numel() != T // max(int(ratio), 1):
-        raise ValueError("dst_entry must hold one slot per new entry (T // ratio)")
+    _status(dev_status)
     _check(lib().csa2_pack_kv(_ptr(kv), _ptr(ik), T, int(ratio), _ptr(dst_entry), kv_pool.shape[0],
                               _ptr(kv_pool), _ptr(ik_pool), _ptr(dev_status), _stream(stream)),
            "csa2_pack_kv")
+
+
+def _query_dims(q, w, ik_pool, seq_base, n_vis):
+    """(B, Q, HI) of an indexer call, after checking the shapes its inputs must share."""
+    _shape(q, (None, None, None, DI), "q")
+    B, Q, HI, _ = q.shape
+    _shape(w, (B, Q, HI), "w")
+    _shape(ik_pool, (None, IK_BYTES), "ik_pool")
+    _rows(seq_base, B, "seq_base")
+    _shape(n_vis, (B, Q), "n_vis")
+    return B, Q, HI
 
 
 # ---- a2/a3 ------------------------------------------------------------------------------
@@ -143,6 +181,9 @@ def csa2_index_full(q, w, ik_pool, seq_base, n_vis, K, max_n_vis, topk, topk_sco
                     dev_status=None, stream=None):
     """q f32 [B,Q,HI,128], w f32 [B,Q,HI], ik_pool u8 [P,68], seq_base i64 [B],
     n_vis i32 [B,Q] -> topk i32 [B,Q,K] (+ topk_score f32 [B,Q,K])."""
+    B, Q, HI = _query_dims(q, w, ik_pool, seq_base, n_vis)
+    _shape(topk, (B, Q, K), "topk")
+    _shape(topk_score, (B, Q, K), "topk_score")
     _need(q, torch.float32, "q", 4)
     _need(w, torch.float32, "w", 3)
     _need(ik_pool, torch.uint8, "ik_pool", 2)
@@ -150,7 +191,7 @@ def csa2_index_full(q, w, ik_pool, seq_base, n_vis, K, max_n_vis, topk, topk_sco
     _need(n_vis, torch.int32, "n_vis", 2)
     _need(topk, torch.int32, "topk", 3)
     _need(topk_score, torch.float32, "topk_score", 3)
-    B, Q, HI, _ = q.shape
+    _status(dev_status)
     if ws is None:
         ws = workspace(csa2_index_full_workspace_size(B, Q, HI, K, max_n_vis), q.device)
     _check(lib().csa2_index_full(_ptr(q), _ptr(w), _ptr(ik_pool), ik_pool.shape[0], _ptr(seq_base),
@@ -166,6 +207,9 @@ def csa2_index_hier_workspace_size(B, Q, HI, n_blocks, block, max_n_vis):
 
 def csa2_index_hier(q, w, ik_pool, seq_base, n_vis, n_blocks, block, max_n_vis, blocks, block_score=None,
                     ws=None, dev_status=None, stream=None):
+    B, Q, HI = _query_dims(q, w, ik_pool, seq_base, n_vis)
+    _shape(blocks, (B, Q, n_blocks), "blocks")
+    _shape(block_score, (B, Q, n_blocks), "block_score")
     _need(q, torch.float32, "q", 4)
     _need(w, torch.float32, "w", 3)
     _need(ik_pool, torch.uint8, "ik_pool", 2)
@@ -173,7 +217,7 @@ def csa2_index_hier(q, w, ik_pool, seq_base, n_vis, n_blocks, block, max_n_vis, 
     _need(n_vis, torch.int32, "n_vis", 2)
     _need(blocks, torch.int32, "blocks", 3)
     _need(block_score, torch.float32, "block_score", 3)
-    B, Q, HI, _ = q.shape
+    _status(dev_status)
     if ws is None:
         ws = workspace(csa2_index_hier_workspace_size(B, Q, HI, n_blocks, block, max_n_vis), q.device)
     _check(lib().csa2_index_hier(_ptr(q), _ptr(w), _ptr(ik_pool), ik_pool.shape[0], _ptr(seq_base),
@@ -190,6 +234,10 @@ def csa2_reindex_workspace_size(B, Q, HI, n_blocks, block, K):
 
 def csa2_reindex(q, w, ik_pool, seq_base, n_vis, blocks, block, K, topk, topk_score=None, ws=None,
                  dev_status=None, stream=None):
+    B, Q, HI = _query_dims(q, w, ik_pool, seq_base, n_vis)
+    _shape(blocks, (B, Q, None), "blocks")
+    _shape(topk, (B, Q, K), "topk")
+    _shape(topk_score, (B, Q, K), "topk_score")
     _need(q, torch.float32, "q", 4)
     _need(w, torch.float32, "w", 3)
     _need(ik_pool, torch.uint8, "ik_pool", 2)
@@ -198,7 +246,7 @@ def csa2_reindex(q, w, ik_pool, seq_base, n_vis, blocks, block, K, topk, topk_sc
     _need(blocks, torch.int32, "blocks", 3)
     _need(topk, torch.int32, "topk", 3)
     _need(topk_score, torch.float32, "topk_score", 3)
-    B, Q, HI, _ = q.shape
+    _status(dev_status)
     n_blocks = blocks.shape[-1]
     if ws is None:
         ws = workspace(csa2_reindex_workspace_size(B, Q, HI, n_blocks, block, K), q.device)
@@ -216,6 +264,10 @@ def csa2_reindex_static(q, w, ik_pool, seq_base, n_vis, blocks, block, K, topk, 
                         dev_status=None, stream=None):
     """csa2_reindex with the library's own static device scratch instead of a workspace:
     for callers that cannot allocate device memory for the call (see include/csa2.h)."""
+    B, Q, HI = _query_dims(q, w, ik_pool, seq_base, n_vis)
+    _shape(blocks, (B, Q, None), "blocks")
+    _shape(topk, (B, Q, K), "topk")
+    _shape(topk_score, (B, Q, K), "topk_score")
     _need(q, torch.float32, "q", 4)
     _need(w, torch.float32, "w", 3)
     _need(ik_pool, torch.uint8, "ik_pool", 2)
@@ -224,7 +276,7 @@ def csa2_reindex_static(q, w, ik_pool, seq_base, n_vis, blocks, block, K, topk, 
     _need(blocks, torch.int32, "blocks", 3)
     _need(topk, torch.int32, "topk", 3)
     _need(topk_score, torch.float32, "topk_score", 3)
-    B, Q, HI, _ = q.shape
+    _status(dev_status)
     n_blocks = blocks.shape[-1]
     _check(lib().csa2_reindex_static(_ptr(q), _ptr(w), _ptr(ik_pool), ik_pool.shape[0], _ptr(seq_base),
                                      _ptr(n_vis), _ptr(blocks), n_blocks, block, B, Q, HI, K, _ptr(topk),
@@ -241,6 +293,20 @@ def csa2_sparse_attn(q, kv_pool, seq_base, topk, swa, swa_start, q_pos, sm_scale
                      ws=None, dev_status=None, stream=None):
     """q f32 [B,Q,H,512]; kv_pool u8 [P,288]; topk i32 [B,Q,K]; swa u8 [B,S_w,512] or None;
     swa_start i64 [B]; q_pos i64 [B,Q] -> out f32 [B,Q,H,512], lse f32 [B,Q,H]."""
+    _shape(q, (None, None, None, D), "q")
+    B, Q, H, _ = q.shape
+    _shape(kv_pool, (None, KV_BYTES), "kv_pool")
+    _rows(seq_base, B, "seq_base")
+    _shape(topk, (B, Q, None), "topk")
+    _shape(swa, (None, None, D), "swa")
+    if swa is not None and swa.shape[0] < B:
+        raise ValueError(f"swa must hold at least {B} sequences, got {tuple(swa.shape)}")
+    if swa is not None and swa.shape[1] > 0 and swa_start is None:
+        raise ValueError("swa_start is required with a window buffer")
+    _rows(swa_start, B, "swa_start")
+    _shape(q_pos, (B, Q), "q_pos")
+    _shape(out, (B, Q, H, D), "out")
+    _shape(lse, (B, Q, H), "lse")
     _need(q, torch.float32, "q", 4)
     _need(kv_pool, torch.uint8, "kv_pool", 2)
     _need(seq_base, torch.int64, "seq_base", 1)
@@ -250,7 +316,7 @@ def csa2_sparse_attn(q, kv_pool, seq_base, topk, swa, swa_start, q_pos, sm_scale
     _need(q_pos, torch.int64, "q_pos", 2)
     _need(out, torch.float32, "out", 4)
     _need(lse, torch.float32, "lse", 3)
-    B, Q, H, _ = q.shape
+    _status(dev_status)
     K = topk.shape[-1] if topk is not None else 0
     S_w = swa.shape[1] if swa is not None else 0
     if ws is None:

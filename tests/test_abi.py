@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from sparse_attention_fp4_pack_b200 import build as libbuild
 from sparse_attention_fp4_pack_b200 import csa2
@@ -99,3 +100,99 @@ def test_attn_rejects_bad_args(L):
     assert L.csa2_sparse_attn(*base(64, 512, 4096, 0.04, FAKE, 128)) == 2       # window too large
     assert L.csa2_sparse_attn(*base(64, 512, 128, float("nan"), FAKE, 128)) == 1  # scale
     assert L.csa2_sparse_attn(*base(64, 512, 128, 0.04, None, 128)) == 1        # window data missing
+
+
+def test_binding_checks_shapes_before_the_device():
+    """The binding checks that the buffers agree with the sizes it passes to the C entry
+    points (which cannot see a buffer's extent), before anything reaches the device: right
+    shapes on host tensors fail only at the device check, wrong ones name the argument."""
+    from sparse_attention_fp4_pack_b200 import csa2
+    i32, i64, u8, bf16 = torch.int32, torch.int64, torch.uint8, torch.bfloat16
+    B, Q, HI, K, H, NB = 2, 3, 4, 16, 16, 8
+    q = torch.zeros(B, Q, HI, 128)
+    w = torch.zeros(B, Q, HI)
+    ikp = torch.zeros(10, 68, dtype=u8)
+    base = torch.zeros(B, dtype=i64)
+    nv = torch.zeros(B, Q, dtype=i32)
+    topk = torch.zeros(B, Q, K, dtype=i32)
+    blocks = torch.zeros(B, Q, NB, dtype=i32)
+
+    def full(**kw):
+        a = dict(q=q, w=w, ik_pool=ikp, seq_base=base, n_vis=nv, K=K, max_n_vis=10, topk=topk)
+        a.update(kw)
+        csa2.csa2_index_full(**a)
+
+    def hier(**kw):
+        a = dict(q=q, w=w, ik_pool=ikp, seq_base=base, n_vis=nv, n_blocks=NB, block=8, max_n_vis=10,
+                 blocks=blocks)
+        a.update(kw)
+        csa2.csa2_index_hier(**a)
+
+    def reidx(fn, **kw):
+        a = dict(q=q, w=w, ik_pool=ikp, seq_base=base, n_vis=nv, blocks=blocks, block=8, K=K, topk=topk)
+        a.update(kw)
+        fn(**a)
+
+    with pytest.raises(ValueError, match="CUDA"):
+        full()
+    with pytest.raises(ValueError, match="CUDA"):
+        hier()
+    for fn in (csa2.csa2_reindex, csa2.csa2_reindex_static):
+        with pytest.raises(ValueError, match="CUDA"):
+            reidx(fn)
+    with pytest.raises(ValueError, match="CUDA"):   # extra per-sequence rows are allowed
+        full(seq_base=torch.zeros(B + 3, dtype=i64))
+    bad_full = {"topk": topk[:, :, :-1], "w": torch.zeros(B, Q, HI + 1), "n_vis": torch.zeros(B, Q + 1, dtype=i32),
+                "seq_base": torch.zeros(B - 1, dtype=i64), "q": torch.zeros(B, Q, HI, 64),
+                "topk_score": torch.zeros(B, Q, K - 1), "ik_pool": torch.zeros(10, 72, dtype=u8)}
+    for name, t in bad_full.items():
+        with pytest.raises(ValueError, match=rf"^{name}\b"):
+            full(**{name: t})
+    for name, t in {"blocks": blocks[:, :, :-1], "block_score": torch.zeros(B, Q, NB + 1)}.items():
+        with pytest.raises(ValueError, match=rf"^{name}\b"):
+            hier(**{name: t})
+    for fn in (csa2.csa2_reindex, csa2.csa2_reindex_static):
+        for name, t in {"blocks": torch.zeros(B + 1, Q, NB, dtype=i32), "topk": topk[:1]}.items():
+            with pytest.raises(ValueError, match=rf"^{name}\b"):
+                reidx(fn, **{name: t})
+
+    S = 130
+    aq = torch.zeros(B, Q, H, 512)
+    kvp = torch.zeros(10, 288, dtype=u8)
+    swa = torch.zeros(B, S, 512, dtype=u8)
+    start = torch.zeros(B, dtype=i64)
+    qpos = torch.zeros(B, Q, dtype=i64)
+    out = torch.zeros(B, Q, H, 512)
+    lse = torch.zeros(B, Q, H)
+
+    def attn(**kw):
+        a = dict(q=aq, kv_pool=kvp, seq_base=base, topk=topk, swa=swa, swa_start=start, q_pos=qpos,
+                 sm_scale=0.04, out=out, lse=lse)
+        a.update(kw)
+        csa2.csa2_sparse_attn(**a)
+
+    with pytest.raises(ValueError, match="CUDA"):
+        attn()
+    with pytest.raises(ValueError, match="CUDA"):
+        attn(swa=None, swa_start=None)
+    bad_attn = {"out": torch.zeros(B, Q, H, 256), "lse": torch.zeros(B, Q, H + 1), "q_pos": torch.zeros(B, Q + 1, dtype=i64),
+                "swa": torch.zeros(B - 1, S, 512, dtype=u8), "swa_start": torch.zeros(B - 1, dtype=i64),
+                "topk": torch.zeros(B, Q - 1, K, dtype=i32), "kv_pool": torch.zeros(10, 256, dtype=u8),
+                "q": torch.zeros(B, Q, H, 128)}
+    for name, t in bad_attn.items():
+        with pytest.raises(ValueError, match=rf"^{name}\b"):
+            attn(**{name: t})
+    with pytest.raises(ValueError, match=r"^swa_start\b"):
+        attn(swa_start=None)
+
+    T = 4
+    kv, ik = torch.zeros(T, 512, dtype=bf16), torch.zeros(T, 128, dtype=bf16)
+    pool, ipool = torch.zeros(8, 288, dtype=u8), torch.zeros(8, 68, dtype=u8)
+    with pytest.raises(ValueError, match="CUDA"):
+        csa2.csa2_pack_kv(kv, ik, 2, pool, ipool, dst_entry=torch.zeros(2, dtype=i64))
+    with pytest.raises(ValueError, match=r"^ik\b"):
+        csa2.csa2_pack_kv(kv, torch.zeros(T + 1, 128, dtype=bf16), 1, pool, ipool)
+    with pytest.raises(ValueError, match=r"^ik_pool\b"):
+        csa2.csa2_pack_kv(kv, ik, 1, pool, torch.zeros(7, 68, dtype=u8))
+    with pytest.raises(ValueError, match=r"^dst_entry\b"):
+        csa2.csa2_pack_kv(kv, ik, 2, pool, ipool, dst_entry=torch.zeros(3, dtype=i64))
