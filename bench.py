@@ -49,8 +49,8 @@ WORKLOAD_TEXT = {
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=10)
-    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--workload", default="hier1m", choices=list(WORKLOAD_TEXT))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--cpu-seqs", type=int, default=1, help="sequences in the oracle's timed sample")
