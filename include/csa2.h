@@ -122,7 +122,10 @@ csa2_status csa2_pack_kv(const void* kv, const void* ik, int64_t T, int ratio,
  *
  * score_j = sum_h w_h * max(0, q_h . k_j) over dequantised keys k_j, accumulated in
  * fp32.  The result is a SET (slot order unspecified); equal scores at the cut prefer
- * lower indices.  1 <= K <= 2048, 1 <= HI <= 16.
+ * lower indices while a query sees at most 131,072 entries.  Beyond that (a selection
+ * CTA then holds several 16,384-key chunks) the tie at the cut is still broken the same
+ * way on every run, but not always towards the lower index.  1 <= K <= 2048,
+ * 1 <= HI <= 16.
  * --------------------------------------------------------------------------------- */
 size_t csa2_index_full_workspace_size(int B, int Q, int HI, int K, int64_t max_n_vis);
 csa2_status csa2_index_full(const float* q, const float* w, const uint8_t* ik_pool,
