@@ -74,6 +74,30 @@ MUTANTS = [
     ("output not normalised", "for (int c = 0; c < ORC_D; ++c) oh[c] /= l;", ""),
     ("value is the query", "oh[c] += p * keys[(size_t)i * ORC_D + c];", "oh[c] += p * (double)qh[c];"),
     ("empty slots not skipped", "if (j < 0) continue;\n      orc_dequant_kv", "if (j < -1) continue;\n      orc_dequant_kv"),
+    # second batch
+    ("e4m3 0x7F is a number", "if (e == 15 && m == 7) return NAN;", ""),
+    ("e4m3 ties to the odd code", "(d == best_d && (c & 1u) == 0)", "(d == best_d && (c & 1u) == 1)"),
+    ("bf16 bits shifted by 15", "uint32_t u = (uint32_t)bits << 16;", "uint32_t u = (uint32_t)bits << 15;"),
+    ("ik amax over half the dims", "for (int d = 0; d < ORC_DI; ++d) {\n    float a = fabsf(x[d]);",
+     "for (int d = 0; d < ORC_DI / 2; ++d) {\n    float a = fabsf(x[d]);"),
+    ("ik nibble order swapped", "out[d / 2] |= (uint8_t)(code << ((d & 1) ? 4 : 0));",
+     "out[d / 2] |= (uint8_t)(code << ((d & 1) ? 0 : 4));"),
+    ("kv dequant nibble order", "unsigned code = (e[c / 2] >> ((c & 1) ? 4 : 0)) & 15u;",
+     "unsigned code = (e[c / 2] >> ((c & 1) ? 0 : 4)) & 15u;"),
+    ("ratio-2 mean of the second token twice", "float a = orc_bf16_value(kv[(2 * j) * ORC_D + c]);",
+     "float a = orc_bf16_value(kv[(2 * j + 1) * ORC_D + c]);"),
+    ("top-k drops its last slot", "    if (k < n) {\n      idx_out[k]", "    if (k < n - 1) {\n      idx_out[k]"),
+    ("block score reaches into the next block", "for (int64_t j = c * block; j < (c + 1) * block && j < n; ++j)\n        if (sc[j] > m)",
+     "for (int64_t j = c * block; j <= (c + 1) * block && j < n; ++j)\n        if (sc[j] > m)"),
+    ("reindex skips block 0", "if (c < 0) continue;\n      for (int64_t j", "if (c <= 0) continue;\n      for (int64_t j"),
+    ("window token decoded as e2m1", "keys[(size_t)nk * ORC_D + c] = orc_e4m3_value(row[c]);",
+     "keys[(size_t)nk * ORC_D + c] = orc_e2m1_value(row[c] & 15u);"),
+    ("window misses the current token", "for (int64_t u = lo; u <= t; ++u) {", "for (int64_t u = lo; u < t; ++u) {"),
+    ("softmax without the max shift", "double p = exp(logit[i] - mx);", "double p = exp(logit[i]);"),
+    ("window rows ignore the sequence", "const uint8_t* row = swa + ((size_t)b * S_w + (size_t)r) * ORC_D;",
+     "const uint8_t* row = swa + ((size_t)r) * ORC_D;"),
+    ("entries ignore the sequence base", "orc_dequant_kv(kv_pool + (seq_base[b] + j) * ORC_KV_BYTES",
+     "orc_dequant_kv(kv_pool + (j) * ORC_KV_BYTES"),
 ]
 
 
