@@ -97,6 +97,13 @@ def max_over_ranks(x, world):
 
 
 # ---- clocks during the timed region ---------------------------------------------------------
+def l2_note(cache_bytes, flush_bytes=256 << 20, l2_bytes=126 << 20):
+    """How the timed steps see L2: the cache's size against L2, and the flush between steps."""
+    rel = ">" if cache_bytes > l2_bytes else "<="
+    size = f"{cache_bytes / 1e9:.2f} GB" if cache_bytes >= 1e9 else f"{cache_bytes / 1e6:.1f} MB"
+    return f"cache {size} {rel} L2 ({l2_bytes >> 20} MB) and a {flush_bytes >> 20} MB L2 flush between timed steps"
+
+
 def step_stats(ms_list):
     """Median, 10th and 90th percentile (nearest rank) of per-step device times in ms."""
     if not ms_list:
@@ -379,7 +386,7 @@ def run_ours(args, world, rank, local):
         "config": {"workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}", "B": wl.B, "Q": wl.Q,
                    "H": wl.H, "HI": wl.HI, "K": wl.K, "window": wl.window, "layers": len(sched),
                    "entries_per_seq": max(wl.lengths), "parallelism": f"replicas x{world}",
-                   "l2": "cache 1.5 GB > L2 and a 256 MB L2 flush between timed steps",
+                   "l2": l2_note(x.kv_pool.numel() + x.ik_pool.numel()),
                    "graph": "CUDA graph replay"},
         "e2e": {"value": round(e2e_us, 3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": step.launches_per_step() * args.steps,

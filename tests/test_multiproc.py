@@ -95,3 +95,19 @@ def test_step_stats_nearest_rank():
     st = bench.step_stats([0.25, 0.75, 0.5])
     assert st["median"] == 0.5 and st["p10"] == 0.25 and st["p90"] == 0.75 and st["n"] == 3
     assert isinstance(bench.cpu_model(), (str, type(None)))
+
+
+def test_l2_note_and_algorithmic_units():
+    """The config's L2 note follows the cache size; the roofline's algorithmic figures are the
+    per-unit ones: 212,992 B of keys and 4·H·(K+W)·512 flops per attention query-layer, 68 B
+    per scanned key, 1280 B read + 356 B written per packed token."""
+    import bench
+    import synth
+    assert bench.l2_note(4 * (1 << 20) * 356).startswith("cache 1.49 GB > L2 (126 MB)")
+    assert bench.l2_note(4096 * 356).startswith("cache 1.5 MB <= L2 (126 MB)")
+    wl = synth.workload("hier1m")
+    assert bench.algorithmic(wl, "attn", 1) == (4 * 212_992, 4 * 4 * 64 * 640 * 512)
+    assert bench.algorithmic(wl, "attn", 20) == (20 * 4 * 212_992, 20 * 4 * 4 * 64 * 640 * 512)
+    assert bench.algorithmic(wl, "reindex", 1) == (4 * 16_384 * 68, 2 * 8 * 128 * 4 * 16_384)
+    assert bench.algorithmic(wl, "index_hier", 1)[0] == 4 * (1 << 20) * 68
+    assert bench.algorithmic(wl, "pack", 1) == (4 * 1280 + 4 * 356, 0)
