@@ -111,3 +111,19 @@ def test_l2_note_and_algorithmic_units():
     assert bench.algorithmic(wl, "reindex", 1) == (4 * 16_384 * 68, 2 * 8 * 128 * 4 * 16_384)
     assert bench.algorithmic(wl, "index_hier", 1)[0] == 4 * (1 << 20) * 68
     assert bench.algorithmic(wl, "pack", 1) == (4 * 1280 + 4 * 356, 0)
+
+
+def test_reference_arm_single_process():
+    """bench.py --impl reference at N=1 (no torchrun): the oracle's line with the contract's keys."""
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+           "--steps", "1", "--warmup", "0"]
+    out = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["n_gpus"] == 1 and d["higher_is_better"] is False
+    assert d["cpu_baseline"]["value"] == d["value"] == d["e2e"]["value"] and d["cpu_baseline"]["cores"] >= 1
