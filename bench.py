@@ -59,6 +59,8 @@ def parse_args():
                    help="skip the separate FP4 pack throughput measurement (2^20 tokens)")
     p.add_argument("--no-call-timing", action="store_true",
                    help="time the step without the per-call events (no breakdown or roofline)")
+    p.add_argument("--no-configs", action="store_true",
+                   help="measure only --workload (by default hier1m also brings full128k and verify)")
     return p.parse_args()
 
 
@@ -244,13 +246,17 @@ class ClockSampler:
 
 # ---- roofline bookkeeping -------------------------------------------------------------------
 def load_peaks():
+    """Roofline denominators.  Every call here is timed inside a step of well under a second,
+    so tensor-bound calls take the burst GEMM figure (the sustained one is for seconds-long
+    loops under the power cap)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as f:
             p = json.load(f)
-        return {"hbm": p["hbm_gbs"], "bf16": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+        return {"hbm": p["hbm_gbs"], "bf16": p["bf16_tflops"],
+                "bf16_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
                 "sm_mhz": p.get("sm_max_mhz", 1965.0), "src": "measured"}
-    return {"hbm": 6650.0, "bf16": 1400.0, "sm_mhz": 1965.0, "src": "fallback"}
+    return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "sm_mhz": 1965.0, "src": "fallback"}
 
 
 def algorithmic(wl, name, count):
@@ -262,14 +268,14 @@ def algorithmic(wl, name, count):
         # a query reads each visible 68 B key once; Q queries of a sequence share its keys
         nbytes = sum(int(n_vis[b].max()) for b in range(wl.B)) * 68
         flops = 2 * wl.HI * 128 * int(n_vis.sum())
-        return nbytes, flops
+        return count * nbytes, count * flops
     if name == "reindex":
         return count * BQ * wl.n_blocks * wl.block * 68, count * 2 * wl.HI * 128 * BQ * wl.n_blocks * wl.block
     if name == "attn":
         return count * BQ * (Kent * 288 + W * 512), count * BQ * 4 * H * (Kent + W) * 512
     if name == "pack":
         t = wl.B * wl.new_tokens
-        return t * 1280 + (t // wl.ratio) * 356, 0
+        return count * (t * 1280 + (t // wl.ratio) * 356), 0
     return 0, 0
 
 
@@ -278,22 +284,88 @@ def query_positions(wl):
     return synth.query_positions(wl)
 
 
+# the kernels behind each library call, and what bounds the call
+CALL_KERNELS = {
+    "index_hier": ("stream_scan_kernel<hier> + select_kernel", "hbm"),
+    "index_full": ("stream_scan_kernel<flat> + select_kernel", "hbm"),
+    "reindex": ("reindex_scan_kernel + select_kernel", "hbm"),
+    "attn": ("attn_tc_kernel", "tensor"),
+    "pack": ("pack_kv_kernel", "hbm"),
+}
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the call's
+# dominant kernel, from an ncu capture of that kernel as it is now, per workload; a kernel
+# that changes drops out of this table until it is captured again.
+NCU_DRAM_BYTES_PER_LAUNCH = {("hier1m", "attn"): 1656064}
+
+
+def call_rooflines(wl, per_call, counts, steps, peaks):
+    """Per library call of the step: its device time and its algorithmic HBM bandwidth as a
+    fraction of the measured copy peak; attention also as algorithmic tensor flops against
+    the burst bf16 peak (f16 has the same nominal rate)."""
+    out = {}
+    for name, ms in per_call.items():
+        n = counts[name]
+        step_ms = ms / steps
+        avg_ms = step_ms / n
+        nbytes, flops = algorithmic(wl, name, 1)
+        gbs = nbytes / (avg_ms * 1e-3) / 1e9
+        kernel, bound = CALL_KERNELS[name]
+        d = {"kernel": kernel, "bound": bound, "launches": n, "ms_per_step": round(step_ms, 4),
+             "avg_launch_ms": round(avg_ms, 4), "algorithmic_bytes": nbytes,
+             "hbm_gbs": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm"], 4)}
+        if flops and name != "pack":
+            tf = flops / (avg_ms * 1e-3) / 1e12
+            d.update({"algorithmic_flops": flops, "tflops": round(tf, 2)})
+            if bound == "tensor":
+                d["tensor_frac"] = round(tf / peaks["bf16"], 4)
+        out[name] = d
+    return out
+
+
+def dominant_roofline(wl, calls, peaks):
+    """The roofline object of the call with the largest share of the step."""
+    dom = max(calls, key=lambda k: calls[k]["ms_per_step"])
+    c = calls[dom]
+    if c["bound"] == "hbm":
+        roof = {"bound": "hbm", "achieved": c["hbm_gbs"], "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": c["hbm_frac"]}
+    else:
+        roof = {"bound": "tensor", "achieved": c["tflops"], "peak": peaks["bf16"], "unit": "TFLOP/s",
+                "frac": c["tensor_frac"]}
+    roof["traffic"] = NCU_DRAM_BYTES_PER_LAUNCH.get((wl.name, dom))
+    roof.update({"kernel": c["kernel"], "call": dom, "avg_launch_ms": c["avg_launch_ms"],
+                 "algorithmic_bytes": c["algorithmic_bytes"], "algorithmic_flops": c.get("algorithmic_flops"),
+                 "peak_src": peaks["src"] + (" (bf16 burst; f16 has the same nominal rate)"
+                                             if c["bound"] == "tensor" else " (copy bandwidth)")})
+    return roof
+
+
+# arithmetic of the path: int8 x int8 -> int32 indexer dots (tcgen05 kind::i8) and
+# f16 x f16 -> fp32 attention (tcgen05 kind::f16), fp32 epilogues; FP4/FP8 storage
+DTYPE = "f16+i8"
+
+
 # ---- our implementation ---------------------------------------------------------------------
-def run_ours(args, world, rank, local):
+def measure(name, steps, warmup, world, dev, call_timing=True, e2e=True):
+    """One workload's decode step: device time of a CUDA-graph replay (inputs resident, L2
+    flushed between steps), the per-call breakdown from a second graph with timing events,
+    and the end-to-end time through the public API with host buffers."""
     import synth
-    from sparse_attention_fp4_pack_b200 import csa2
     from sparse_attention_fp4_pack_b200.decode import CallTimer, DecodeStep
     from sparse_attention_fp4_pack_b200.workload import build_state
 
-    csa2.lib()
-    dev = torch.device("cuda", torch.cuda.current_device())
-    wl = synth.workload(args.workload)
+    wl = synth.workload(name)
     sched = synth.layer_schedule(wl)
     qd = synth.step_queries(wl)
     x = build_state(wl, lambda b: synth.seq_tokens(wl, b, device=dev), qd, device=dev)
-    step = DecodeStep(B=wl.B, Q=wl.Q, H=wl.H, HI=wl.HI, K=wl.K, window=wl.window, ratio=wl.ratio,
-                      schedule=sched, hier=wl.hier, max_n_vis=max(wl.lengths), n_blocks=wl.n_blocks,
-                      block=wl.block, device=dev)
+
+    def new_step():
+        return DecodeStep(B=wl.B, Q=wl.Q, H=wl.H, HI=wl.HI, K=wl.K, window=wl.window, ratio=wl.ratio,
+                          schedule=sched, hier=wl.hier, max_n_vis=max(wl.lengths), n_blocks=wl.n_blocks,
+                          block=wl.block, device=dev)
+
+    step = new_step()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # 256 MB > 126 MB L2
 
     def one(graph_step):
@@ -306,19 +378,16 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         return e0.elapsed_time(e1), (graph_step.timer.collect() if graph_step.timer else {})
 
-    # Per-call breakdown and the roofline come from a separate graph that brackets every
-    # library call with timing events (each event node adds about 2 us, so the headline
-    # step is timed from a graph without them).
+    # Per-call breakdown from a separate graph that brackets every library call with timing
+    # events (each event node adds about 2 us, so the headline step is timed without them).
     per_call, counts = {}, {}
-    if not args.no_call_timing:
-        probe = DecodeStep(B=wl.B, Q=wl.Q, H=wl.H, HI=wl.HI, K=wl.K, window=wl.window, ratio=wl.ratio,
-                           schedule=sched, hier=wl.hier, max_n_vis=max(wl.lengths), n_blocks=wl.n_blocks,
-                           block=wl.block, device=dev)
+    if call_timing:
+        probe = new_step()
         probe.timer = CallTimer()
         probe.capture(x)
-        for i in range(args.warmup + args.steps):
+        for i in range(warmup + steps):
             _, calls = one(probe)
-            if i >= args.warmup:
+            if i >= warmup:
                 for k, v in calls.items():
                     per_call[k] = per_call.get(k, 0.0) + v
         counts = probe.timer.counts()
@@ -327,7 +396,7 @@ def run_ours(args, world, rank, local):
     step.capture(x)
 
     clocks = ClockSampler(dev)  # its poller starts now and is running by the timed steps
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         one(step)
     step.check_status()
     barrier(world)
@@ -335,7 +404,7 @@ def run_ours(args, world, rank, local):
     clocks.start()
     total_ms = 0.0
     step_ms = []
-    for _ in range(args.steps):
+    for _ in range(steps):
         ms, _ = one(step)
         total_ms += ms
         step_ms.append(ms)
@@ -344,100 +413,87 @@ def run_ours(args, world, rank, local):
     clk = clocks.stop()
     step.check_status()
     t_max = max_over_ranks(total_ms, world)
-
-    # ---- end to end through the public API: pinned host inputs in, results out ----------
-    h_in = {k: getattr(x, k).cpu().pin_memory() for k in ("new_kv", "new_ik", "q", "qi", "w", "swa")}
-    h_out = {"out": torch.empty_like(step.out, device="cpu").pin_memory(),
-             "lse": torch.empty_like(step.lse, device="cpu").pin_memory(),
-             "topk": torch.empty_like(step.topk, device="cpu").pin_memory()}
-    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
-    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
-    # the step as a user runs it with host data: DecodeStep.run_io captured in a graph, which
-    # overlaps each layer's input copies and output read-back with the other layers' work
-    step.capture_io(x, h_in, h_out)
-    e2e_ms = 0.0
-    for i in range(args.warmup + args.steps):
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
-        step.replay_io()
-        e1.record()
-        torch.cuda.synchronize()
-        if i >= args.warmup:
-            e2e_ms += e0.elapsed_time(e1)
-        flush.fill_(1)
-    step.check_status()
-    e2e_max = max_over_ranks(e2e_ms, world)
-
     tokens = wl.B * wl.Q * world
-    us_per_token = t_max * 1000.0 / (args.steps * tokens)
-    e2e_us = e2e_max * 1000.0 / (args.steps * tokens)
+    res = {"wl": wl, "sched": sched, "us_per_token": t_max * 1000.0 / (steps * tokens),
+           "ms_per_step": t_max / steps, "stats": step_stats(step_ms), "clocks": clk,
+           "launches": step.launches_per_step() * steps, "per_call": per_call, "counts": counts,
+           "cache_bytes": x.kv_pool.numel() + x.ik_pool.numel()}
 
-    # roofline of the dominant call (from the calibration graph)
-    roof = roofline(wl, per_call, counts, args.steps) if per_call else None
+    if e2e:
+        # the step as a user runs it with host data: DecodeStep.run_io captured in a graph,
+        # which overlaps each layer's input copies and output read-back with the other
+        # layers' work; pinned host inputs in, results out, every step
+        h_in = {k: getattr(x, k).cpu().pin_memory() for k in ("new_kv", "new_ik", "q", "qi", "w", "swa")}
+        h_out = {"out": torch.empty_like(step.out, device="cpu").pin_memory(),
+                 "lse": torch.empty_like(step.lse, device="cpu").pin_memory(),
+                 "topk": torch.empty_like(step.topk, device="cpu").pin_memory()}
+        h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+        d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+        step.capture_io(x, h_in, h_out)
+        e2e_ms = 0.0
+        for i in range(warmup + steps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            step.replay_io()
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= warmup:
+                e2e_ms += e0.elapsed_time(e1)
+            flush.fill_(1)
+        step.check_status()
+        e2e_max = max_over_ranks(e2e_ms, world)
+        res["e2e"] = {"value": round(e2e_max * 1000.0 / (steps * tokens), 3), "unit": UNIT,
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del step, x, flush
+    torch.cuda.empty_cache()
+    return res
 
-    breakdown = {k: round(v / args.steps, 4) for k, v in per_call.items()}
+
+def config_of(name, wl, sched, world, cache_bytes):
+    return {"workload": f"{name}: {WORKLOAD_TEXT[name]}", "B": wl.B, "Q": wl.Q, "H": wl.H, "HI": wl.HI,
+            "K": wl.K, "window": wl.window, "layers": len(sched), "entries_per_seq": max(wl.lengths),
+            "parallelism": f"replicas x{world}", "l2": l2_note(cache_bytes), "graph": "CUDA graph replay"}
+
+
+def run_ours(args, world, rank, local):
+    from sparse_attention_fp4_pack_b200 import csa2
+
+    csa2.lib()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks = load_peaks()
+    r = measure(args.workload, args.steps, args.warmup, world, dev, call_timing=not args.no_call_timing)
+    wl = r["wl"]
+    calls = call_rooflines(wl, r["per_call"], r["counts"], args.steps, peaks) if r["per_call"] else {}
     line = {
-        "metric": METRIC, "value": round(us_per_token, 3), "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 4),
-        "ms_per_step_rank0": step_stats(step_ms),
+        "metric": METRIC, "value": round(r["us_per_token"], 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["ms_per_step"], 4),
+        "ms_per_step_rank0": r["stats"],
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": DTYPE,
         "data": "synthetic (seeded)",
-        "config": {"workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}", "B": wl.B, "Q": wl.Q,
-                   "H": wl.H, "HI": wl.HI, "K": wl.K, "window": wl.window, "layers": len(sched),
-                   "entries_per_seq": max(wl.lengths), "parallelism": f"replicas x{world}",
-                   "l2": l2_note(x.kv_pool.numel() + x.ik_pool.numel()),
-                   "graph": "CUDA graph replay"},
-        "e2e": {"value": round(e2e_us, 3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": step.launches_per_step() * args.steps,
-        "roofline": roof,
-        "ms_per_call": breakdown,
-        "clocks": clk,
+        "config": config_of(args.workload, wl, r["sched"], world, r["cache_bytes"]),
+        "e2e": r["e2e"],
+        "gpu_launches": r["launches"],
+        "roofline": dominant_roofline(wl, calls, peaks) if calls else None,
+        "calls": calls,
+        "clocks": r["clocks"],
+        "peaks": peaks,
     }
-    return line, wl, x
-
-
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the call's
-# dominant kernel, from an ncu capture of that kernel as it is now, per workload; a kernel
-# that changes drops out of this table until it is captured again.
-NCU_DRAM_BYTES_PER_LAUNCH = {("hier1m", "attn"): 1656064}
-
-
-def roofline(wl, per_call, counts, steps):
-    peaks = load_peaks()
-    dom = max(per_call, key=lambda k: per_call[k])
-    avg_ms = per_call[dom] / steps / counts[dom]
-    nbytes, flops = algorithmic(wl, dom, 1)
-    kernel_info = dominant_kernel_info(dom)
-    if kernel_info["bound"] == "hbm":
-        achieved = nbytes / (avg_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm"], 4), "traffic": None}
-    else:
-        achieved = flops / (avg_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16"], "unit": "TFLOP/s",
-                "frac": round(achieved / peaks["bf16"], 4), "traffic": None}
-    roof["traffic"] = NCU_DRAM_BYTES_PER_LAUNCH.get((wl.name, dom))
-    roof.update({"kernel": kernel_info["kernel"], "call": dom, "avg_launch_ms": round(avg_ms, 4),
-                 "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
-                 "peak_src": peaks["src"] + (" (bf16 sustained; f16 has the same nominal rate)"
-                                             if kernel_info["bound"] == "tensor" else "")})
-    return roof
-
-
-def dominant_kernel_info(call):
-    return {
-        "index_hier": {"kernel": "stream_scan_kernel<hier> + select_kernel", "bound": "hbm"},
-        "index_full": {"kernel": "stream_scan_kernel<flat> + select_kernel", "bound": "hbm"},
-        "reindex": {"kernel": "reindex_scan_kernel + select_kernel", "bound": "hbm"},
-        "attn": {"kernel": "attn_tc_kernel", "bound": "tensor"},
-        "pack": {"kernel": "pack_kv_kernel", "bound": "hbm"},
-    }[call]
-
-
-# arithmetic of the path: int8 x int8 -> int32 indexer dots (tcgen05 kind::i8) and
-# f16 x f16 -> fp32 attention (tcgen05 kind::f16), fp32 epilogues; FP4/FP8 storage
-DTYPE = "f16+i8"
+    # the metric's other decode configurations, each measured the same way
+    configs = {}
+    if not args.no_configs and args.workload == "hier1m":
+        for name in ("full128k", "verify"):
+            c = measure(name, args.steps, args.warmup, world, dev, call_timing=not args.no_call_timing)
+            cc = call_rooflines(c["wl"], c["per_call"], c["counts"], args.steps, peaks) if c["per_call"] else {}
+            configs[name] = {"value": round(c["us_per_token"], 3), "unit": UNIT,
+                             "ms_per_step": round(c["ms_per_step"], 4), "ms_per_step_rank0": c["stats"],
+                             "config": config_of(name, c["wl"], c["sched"], world, c["cache_bytes"]),
+                             "e2e": c["e2e"], "gpu_launches": c["launches"], "calls": cc,
+                             "roofline": dominant_roofline(c["wl"], cc, peaks) if cc else None,
+                             "clocks": c["clocks"]}
+    if configs:
+        line["configs"] = configs
+    return line, wl
 
 
 # ---- the oracle, timed on the host cores ------------------------------------------------------
@@ -540,10 +596,18 @@ def time_oracle(wl, nseq, steps, warmup, device):
         oracle_step(wl, st)
     dt = time.perf_counter() - t0
     tokens = nseq * wl.Q
-    cores = min(oracle.num_threads(), nseq * wl.Q)
+    # the oracle spreads queries over its threads, or the work inside a query when there
+    # are fewer queries than threads, so every thread takes part either way
+    cores = oracle.num_threads()
     sample = (f"{nseq} of {wl.B} sequences of the {wl.name} workload (full context, all "
-              f"{wl.n_layers} layers), {steps} step(s)")
+              f"{wl.n_layers} layers, {wl.Q} quer{'y' if wl.Q == 1 else 'ies'} each), {steps} step(s)")
     return dt * 1e6 / (steps * tokens), cores, sample
+
+
+def cpu_baseline(wl, nseq):
+    v, cores, sample = time_oracle(wl, nseq, 1, 0, "cuda")
+    return {"value": round(v, 1), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+            "cpu_model": cpu_model()}
 
 
 def main():
@@ -566,18 +630,17 @@ def main():
         if world > 1:
             torch.distributed.destroy_process_group()
         return
-    line, wl, x = run_ours(args, world, rank, local)
-    del x
-    torch.cuda.empty_cache()
+    line, wl = run_ours(args, world, rank, local)
     if not args.no_pack_throughput:
         pk = time_pack(5, 3, "cuda")
         peak = load_peaks()["hbm"]
         line["pack_throughput"] = {"tokens": 1 << 20, "unit": "GB/s", "peak": peak,
                                    **{k: dict(v, frac=round(v["GB/s"] / peak, 3)) for k, v in pk.items()}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, sample = time_oracle(wl, args.cpu_seqs, 1, 0, "cuda")
-        line["cpu_baseline"] = {"value": round(v, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": sample, "cpu_model": cpu_model()}
+        import synth
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seqs)
+        for name, c in line.get("configs", {}).items():
+            c["cpu_baseline"] = cpu_baseline(synth.workload(name), 1)
     if rank == 0:
         print(json.dumps(line, ensure_ascii=False), flush=True)
     if world > 1:

@@ -14,7 +14,7 @@
  *    after returning, holds no global mutable state and never synchronises: each call
  *    validates its host-visible arguments, enqueues its kernels on `stream` and returns.
  *    The one exception is csa2_reindex_static (end of this file), which uses a device
- *    array compiled into the library and caches its address per device.
+ *    array compiled into the library and caches its address per device context.
  *  - On CSA2_ERR_INVALID_ARG or CSA2_ERR_UNSUPPORTED nothing has been launched.
  *    CSA2_ERR_CUDA reports a launch failure (cudaGetLastError after the launch).
  *  - Values that live on the device (sequence bases, visible counts, Top-K indices,
@@ -120,12 +120,13 @@ csa2_status csa2_pack_kv(const void* kv, const void* ik, int64_t T, int ratio,
  *   topk int32 [B][Q][K]  out: the K best visible entries (indices relative to
  *        seq_base), -1 in unused slots; topk_score fp32 [B][Q][K] (may be NULL)
  *
- * score_j = sum_h w_h * max(0, q_h . k_j) over dequantised keys k_j, accumulated in
- * fp32.  The result is a SET (slot order unspecified); equal scores at the cut prefer
- * lower indices while a query sees at most 131,072 entries.  Beyond that (a selection
- * CTA then holds several 16,384-key chunks) the tie at the cut is still broken the same
- * way on every run, but not always towards the lower index.  1 <= K <= 2048,
- * 1 <= HI <= 16.
+ * score_j = sum_h w_h * max(0, q_h . k_j) over dequantised keys k_j.  Arithmetic: each
+ * query head is scaled by a power of two and split into four int8 limbs (representing
+ * it to 2^-21 of its largest element); the dot products of the limbs with the key's E2M1
+ * codes are exact int32 sums on the tensor cores; fp32 is used only to combine the four
+ * limbs, apply the ReLU, the head weights and the key's scale.  The result is a SET
+ * (slot order unspecified); equal scores at the cut prefer lower indices.
+ * 1 <= K <= 2048, 1 <= HI <= 16.
  * --------------------------------------------------------------------------------- */
 size_t csa2_index_full_workspace_size(int B, int Q, int HI, int K, int64_t max_n_vis);
 csa2_status csa2_index_full(const float* q, const float* w, const uint8_t* ik_pool,
@@ -214,8 +215,10 @@ csa2_status csa2_sparse_attn(const float* q, const uint8_t* kv_pool, int64_t poo
  *    CSA2_STATIC_SCRATCH_BYTES the call returns CSA2_ERR_UNSUPPORTED before touching
  *    the device (n_blocks * block = 16,384 candidates fit 64 queries).
  *  - Set-up: the first call on a device, with that device current, looks up the array's
- *    device address (cudaGetSymbolAddress) and caches it; CSA2_ERR_CUDA if that fails.
- *    Make the first call on each device before any stream capture.
+ *    device address (cudaGetSymbolAddress) and caches it for that device context;
+ *    CSA2_ERR_CUDA if that fails.  A reset device (cudaDeviceReset) has a new context,
+ *    so the first call after it looks the address up again.  Make the first call on
+ *    each device, and the first after a reset, before any stream capture.
  *  - Nothing in the array needs to start at zero: the scan writes every key the
  *    selection reads back within the same call.
  *  - One array per device: calls whose kernels overlap on the same device (several

@@ -4,7 +4,7 @@ TEST INFRASTRUCTURE ONLY.  This package is loaded by ``tests/``, by
 ``__graft_entry__.smoke()`` and by the CPU-baseline leg of ``bench.py``; the product path
 (the CUDA library and its binding) never imports it, and it never imports them.
 
-The arithmetic lives in ``csa2_oracle.c`` (plain C, doubles, OpenMP over queries); this
+The arithmetic lives in ``csa2_oracle.c`` (plain C, doubles, OpenMP over queries, or inside a query when there are fewer queries than threads); this
 module only marshals numpy arrays through ctypes.  Every function cites the page passage
 it follows in the C source.
 """

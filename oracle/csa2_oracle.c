@@ -42,6 +42,20 @@ int orc_num_threads(void) {
 #endif
 }
 
+/* Threads.  Queries, entries and heads are independent, so every result is the same
+ * whatever the thread count.  A call with at least as many queries as threads spreads
+ * its queries over the threads; a call with fewer spreads the work inside each query
+ * instead (the entries of a scan, the candidates of a Reindex, the heads of an attention
+ * call), so a one-query sample still uses every core. */
+static int orc_queries_parallel(int64_t n_queries) { return n_queries >= orc_num_threads(); }
+static int orc_in_parallel(void) {
+#ifdef _OPENMP
+  return omp_in_parallel();
+#else
+  return 1;
+#endif
+}
+
 /* ------------------------------------------------------------------------------------
  * Element formats (P2 §KV 캐시 네 가지: "E2M1 family, shared scale";
  * P3 §4비트로 적어도 되는 이유: NVFP4 without the second-level global scale, one 8-bit
@@ -236,6 +250,7 @@ static double score_one(const float* q, const float* w, int HI, const uint8_t* e
 
 void orc_index_scores(const float* q, const float* w, int HI, const uint8_t* ik_seq, int64_t n,
                       double* scores) {
+#pragma omp parallel for schedule(static) if (!orc_in_parallel())
   for (int64_t j = 0; j < n; ++j) scores[j] = score_one(q, w, HI, ik_seq + j * ORC_IK_BYTES);
 }
 
@@ -284,7 +299,7 @@ void orc_topk(const double* scores, int64_t n, int K, int32_t* idx_out, double* 
 void orc_index_full(const float* q, const float* w, const uint8_t* ik_pool, const int64_t* seq_base,
                     const int32_t* n_vis, int B, int Q, int HI, int K, int32_t* topk,
                     double* topk_score) {
-#pragma omp parallel for schedule(dynamic, 1)
+#pragma omp parallel for schedule(dynamic, 1) if (orc_queries_parallel((int64_t)B * Q))
   for (int64_t bq = 0; bq < (int64_t)B * Q; ++bq) {
     int64_t b = bq / Q;
     int64_t n = n_vis[bq];
@@ -303,7 +318,7 @@ void orc_index_full(const float* q, const float* w, const uint8_t* ik_pool, cons
 void orc_index_hier(const float* q, const float* w, const uint8_t* ik_pool, const int64_t* seq_base,
                     const int32_t* n_vis, int B, int Q, int HI, int n_blocks, int block,
                     int32_t* blocks, double* block_score) {
-#pragma omp parallel for schedule(dynamic, 1)
+#pragma omp parallel for schedule(dynamic, 1) if (orc_queries_parallel((int64_t)B * Q))
   for (int64_t bq = 0; bq < (int64_t)B * Q; ++bq) {
     int64_t b = bq / Q;
     int64_t n = n_vis[bq];
@@ -331,7 +346,7 @@ void orc_index_hier(const float* q, const float* w, const uint8_t* ik_pool, cons
 void orc_reindex(const float* q, const float* w, const uint8_t* ik_pool, const int64_t* seq_base,
                  const int32_t* n_vis, const int32_t* blocks, int n_blocks, int block, int B, int Q,
                  int HI, int K, int32_t* topk, double* topk_score) {
-#pragma omp parallel for schedule(dynamic, 1)
+#pragma omp parallel for schedule(dynamic, 1) if (orc_queries_parallel((int64_t)B * Q))
   for (int64_t bq = 0; bq < (int64_t)B * Q; ++bq) {
     int64_t b = bq / Q;
     int64_t n = n_vis[bq];
@@ -344,11 +359,13 @@ void orc_reindex(const float* q, const float* w, const uint8_t* ik_pool, const i
       int64_t c = blocks[bq * n_blocks + s];
       if (c < 0) continue;
       for (int64_t j = c * block; j < (c + 1) * block && j < n; ++j) {
-        sc[m] = score_one(q + bq * HI * ORC_DI, w + bq * HI, HI, seq + j * ORC_IK_BYTES);
         lab[m] = j;
         ++m;
       }
     }
+#pragma omp parallel for schedule(static) if (!orc_in_parallel())
+    for (int64_t i = 0; i < m; ++i)
+      sc[i] = score_one(q + bq * HI * ORC_DI, w + bq * HI, HI, seq + lab[i] * ORC_IK_BYTES);
     topk_labeled(sc, lab, m, K, topk + bq * K, topk_score ? topk_score + bq * K : NULL);
     free(sc);
     free(lab);
@@ -372,7 +389,7 @@ void orc_sparse_attn(const float* q /*[B][Q][H][512]*/, const uint8_t* kv_pool, 
                      int S_w, const int64_t* swa_start /*[B]*/, const int64_t* q_pos /*[B][Q]*/,
                      int window, int B, int Q, int H, double sm_scale, double* out /*[B][Q][H][512]*/,
                      double* lse /*[B][Q][H]*/) {
-#pragma omp parallel for schedule(dynamic, 1)
+#pragma omp parallel for schedule(dynamic, 1) if (orc_queries_parallel((int64_t)B * Q))
   for (int64_t bq = 0; bq < (int64_t)B * Q; ++bq) {
     int64_t b = bq / Q;
     int64_t t = q_pos[bq];
@@ -396,13 +413,15 @@ void orc_sparse_attn(const float* q /*[B][Q][H][512]*/, const uint8_t* kv_pool, 
         ++nk;
       }
     }
-    double* logit = (double*)malloc(sizeof(double) * (size_t)(nk > 0 ? nk : 1));
+#pragma omp parallel for schedule(dynamic, 1) if (!orc_in_parallel())
     for (int h = 0; h < H; ++h) {
+      double* logit = (double*)malloc(sizeof(double) * (size_t)(nk > 0 ? nk : 1));
       const float* qh = q + (bq * H + h) * ORC_D;
       double* oh = out + (bq * H + h) * ORC_D;
       if (nk == 0) {
         for (int c = 0; c < ORC_D; ++c) oh[c] = 0.0;
         lse[bq * H + h] = -HUGE_VAL;
+        free(logit);
         continue;
       }
       double mx = -HUGE_VAL;
@@ -421,8 +440,8 @@ void orc_sparse_attn(const float* q /*[B][Q][H][512]*/, const uint8_t* kv_pool, 
       }
       for (int c = 0; c < ORC_D; ++c) oh[c] /= l;
       lse[bq * H + h] = mx + log(l);
+      free(logit);
     }
-    free(logit);
     free(keys);
   }
 }

@@ -1005,9 +1005,30 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
   const uint32_t e_take = need > cta_eq ? min(E, need - cta_eq) : 0u;
   int32_t* s_idx = reinterpret_cast<int32_t*>(sub);  // [G + e_take <= K]
   float* s_sc = reinterpret_cast<float*>(sub + CSA2_MAX_K);
-  uint32_t lg = (uint32_t)mine, le = (uint32_t)(mine >> 32);
+  // With one chunk, thread order is index order and the counting pass's prefix places
+  // every item.  With several, a thread's items are not contiguous in index order across
+  // chunks, so each chunk gets its own block-wide prefix on top of the counts of the
+  // chunks before it: the staged order is then index order throughout.
+  uint32_t base_g = 0u, base_e = 0u;
   for (int ch = 0; ch < nchunks; ++ch) {
-    if (nchunks > 1) load_chunk(ch, false);
+    uint32_t lg = (uint32_t)mine, le = (uint32_t)(mine >> 32);
+    if (nchunks > 1) {
+      load_chunk(ch, false);
+      uint32_t cg = 0u, ce = 0u;
+#pragma unroll 4
+      for (int e = 0; e < kPer; ++e) {
+        bool gt, eq;
+        classify(mk[e], gt, eq);
+        cg += gt;
+        ce += eq;
+      }
+      uint64_t ctot;
+      const uint64_t cm = block_excl_scan64((uint64_t)cg | ((uint64_t)ce << 32), scan_ws, &ctot);
+      lg = base_g + (uint32_t)cm;
+      le = base_e + (uint32_t)(cm >> 32);
+      base_g += (uint32_t)ctot;
+      base_e += (uint32_t)(ctot >> 32);
+    }
     const int64_t i0 = lo + (int64_t)ch * kSelChunk + (int64_t)tid * kPer;
 #pragma unroll 2
     for (int e = 0; e < kPer; ++e) {

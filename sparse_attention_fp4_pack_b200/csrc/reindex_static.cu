@@ -9,20 +9,23 @@
 //
 // How: g_reindex_scratch below is a file-scope __device__ array of
 // CSA2_STATIC_SCRATCH_BYTES.  Every GPU on which the library's device code is loaded
-// holds that array until the process exits.  The first call on a device, with that
-// device current, looks up the array's device address with cudaGetSymbolAddress (the
-// host-side symbol is not a device address) and caches it per device; later calls
-// reuse it.  This set-up runs inside the first call, so the first call on each device
-// should come before any stream capture.  The call then runs csa2_reindex unchanged
-// with the array as its workspace.  Nothing here allocates: no cudaMalloc, no
-// cudaFree, no allocating library routine.
+// holds that array until the process exits.  In host code the array's name is only a
+// host-side stand-in, so the call looks up its device address with cudaGetSymbolAddress,
+// with the device current, the first time it runs in a device context, and caches it
+// keyed by the device and the context's unique id.  A context that is destroyed and
+// created again (cudaDeviceReset) gets a new id, so the next call looks the address up
+// again instead of reusing a stale one.  This set-up runs inside the call, so the first
+// call on each device (and the first after a reset) should come before any stream
+// capture.  The call then runs csa2_reindex unchanged with the array as its workspace.
+// Nothing here allocates: no cudaMalloc, no cudaFree, no allocating library routine.
 //
 // The scratch holds the per-candidate keys that the Reindex scan writes and the Top-K
 // selection reads back; the scan writes every key the selection reads, so nothing in
 // the array has to start at zero.  There is one array per device: two calls whose
 // kernels overlap on the same device (two streams, or two host threads) race on it
 // and their results are undefined.  Serialise the calls (one stream) on each device.
-#include <atomic>
+#include <cuda.h>
+
 #include <mutex>
 
 #include "csa2_device.cuh"
@@ -32,27 +35,64 @@ namespace {
 static __device__ __align__(256) uint8_t g_reindex_scratch[CSA2_STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-std::atomic<void*> g_scratch_addr[kMaxDevices];  // device address of the array, per device
-std::mutex g_scratch_setup;
+struct ScratchSlot {
+  unsigned long long ctx_id;  // unique id of the context the address belongs to (0: none)
+  void* addr;                 // device address of the array in that context
+};
+ScratchSlot g_scratch[kMaxDevices];
+std::mutex g_scratch_mu;
 
-// Device address of the array on the current device (looked up once per device).
+// Driver entry points for the current context's unique id, fetched through the runtime
+// (so the library needs no link against the driver library).  Null when unavailable.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+std::once_flag g_driver_once;
+
+void load_driver_entry_points() {
+  void* f = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+  f = nullptr;
+  if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(f);
+  cudaGetLastError();
+}
+
+// Unique id of the current context, or 0 if there is none yet or the driver cannot say.
+unsigned long long current_ctx_id() {
+  std::call_once(g_driver_once, load_driver_entry_points);
+  if (!g_ctx_get_current || !g_ctx_get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  if (g_ctx_get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of the array in the current device's current context.
 csa2_status scratch_on_current_device(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return CSA2_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return CSA2_ERR_UNSUPPORTED;
-  void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
-  if (!p) {
-    std::lock_guard<std::mutex> lock(g_scratch_setup);
-    p = g_scratch_addr[dev].load(std::memory_order_relaxed);
-    if (!p) {
-      if (cudaGetSymbolAddress(&p, g_reindex_scratch) != cudaSuccess || !p) {
-        cudaGetLastError();  // clear the error so a later launch check does not report it
-        return CSA2_ERR_CUDA;
-      }
-      g_scratch_addr[dev].store(p, std::memory_order_release);
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  const unsigned long long id = current_ctx_id();
+  ScratchSlot& slot = g_scratch[dev];
+  if (id == 0 || slot.ctx_id != id || !slot.addr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_reindex_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();  // clear the error so a later launch check does not report it
+      return CSA2_ERR_CUDA;
     }
+    // the lookup makes the context current if the runtime had not yet; take its id now
+    slot.ctx_id = id != 0 ? id : current_ctx_id();
+    slot.addr = p;
   }
-  *out = p;
+  *out = slot.addr;
   return CSA2_OK;
 }
 

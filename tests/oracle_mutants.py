@@ -64,8 +64,8 @@ MUTANTS = [
      "ik_pool, n,\n                     sc);\n    topk_labeled(sc, NULL, n, K"),
     ("block score is the first entry", "if (sc[j] > m) m = sc[j];", "if (m == -HUGE_VAL) m = sc[j];"),
     ("block count drops the ragged block", "int64_t nb = (n + block - 1) / block;", "int64_t nb = n / block;"),
-    ("reindex ignores visibility", "for (int64_t j = c * block; j < (c + 1) * block && j < n; ++j) {\n        sc[m]",
-     "for (int64_t j = c * block; j < (c + 1) * block; ++j) {\n        sc[m]"),
+    ("reindex ignores visibility", "for (int64_t j = c * block; j < (c + 1) * block && j < n; ++j) {\n        lab[m]",
+     "for (int64_t j = c * block; j < (c + 1) * block; ++j) {\n        lab[m]"),
     # attention
     ("window one token too long", "int64_t lo = t - window + 1;", "int64_t lo = t - window;"),
     ("window ignores its buffer start", "int64_t r = u - swa_start[b];", "int64_t r = u;"),

@@ -291,3 +291,59 @@ def test_hier1m_sampled(orc):
         assert_topk_set(topk.cpu().numpy()[2, 0], o_topk, sl[cand], 512, labels=cand, what=f"layer {l}")
     torch.cuda.synchronize()
     assert int(st.item()) == 0
+
+
+# ---- selections longer than 131,072 keys: several 16,384-key chunks per selection CTA -----
+def test_flat_1m_sampled(orc):
+    """Flat Top-512 over 2^20 (+ a ragged tail) visible keys: 8 selection CTAs of 9 chunks
+    each.  Sets equal the oracle's within the tie band."""
+    T = (1 << 20) + 3001
+    kv, ik = synth.kv_tokens(90, T, device="cuda", recipe="clipped")
+    kvp = torch.empty(T, 288, dtype=torch.uint8, device="cuda")
+    ikp = torch.zeros(T, 68, dtype=torch.uint8, device="cuda")
+    csa2.csa2_pack_kv(kv, ik, 1, kvp, ikp)
+    del kvp, kv
+    # the oracle packs both pools; its indexer pool does not depend on the main-KV tokens
+    _, o_ik = orc.pack_kv(np.zeros((T, 512), np.uint16), bf16_bits(ik), 1)
+    del ik
+    assert np.array_equal(np_u8(ikp), o_ik)
+    HI, K = 8, 512
+    n_vis = np.array([[T, (1 << 20) - 777, 300000]], np.int32)
+    q, w = synth.index_queries(91, 1, 3, HI)
+    topk, _, st = run_full(q.cuda(), w.cuda(), ikp, torch.zeros(1, dtype=torch.int64, device="cuda"),
+                           torch.from_numpy(n_vis).cuda(), K, T)
+    assert st == 0
+    for i in range(3):
+        n = int(n_vis[0, i])
+        s = orc.index_scores(q[0, i].numpy(), w[0, i].numpy(), o_ik[:n])
+        o_topk, _ = orc.topk(s, K)
+        assert_topk_set(topk[0, i], o_topk, s, K, what=f"query {i} n{n}")
+
+
+def test_flat_1m_ties_prefer_lower_index(orc):
+    """Ties at the cut across chunks: with 2 heads q = (+1..., -1...) and w = (1, -1), keys
+    of all +1 score 128, keys of all -1 score -128 and zero keys score 0.  Entries
+    [0, 150000) are -1, 100 entries from 900000 are +1 and the rest are 0, so the Top-300 is
+    the 100 positive keys and the 200 lowest-index zero keys, 150000..150199, which sit in a
+    later chunk of their selection CTA than some other zero keys of the same threads."""
+    T = (1 << 20) + 17
+    kv = torch.zeros(T, 512, dtype=torch.bfloat16, device="cuda")
+    ik = torch.zeros(T, 128, dtype=torch.bfloat16, device="cuda")
+    ik[:150000] = -1.0
+    ik[900000:900100] = 1.0
+    kvp = torch.empty(T, 288, dtype=torch.uint8, device="cuda")
+    ikp = torch.zeros(T, 68, dtype=torch.uint8, device="cuda")
+    csa2.csa2_pack_kv(kv, ik, 1, kvp, ikp)
+    del kvp, kv
+    q = torch.stack([torch.ones(128), -torch.ones(128)]).reshape(1, 1, 2, 128)
+    w = torch.tensor([1.0, -1.0]).reshape(1, 1, 2)
+    topk, _, st = run_full(q.cuda(), w.cuda(), ikp, torch.zeros(1, dtype=torch.int64, device="cuda"),
+                           torch.tensor([[T]], dtype=torch.int32, device="cuda"), 300, T)
+    assert st == 0
+    want = list(range(150000, 150200)) + list(range(900000, 900100))
+    assert sorted(topk[0, 0].tolist()) == want
+    # the oracle, from its own pack of the same tokens, agrees
+    _, o_ik = orc.pack_kv(np.zeros((T, 512), np.uint16), bf16_bits(ik), 1)
+    assert np.array_equal(np_u8(ikp), o_ik)
+    o_topk, _ = orc.index_full(q.numpy(), w.numpy(), o_ik, np.zeros(1, np.int64), np.array([[T]], np.int32), 300)
+    assert sorted(o_topk[0, 0].tolist()) == want

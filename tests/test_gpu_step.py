@@ -221,3 +221,44 @@ def test_io_step_matches_device_step():
     for l, mode in enumerate(sched):
         if mode != "reuse":
             assert torch.equal(h_out["topk"][l], ref["topk"][l].cpu()), f"topk layer {l}"
+
+
+def test_verify_step_graph_sampled(orc):
+    """The verify workload at full size (8 sequences x 2^17 entries at 2:1, 64 draft queries
+    each, Full + Reuse layer) in the benchmark's launch configuration (captured CUDA graph,
+    replayed), so attention runs its 512-query launch.  Checked against the oracle on three
+    queries of two sequences: both layers' Top-512 (the Reuse layer's is inherited) at the
+    tie band, and both layers' attention outputs and log-sum-exp with the GPU's list."""
+    wl = synth.workload("verify")
+    sched = synth.layer_schedule(wl)
+    qd = synth.step_queries(wl)
+    x = build_state(wl, lambda b: synth.seq_tokens(wl, b, device="cuda"), qd)
+    step = DecodeStep(B=wl.B, Q=wl.Q, H=wl.H, HI=wl.HI, K=wl.K, window=wl.window, ratio=wl.ratio,
+                      schedule=sched, hier=False, max_n_vis=max(wl.lengths))
+    step.capture(x)
+    step.replay()
+    torch.cuda.synchronize()
+    step.check_status()
+    for b in (1, 6):
+        N = int(wl.lengths[b])
+        base = int(x.seq_base[b])
+        kv, ik = synth.seq_tokens(wl, b, device="cuda")
+        o_kv, o_ik = orc.pack_kv(bf16_bits(kv), bf16_bits(ik), wl.ratio)
+        del kv, ik
+        assert np.array_equal(np_u8(x.kv_pool[base:base + N]), o_kv), f"seq {b}: pool"
+        assert np.array_equal(np_u8(x.ik_pool[base:base + N]), o_ik), f"seq {b}: indexer pool"
+        for i in (0, 31, 63):
+            n_vis = int(qd["n_vis"][b, i])
+            s = orc.index_scores(qd["qi"][0][b, i].numpy(), qd["w"][0][b, i].numpy(), o_ik[:n_vis])
+            o_sel, _ = orc.topk(s, wl.K)
+            g_sel = step.topk[0].cpu().numpy()[b, i]
+            assert_topk_set(g_sel, o_sel, s, wl.K, what=f"seq {b} query {i}")
+            one = lambda t: t[b:b + 1, i:i + 1].numpy()
+            for l in range(len(sched)):
+                o_out, o_lse = orc.sparse_attn(one(qd["q"][l]), o_kv, np.zeros(1, np.int64),
+                                               g_sel.reshape(1, 1, -1), qd["swa"][l][b:b + 1].numpy(),
+                                               qd["swa_start"][b:b + 1].numpy(), one(qd["q_pos"]), SM,
+                                               window=wl.window)
+                assert_attn_close(step.out[l].cpu().numpy()[b:b + 1, i:i + 1], o_out,
+                                  what=f"seq {b} query {i} layer {l}")
+                assert np.abs(step.lse[l].cpu().numpy()[b:b + 1, i:i + 1] - o_lse).max() < 1e-2
