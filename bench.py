@@ -43,6 +43,8 @@ WORKLOAD_TEXT = {
                 "layer, H=64 x 512, HI=8 x 128, W=128",
     "verify": "multi-query verify: B=8 x 128K entries (2:1 of 256K tokens), Q=64 drafts, Full + Reuse layer",
     "tiny": "tiny decode: 1 sequence, 4096 entries, H=16, HI=4, Top-512, W=128",
+    "prefill": "chunked prefill: 1 sequence of 256K tokens at 2:1 (128K entries), a chunk of 1024 new "
+               "tokens as queries (own causal limits), Full + Reuse layer, H=64 x 512, HI=8 x 128, Top-512",
 }
 
 
@@ -60,7 +62,7 @@ def parse_args():
     p.add_argument("--no-call-timing", action="store_true",
                    help="time the step without the per-call events (no breakdown or roofline)")
     p.add_argument("--no-configs", action="store_true",
-                   help="measure only --workload (by default hier1m also brings full128k and verify)")
+                   help="measure only --workload (by default hier1m also brings full128k, verify and prefill)")
     return p.parse_args()
 
 
@@ -289,14 +291,14 @@ CALL_KERNELS = {
     "index_hier": ("stream_scan_kernel<hier> + select_kernel", "hbm"),
     "index_full": ("stream_scan_kernel<flat> + select_kernel", "hbm"),
     "reindex": ("reindex_scan_kernel + select_kernel", "hbm"),
-    "attn": ("attn_tc_kernel", "tensor"),
+    "attn": ("attn_kernel", "tensor"),
     "pack": ("pack_kv_kernel", "hbm"),
 }
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the call's
 # dominant kernel, from an ncu capture of that kernel as it is now, per workload; a kernel
 # that changes drops out of this table until it is captured again.
-NCU_DRAM_BYTES_PER_LAUNCH = {("hier1m", "attn"): 1656064}
+NCU_DRAM_BYTES_PER_LAUNCH = {}
 
 
 def call_rooflines(wl, per_call, counts, steps, peaks):
@@ -482,7 +484,7 @@ def run_ours(args, world, rank, local):
     # the metric's other decode configurations, each measured the same way
     configs = {}
     if not args.no_configs and args.workload == "hier1m":
-        for name in ("full128k", "verify"):
+        for name in ("full128k", "verify", "prefill"):
             c = measure(name, args.steps, args.warmup, world, dev, call_timing=not args.no_call_timing)
             cc = call_rooflines(c["wl"], c["per_call"], c["counts"], args.steps, peaks) if c["per_call"] else {}
             configs[name] = {"value": round(c["us_per_token"], 3), "unit": UNIT,
@@ -497,9 +499,10 @@ def run_ours(args, world, rank, local):
 
 
 # ---- the oracle, timed on the host cores ------------------------------------------------------
-def oracle_sample_state(wl, nseq, device):
+def oracle_sample_state(wl, nseq, device, nq=None):
     """The oracle's own pool for the first `nseq` sequences (packed from the same seeded
-    tokens) plus the step inputs of those sequences."""
+    tokens) plus the step inputs of those sequences (of their first `nq` queries only,
+    when given: the new tokens are still all packed)."""
     import oracle
     import synth
     lengths = [int(n) for n in wl.lengths[:nseq]]
@@ -517,12 +520,12 @@ def oracle_sample_state(wl, nseq, device):
         new_kv.append(kvb[old:])
         new_ik.append(ikb[old:])
     qd = synth.step_queries(wl)
-    sl = slice(0, nseq)
+    sl, ql = slice(0, nseq), slice(0, nq if nq else wl.Q)
     return dict(kv_pool=np.concatenate(kv_pools), ik_pool=np.concatenate(ik_pools), base=bases,
                 lengths=lengths, new_kv=new_kv, new_ik=new_ik,
-                q=qd["q"][:, sl].numpy(), qi=qd["qi"][:, sl].numpy(), w=qd["w"][:, sl].numpy(),
+                q=qd["q"][:, sl, ql].numpy(), qi=qd["qi"][:, sl, ql].numpy(), w=qd["w"][:, sl, ql].numpy(),
                 swa=qd["swa"][:, sl].numpy(), swa_start=qd["swa_start"][sl].numpy(),
-                q_pos=qd["q_pos"][sl].numpy(), n_vis=qd["n_vis"][sl].numpy())
+                q_pos=qd["q_pos"][sl, ql].numpy(), n_vis=qd["n_vis"][sl, ql].numpy())
 
 
 def oracle_step(wl, st):
@@ -586,26 +589,27 @@ def time_pack(steps, warmup, device):
     return res
 
 
-def time_oracle(wl, nseq, steps, warmup, device):
+def time_oracle(wl, nseq, steps, warmup, device, nq=None):
     import oracle
-    st = oracle_sample_state(wl, nseq, device)
+    st = oracle_sample_state(wl, nseq, device, nq)
     for _ in range(warmup):
         oracle_step(wl, st)
     t0 = time.perf_counter()
     for _ in range(steps):
         oracle_step(wl, st)
     dt = time.perf_counter() - t0
-    tokens = nseq * wl.Q
+    nq = nq if nq else wl.Q
+    tokens = nseq * nq
     # the oracle spreads queries over its threads, or the work inside a query when there
     # are fewer queries than threads, so every thread takes part either way
     cores = oracle.num_threads()
     sample = (f"{nseq} of {wl.B} sequences of the {wl.name} workload (full context, all "
-              f"{wl.n_layers} layers, {wl.Q} quer{'y' if wl.Q == 1 else 'ies'} each), {steps} step(s)")
+              f"{wl.n_layers} layers, {nq} of {wl.Q} quer{'y' if wl.Q == 1 else 'ies'} each), {steps} step(s)")
     return dt * 1e6 / (steps * tokens), cores, sample
 
 
-def cpu_baseline(wl, nseq):
-    v, cores, sample = time_oracle(wl, nseq, 1, 0, "cuda")
+def cpu_baseline(wl, nseq, nq=None):
+    v, cores, sample = time_oracle(wl, nseq, 1, 0, "cuda", nq)
     return {"value": round(v, 1), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
             "cpu_model": cpu_model()}
 
@@ -640,7 +644,8 @@ def main():
         import synth
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seqs)
         for name, c in line.get("configs", {}).items():
-            c["cpu_baseline"] = cpu_baseline(synth.workload(name), 1)
+            # the prefill chunk's oracle sample: 64 of its 1024 queries (about 10 s of CPU)
+            c["cpu_baseline"] = cpu_baseline(synth.workload(name), 1, 64 if name == "prefill" else None)
     if rank == 0:
         print(json.dumps(line, ensure_ascii=False), flush=True)
     if world > 1:

@@ -233,6 +233,23 @@ csa2_status csa2_reindex_static(const float* q, const float* w, const uint8_t* i
                                 int K, int32_t* topk, float* topk_score, uint32_t* dev_status,
                                 cudaStream_t stream);
 
+/* ---------------------------------------------------------------------------------
+ * Test hook (no counterpart in the pages): csa2_index_full with one copy withheld.
+ * The first CTA of the streaming scan never copies tile `withheld_tile` (>= 0) of its
+ * run, so no barrier completes for it: the workers' bounded wait gives up (within about
+ * a second), the scan drains what it issued, releases its tensor memory and sets
+ * CSA2_DEV_TIMEOUT in *dev_status, and the selection that follows reads whatever keys
+ * were written.  The call itself returns CSA2_OK once enqueued.  It exists so tests can
+ * check that an expired device wait is reported and leaves the device usable; results
+ * of the call are unspecified.  Arguments as for csa2_index_full.
+ * --------------------------------------------------------------------------------- */
+csa2_status csa2_test_index_full_withheld_copy(const float* q, const float* w, const uint8_t* ik_pool,
+                                               int64_t pool_entries, const int64_t* seq_base,
+                                               const int32_t* n_vis, int B, int Q, int HI, int K,
+                                               int64_t max_n_vis, int32_t* topk, float* topk_score,
+                                               void* ws, size_t ws_bytes, uint32_t* dev_status,
+                                               cudaStream_t stream, int withheld_tile);
+
 #ifdef __cplusplus
 }
 #endif

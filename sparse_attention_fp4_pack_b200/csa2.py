@@ -51,6 +51,9 @@ def lib():
         L.csa2_index_full_workspace_size.argtypes = [I32, I32, I32, I32, I64]
         L.csa2_index_full.restype = I32
         L.csa2_index_full.argtypes = [P, P, P, I64, P, P, I32, I32, I32, I32, I64, P, P, P, SZ, P, P]
+        L.csa2_test_index_full_withheld_copy.restype = I32
+        L.csa2_test_index_full_withheld_copy.argtypes = [P, P, P, I64, P, P, I32, I32, I32, I32, I64, P, P, P, SZ,
+                                                         P, P, I32]
         L.csa2_index_hier_workspace_size.restype = SZ
         L.csa2_index_hier_workspace_size.argtypes = [I32, I32, I32, I32, I32, I64]
         L.csa2_index_hier.restype = I32
@@ -198,6 +201,29 @@ def csa2_index_full(q, w, ik_pool, seq_base, n_vis, K, max_n_vis, topk, topk_sco
                                  _ptr(n_vis), B, Q, HI, K, int(max_n_vis), _ptr(topk), _ptr(topk_score),
                                  _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)),
            "csa2_index_full")
+
+
+def csa2_test_index_full_withheld_copy(q, w, ik_pool, seq_base, n_vis, K, max_n_vis, topk, withheld_tile,
+                                       topk_score=None, ws=None, dev_status=None, stream=None):
+    """Test hook: csa2_index_full whose streaming scan withholds one tile copy, so a bounded
+    device wait expires and CSA2_DEV_TIMEOUT is set in dev_status (results unspecified)."""
+    B, Q, HI = _query_dims(q, w, ik_pool, seq_base, n_vis)
+    _shape(topk, (B, Q, K), "topk")
+    _shape(topk_score, (B, Q, K), "topk_score")
+    _need(q, torch.float32, "q", 4)
+    _need(w, torch.float32, "w", 3)
+    _need(ik_pool, torch.uint8, "ik_pool", 2)
+    _need(seq_base, torch.int64, "seq_base", 1)
+    _need(n_vis, torch.int32, "n_vis", 2)
+    _need(topk, torch.int32, "topk", 3)
+    _need(topk_score, torch.float32, "topk_score", 3)
+    _status(dev_status)
+    if ws is None:
+        ws = workspace(csa2_index_full_workspace_size(B, Q, HI, K, max_n_vis), q.device)
+    _check(lib().csa2_test_index_full_withheld_copy(
+        _ptr(q), _ptr(w), _ptr(ik_pool), ik_pool.shape[0], _ptr(seq_base), _ptr(n_vis), B, Q, HI, K,
+        int(max_n_vis), _ptr(topk), _ptr(topk_score), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream),
+        int(withheld_tile)), "csa2_test_index_full_withheld_copy")
 
 
 # ---- a4 ---------------------------------------------------------------------------------

@@ -15,7 +15,7 @@ cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t
                          const int32_t* blocks, int B, int Q, int HI, int n_blocks, int block,
                          int K, int64_t max_n_vis, int32_t* out_idx, float* out_score,
                          uint32_t* keys, int64_t key_stride, uint32_t* status,
-                         cudaStream_t stream);
+                         cudaStream_t stream, int withheld_tile = -1);
 size_t attn_workspace_bytes(int B, int Q, int H, int K, int window);
 cudaError_t launch_sparse_attn(const float* q, const uint8_t* kv_pool, int64_t pool_entries,
                                const int64_t* seq_base, const int32_t* topk, int K,
@@ -134,6 +134,27 @@ csa2_status csa2_index_full(const float* q, const float* w, const uint8_t* ik_po
   return launched(csa2::launch_index(0, q, w, ik_pool, pool_entries, seq_base, n_vis, nullptr, B,
                                      Q, HI, 0, 1, K, max_n_vis, topk, topk_score,
                                      static_cast<uint32_t*>(ws), key_row(max_n_vis), dev_status, stream));
+}
+
+csa2_status csa2_test_index_full_withheld_copy(const float* q, const float* w, const uint8_t* ik_pool,
+                                               int64_t pool_entries, const int64_t* seq_base,
+                                               const int32_t* n_vis, int B, int Q, int HI, int K,
+                                               int64_t max_n_vis, int32_t* topk, float* topk_score, void* ws,
+                                               size_t ws_bytes, uint32_t* dev_status, cudaStream_t stream,
+                                               int withheld_tile) {
+  csa2_status st = check_index_common(q, w, ik_pool, pool_entries, seq_base, n_vis, B, Q, HI,
+                                      max_n_vis);
+  if (st != CSA2_OK) return st;
+  if (K < 1 || K > CSA2_MAX_K) return CSA2_ERR_UNSUPPORTED;
+  if (withheld_tile < 0) return CSA2_ERR_INVALID_ARG;
+  if ((int64_t)B * Q == 0) return CSA2_OK;
+  if (!topk || !aligned(topk, 4) || (topk_score && !aligned(topk_score, 4))) return CSA2_ERR_INVALID_ARG;
+  const size_t need = csa2_index_full_workspace_size(B, Q, HI, K, max_n_vis);
+  if ((st = check_ws(ws, ws_bytes, need)) != CSA2_OK) return st;
+  return launched(csa2::launch_index(0, q, w, ik_pool, pool_entries, seq_base, n_vis, nullptr, B,
+                                     Q, HI, 0, 1, K, max_n_vis, topk, topk_score,
+                                     static_cast<uint32_t*>(ws), key_row(max_n_vis), dev_status, stream,
+                                     withheld_tile));
 }
 
 size_t csa2_index_hier_workspace_size(int B, int Q, int HI, int n_blocks, int block,

@@ -61,6 +61,7 @@ struct ScanArgs {
   int64_t key_stride;
   uint32_t* keys;
   uint32_t* status;
+  int withheld_tile;      // test hook: the first CTA never copies this tile (-1: off)
 };
 
 __device__ __forceinline__ int64_t valid_count(const ScanArgs& a, int b, int bq, bool report) {
@@ -311,16 +312,18 @@ __global__ void __launch_bounds__(kScanThreads) reindex_scan_kernel(ScanArgs a) 
 //     copy starts at the 16 B boundary at or below the tile's first key (that lead,
 //     0..12 bytes, is the same for every tile of a sequence) and is rounded up to 16 B,
 //     falling back to word copies when the rounded copy would run past the pool;
-//   * the four worker warps own one tile row each: tile t's epilogue, then tile t+1's A
-//     operand, then thread 0 issues tile t+1's MMA.
-// The CTA is small (about 48 KB of shared memory, 160 threads), so four of them share an
-// SM and hide each other's MMA and copy latency.  Every wait is bounded; the workers
+//   * the four worker warps own one tile row each.  The A operand and the accumulator are
+//     doubled: the workers build tile t+1's A rows, thread 0 issues its MMA into the other
+//     accumulator, and only then do they run tile t's epilogue, whose MMA finished during
+//     the previous step, so the MMA round trip never waits on the chain.
+// The CTA is small (about 56 KB of shared memory, 160 threads), so four of them share an
+// SM and hide each other's copy latency.  Every wait is bounded; the workers
 // agree on giving up through a reducing barrier, and the copy warp waits for its
 // outstanding copies before the CTA exits.
 // ------------------------------------------------------------------------------------
 constexpr int kStreamWorkers = 128;                       // one tile row per thread
 constexpr int kStreamThreads = kStreamWorkers + 32;       // plus the copy warp
-constexpr int kStages = 3;                                // raw tiles in flight per CTA
+constexpr int kStages = 2;                                // raw tiles in flight per CTA
 constexpr int kRawTile = kRows * kIkBytes + 16;           // one tile plus its lead, 16 B multiple
 constexpr int kWorkerBar = 1;                             // named barrier of the workers
 
@@ -329,16 +332,16 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
   chain_enter();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = tc::align_smem_1024(smem_raw);
-  uint8_t* As = sm;                                   // [128 rows x 128 B], 128 B swizzle
-  uint8_t* Bs = As + kRows * 128;                     // [N rows x 128 B]
+  uint8_t* As = sm;                                   // 2 x [128 rows x 128 B], 128 B swizzle
+  uint8_t* Bs = As + 2 * kRows * 128;                 // [N rows x 128 B]
   uint8_t* raw = Bs + a.N * 128;                      // kStages x kRawTile
   int32_t* corr = reinterpret_cast<int32_t*>(raw + kStages * kRawTile);  // [N]
   float* wq = reinterpret_cast<float*>(corr + a.N);                      // [G * HIPAD]
   int64_t* nq = reinterpret_cast<int64_t*>(wq + a.G * HIPAD);            // [G] visible count per query
   uint64_t* full = reinterpret_cast<uint64_t*>(nq + a.G);                // [kStages] raw tile landed
   uint64_t* empty = full + kStages;                                      // [kStages] raw tile consumed
-  uint64_t* dfull = empty + kStages;                                     // accumulator ready
-  uint32_t* misc = reinterpret_cast<uint32_t*>(dfull + 1);               // tmem base, tiles built, issued
+  uint64_t* dfull = empty + kStages;                                     // [2] accumulator ready
+  uint32_t* misc = reinterpret_cast<uint32_t*>(dfull + 2);               // tmem base, tiles built, issued
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b = blockIdx.y / a.n_groups;
@@ -370,6 +373,7 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
       tc::mbar_init(empty_a + 8 * s, kStreamWorkers);
     }
     tc::mbar_init(dfull_a, 1);
+    tc::mbar_init(dfull_a + 8, 1);
   }
 
   // ---- B operand: four int8 limbs of every (query, head), plus epilogue constants ---------
@@ -432,6 +436,8 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
     int issued = 0;
     bool ok = true;
     for (int t = 0; t < ntiles; ++t) {
+      // test hook: stop copying, so the workers' wait for this tile runs out
+      if (t == a.withheld_tile && blockIdx.x == 0 && blockIdx.y == 0) break;
       const int s = t % kStages;
       if (t >= kStages) ok = tc::mbar_wait(empty_a + 8 * s, (uint32_t)((t / kStages) - 1) & 1u, kScanPolls);
       if (!__all_sync(0xffffffffu, ok)) {
@@ -465,10 +471,9 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
     const int row = tid;
     const uint32_t idesc = tc::idesc_i8(kRows, a.N, false, true);
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-    const uint32_t a_row = tc::smem_u32(As) + (uint32_t)row * 128u;  // this thread's A row
     const uint32_t corr_a = tc::smem_u32(corr), wq_a = tc::smem_u32(wq), nq_a = tc::smem_u32(nq);
 
-    // build tile t's A row from its raw buffer; returns false if the copy never landed
+    // build tile t's A row (buffer t & 1) from its raw buffer; false if the copy never landed
     auto build = [&](int t, float& sj, bool& valid) -> bool {
       const int s = t % kStages;
       const bool ok = tc::mbar_wait(full_a + 8 * s, (uint32_t)(t / kStages) & 1u, kScanPolls);
@@ -477,6 +482,7 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
       sj = 0.f;
       if (valid) {
         const uint32_t ea = raw_a + s * kRawTile + lead + row * kIkBytes;
+        const uint32_t a_row = tc::smem_u32(As) + (uint32_t)(t & 1) * (kRows * 128u) + (uint32_t)row * 128u;
         uint32_t cw[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) cw[i] = tc::ld_shared_u32(ea + 4 * i);
@@ -493,27 +499,30 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
       tc::fence_before_sync();
       return ok;
     };
-    auto issue = [&]() {
+    // tile t: A buffer t & 1 -> accumulator t & 1 (columns (t & 1) * N), completion on dfull[t & 1]
+    auto issue = [&](int t) {
       if (tid == 0) {
         tc::fence_after_sync();
-        const uint32_t ab = tc::smem_u32(As), bb = tc::smem_u32(Bs);
+        const uint32_t ab = tc::smem_u32(As) + (uint32_t)(t & 1) * (kRows * 128u), bb = tc::smem_u32(Bs);
+        const uint32_t d = tmem + (uint32_t)((t & 1) * a.N);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)  // K = 128 dims in steps of 32
-          tc::mma_i8(tmem, tc::smem_desc_sw128(ab + ks * 32, 16, 1024), tc::smem_desc_sw128(bb + ks * 32, 16, 1024),
+          tc::mma_i8(d, tc::smem_desc_sw128(ab + ks * 32, 16, 1024), tc::smem_desc_sw128(bb + ks * 32, 16, 1024),
                      idesc, ks > 0 ? 1u : 0u);
-        tc::commit(dfull_a);
+        tc::commit(dfull_a + 8u * (uint32_t)(t & 1));
       }
     };
     // limbs -> fp32 dot products -> ReLU-weighted score -> order-preserving keys of tile t
     auto epilogue = [&](int t, float sj, bool valid) -> bool {
-      const bool ok = tc::mbar_wait(dfull_a, (uint32_t)t & 1u, kScanPolls);
+      const bool ok = tc::mbar_wait(dfull_a + 8u * (uint32_t)(t & 1), (uint32_t)(t >> 1) & 1u, kScanPolls);
       tc::fence_after_sync();
       const int64_t j = item0 + (int64_t)t * kRows + row;
+      const uint32_t acc = lane_addr + (uint32_t)((t & 1) * a.N);
 #pragma unroll
       for (int g = 0; g < 8; ++g) {
         if (g >= G) break;
         uint32_t r[HIPAD * 4];
-        const uint32_t ta = lane_addr + (uint32_t)(g * HIPAD * 4);
+        const uint32_t ta = acc + (uint32_t)(g * HIPAD * 4);
         if (HIPAD == 4) {
           tc::tmem_ld16(ta, r);
         } else {
@@ -553,35 +562,37 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
       return ok;
     };
 
+    // step t: build and issue tile t+1, then the epilogue of tile t (whose MMA was issued
+    // one step earlier and has had the whole build to complete)
     float sj = 0.f, sj_nxt = 0.f;
     bool v = false, v_nxt = false;
-    int built = 0;  // tiles whose raw buffer every worker consumed
+    int issued = 0;  // tiles whose MMA was issued (their raw buffers were consumed)
     bool bad = tc::named_sync_or(kWorkerBar, kStreamWorkers, !build(0, sj, v));
     if (!bad) {
-      issue();
-      built = 1;
+      issue(0);
+      issued = 1;
     }
-    bool last_ok = true;
+    bool pend = false;  // a failed accumulator wait, voted on at the next barrier
     for (int t = 0; t < ntiles && !bad; ++t) {
-      bool fail = !epilogue(t, sj, v);
       if (t + 1 < ntiles) {
-        fail |= !build(t + 1, sj_nxt, v_nxt);
+        const bool fail = !build(t + 1, sj_nxt, v_nxt) || pend;
         bad = tc::named_sync_or(kWorkerBar, kStreamWorkers, fail);
-        if (!bad) {
-          issue();
-          built = t + 2;
-        }
-        sj = sj_nxt;
-        v = v_nxt;
-      } else {
-        last_ok = !fail;
+        if (bad) break;
+        issue(t + 1);
+        issued = t + 2;
       }
+      pend |= !epilogue(t, sj, v);
+      sj = sj_nxt;
+      v = v_nxt;
     }
+    // every worker reaches this vote: either all completed the loop or all left it together
+    bad = tc::named_sync_or(kWorkerBar, kStreamWorkers, bad || pend);
     if (tid == 0) {
-      if (bad || !last_ok) flag(a.status, CSA2_DEV_TIMEOUT);
-      if (bad && built > 0)  // let the last issued MMA finish before the accumulator goes
-        tc::mbar_wait(dfull_a, (uint32_t)(built - 1) & 1u, kScanPolls);
-      misc[1] = (uint32_t)(bad ? (built > 0 ? built - 1 : 0) : ntiles);
+      if (bad) flag(a.status, CSA2_DEV_TIMEOUT);
+      // let the issued MMAs finish before the accumulators go (they complete in order)
+      if (bad && issued > 0)
+        tc::mbar_wait(dfull_a + 8u * (uint32_t)((issued - 1) & 1), (uint32_t)((issued - 1) >> 1) & 1u, kScanPolls);
+      misc[1] = (uint32_t)(bad ? issued : ntiles);
     }
   }
   __syncthreads();
@@ -1133,15 +1144,16 @@ static cudaError_t resident_ctas(F fn, int dev, int threads, size_t dyn_smem, in
 template <int MODE>
 static cudaError_t launch_stream(ScanArgs a, int64_t items, int B, cudaStream_t st) {
   a.hipad = a.HI <= 4 ? 4 : (a.HI <= 8 ? 8 : 16);
-  a.G = max(1, min(a.Q, 256 / (a.hipad * 4)));
+  // accumulator pairs of 2N <= 256 columns, so two CTAs' tensor memory fits an SM
+  a.G = max(1, min(a.Q, 128 / (a.hipad * 4)));
   a.n_groups = (a.Q + a.G - 1) / a.G;
   a.N = a.G * a.hipad * 4;
-  a.tmem_cols = pow2_at_least(a.N);
+  a.tmem_cols = pow2_at_least(2 * a.N);
   const int64_t tiles = (items + kRows - 1) / kRows;
   const int64_t rows = (int64_t)B * a.n_groups;
   if (tiles == 0 || rows == 0) return cudaSuccess;
-  const size_t smem = 1024 + (size_t)kRows * 128 + (size_t)a.N * 128 + (size_t)kStages * kRawTile +
-                      (size_t)a.N * 4 + (size_t)a.G * a.hipad * 4 + (size_t)a.G * 8 + (2 * kStages + 1) * 8 + 16;
+  const size_t smem = 1024 + 2 * (size_t)kRows * 128 + (size_t)a.N * 128 + (size_t)kStages * kRawTile +
+                      (size_t)a.N * 4 + (size_t)a.G * a.hipad * 4 + (size_t)a.G * 8 + (2 * kStages + 2) * 8 + 16;
   int dev = 0, sms = 148, occ = 1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -1182,8 +1194,9 @@ cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t
                          const int32_t* blocks, int B, int Q, int HI, int n_blocks, int block,
                          int K, int64_t max_n_vis, int32_t* out_idx, float* out_score,
                          uint32_t* keys, int64_t key_stride, uint32_t* status,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, int withheld_tile) {
   ScanArgs a;
+  a.withheld_tile = withheld_tile;
   a.q = q;
   a.w = w;
   a.ik_pool = ik_pool;

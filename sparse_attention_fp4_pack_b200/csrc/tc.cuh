@@ -137,10 +137,27 @@ __device__ __forceinline__ void mbar_init(uint32_t mbar_saddr, uint32_t count) {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
+// Nanoseconds of the GPU's global timer.
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Longest a single wait may take before it gives up, whatever its poll budget.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
+
 // Wait for the given phase parity; gives up after max_tries polls (each poll may itself
-// suspend for a bounded time).  Returns false on timeout.
+// suspend for a bounded time) or after kWaitLimitNs of wall time, whichever comes first.
+// Returns false on timeout.
 __device__ __forceinline__ bool mbar_wait(uint32_t mbar_saddr, uint32_t parity, uint32_t max_tries) {
+  uint64_t t0 = 0;
   for (uint32_t i = 0; i < max_tries; ++i) {
+    if ((i & 255u) == 255u) {  // check the clock now and then
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > kWaitLimitNs) return false;
+    }
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"

@@ -14,6 +14,8 @@ Workload shapes follow the five decode configurations of the build's target:
   full128k   B=32, N_b ~ U{65536..131072}, H=64, HI=8, K=512, W=128        (seed 2)
   hier1m     B=4, N=2^20, hierarchical Full + 10 Reindex + 9 Reuse layers  (seed 3)
   verify     B=8, 2^18 tokens at 2:1 = 2^17 entries, Q=64 drafts          (seed 4)
+  prefill    B=1, 2^18 tokens at 2:1 = 2^17 entries, a chunk of Q=1024    (seed 5)
+             new tokens, each a query with its own causal limit
 """
 from dataclasses import dataclass, field
 import zlib
@@ -128,6 +130,9 @@ def workload(name: str) -> DecodeWorkload:
     if name == "verify":
         return DecodeWorkload("verify", 4, B=8, Q=64, H=64, HI=8, K=512, window=128, ratio=2,
                               lengths=[1 << 17] * 8, new_tokens=64)
+    if name == "prefill":
+        return DecodeWorkload("prefill", 5, B=1, Q=1024, H=64, HI=8, K=512, window=128, ratio=2,
+                              lengths=[1 << 17], new_tokens=1024)
     raise ValueError(name)
 
 

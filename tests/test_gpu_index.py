@@ -122,7 +122,8 @@ def test_bad_count_every_query_of_a_sequence(orc):
 
 
 @pytest.mark.parametrize("N,n_blocks,block", [(37, 2, 8), (5003, 64, 8), (16384, 2048, 8),
-                                              (20011, 512, 8), (3000, 100, 1), (9000, 40, 32)])
+                                              (20011, 512, 8), (3000, 100, 1), (9000, 40, 32),
+                                              (40000, 1024, 32)])
 def test_hier_blocks_and_reindex(orc, N, n_blocks, block):
     kv, ik = synth.kv_tokens(60 + N % 97, N, device="cuda")
     _, ikp, _, o_ik = pools_from_tokens(orc, kv, ik)

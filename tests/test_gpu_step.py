@@ -262,3 +262,40 @@ def test_verify_step_graph_sampled(orc):
                 assert_attn_close(step.out[l].cpu().numpy()[b:b + 1, i:i + 1], o_out,
                                   what=f"seq {b} query {i} layer {l}")
                 assert np.abs(step.lse[l].cpu().numpy()[b:b + 1, i:i + 1] - o_lse).max() < 1e-2
+
+
+def test_prefill_chunk_graph_sampled(orc):
+    """Chunked prefill at full size: one sequence of 2^18 tokens at 2:1 (2^17 entries), a chunk
+    of 1024 new tokens whose queries each see their own causal prefix, Full + Reuse layer, in
+    the benchmark's launch configuration (captured graph, replayed).  The packed pool equals
+    the oracle's; five queries spread over the chunk are checked against the oracle: the Full
+    layer's Top-512 at the tie band and both layers' attention with the GPU's list."""
+    wl = synth.workload("prefill")
+    sched = synth.layer_schedule(wl)
+    qd = synth.step_queries(wl)
+    x = build_state(wl, lambda b: synth.seq_tokens(wl, b, device="cuda"), qd)
+    step = DecodeStep(B=wl.B, Q=wl.Q, H=wl.H, HI=wl.HI, K=wl.K, window=wl.window, ratio=wl.ratio,
+                      schedule=sched, hier=False, max_n_vis=max(wl.lengths))
+    step.capture(x)
+    step.replay()
+    torch.cuda.synchronize()
+    step.check_status()
+    b, N = 0, int(wl.lengths[0])
+    kv, ik = synth.seq_tokens(wl, b, device="cuda")
+    o_kv, o_ik = orc.pack_kv(bf16_bits(kv), bf16_bits(ik), wl.ratio)
+    del kv, ik
+    assert np.array_equal(np_u8(x.kv_pool[:N]), o_kv)
+    assert np.array_equal(np_u8(x.ik_pool[:N]), o_ik)
+    for i in (0, 1, 511, 1000, 1023):
+        n_vis = int(qd["n_vis"][b, i])
+        s = orc.index_scores(qd["qi"][0][b, i].numpy(), qd["w"][0][b, i].numpy(), o_ik[:n_vis])
+        o_sel, _ = orc.topk(s, wl.K)
+        g_sel = step.topk[0].cpu().numpy()[b, i]
+        assert_topk_set(g_sel, o_sel, s, wl.K, what=f"query {i}")
+        one = lambda t: t[b:b + 1, i:i + 1].numpy()
+        for l in range(len(sched)):
+            o_out, o_lse = orc.sparse_attn(one(qd["q"][l]), o_kv, np.zeros(1, np.int64), g_sel.reshape(1, 1, -1),
+                                           qd["swa"][l][b:b + 1].numpy(), qd["swa_start"][b:b + 1].numpy(),
+                                           one(qd["q_pos"]), SM, window=wl.window)
+            assert_attn_close(step.out[l].cpu().numpy()[b:b + 1, i:i + 1], o_out, what=f"query {i} layer {l}")
+            assert np.abs(step.lse[l].cpu().numpy()[b:b + 1, i:i + 1] - o_lse).max() < 1e-2
