@@ -39,6 +39,11 @@ def lib():
         L.orc_bf16_value.argtypes = [ctypes.c_uint16]
         L.orc_num_threads.restype = i32
         L.orc_pack_kv.argtypes = [c_p, c_p, i64, i32, c_p, c_p]
+        L.orc_bf16_round.restype = ctypes.c_uint16
+        L.orc_bf16_round.argtypes = [flt]
+        L.orc_norm_rope_row.argtypes = [c_p, c_p, c_p, c_p, flt, c_p]
+        L.orc_pack_kv_normed.restype = i32
+        L.orc_pack_kv_normed.argtypes = [c_p, c_p, i64, i32, c_p, c_p, c_p, i64, c_p, flt, c_p, c_p]
         L.orc_dequant_kv.argtypes = [c_p, c_p]
         L.orc_dequant_ik.argtypes = [c_p, c_p]
         L.orc_index_scores.argtypes = [c_p, c_p, i32, c_p, i64, c_p]
@@ -97,6 +102,42 @@ def pack_kv(kv_bf16: np.ndarray, ik_bf16: np.ndarray, ratio: int):
     ik_out = np.zeros((E, 68), np.uint8)
     lib().orc_pack_kv(_p(kv), _p(ik), T, ratio, _p(kv_out), _p(ik_out))
     return kv_out, ik_out
+
+
+def bf16_round(v: float) -> int:
+    return int(lib().orc_bf16_round(v))
+
+
+def norm_rope_row(x_bf16: np.ndarray, cos_p: np.ndarray, sin_p: np.ndarray, gamma=None, eps=1e-6) -> np.ndarray:
+    """One token [512] bf16 bits -> fp32 [512], normalised and rotated (cos_p, sin_p [256])."""
+    x = _c(x_bf16, np.uint16)
+    c = _c(cos_p, np.float32)
+    s = _c(sin_p, np.float32)
+    g = None if gamma is None else _c(gamma, np.float32)
+    assert x.shape == (512,) and c.shape == (256,) and s.shape == (256,)
+    y = np.zeros(512, np.float32)
+    lib().orc_norm_rope_row(_p(x), _p(c), _p(s), _p(g), float(eps), _p(y))
+    return y
+
+
+def pack_kv_normed(kv_bf16, ik_bf16, ratio, pos, rope_cos, rope_sin, gamma=None, eps=1e-6):
+    """Producer: raw kv [T,512] / ik [T,128] bf16 bits, positions [T] into the tables
+    rope_cos / rope_sin [n_pos,256] -> (kv [T/ratio,288], ik [T/ratio,68], any_bad_position)."""
+    kv = _c(kv_bf16, np.uint16)
+    ik = _c(ik_bf16, np.uint16)
+    T = kv.shape[0]
+    assert kv.shape == (T, 512) and ik.shape == (T, 128) and ratio in (1, 2) and T % ratio == 0
+    ps = _c(pos, np.int64)
+    c = _c(rope_cos, np.float32)
+    s = _c(rope_sin, np.float32)
+    assert ps.shape == (T,) and c.shape == s.shape and c.shape[1] == 256
+    g = None if gamma is None else _c(gamma, np.float32)
+    E = T // ratio
+    kv_out = np.zeros((E, 288), np.uint8)
+    ik_out = np.zeros((E, 68), np.uint8)
+    bad = lib().orc_pack_kv_normed(_p(kv), _p(ik), T, ratio, _p(ps), _p(c), _p(s), c.shape[0], _p(g), float(eps),
+                                   _p(kv_out), _p(ik_out))
+    return kv_out, ik_out, bool(bad)
 
 
 def dequant_kv(entries: np.ndarray) -> np.ndarray:

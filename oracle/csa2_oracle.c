@@ -212,6 +212,102 @@ void orc_pack_kv(const uint16_t* kv, const uint16_t* ik, int64_t T, int ratio, u
   }
 }
 
+/* ------------------------------------------------------------------------------------
+ * Producer: RMSNorm + rotary position encoding, then the pack above (P3 §4비트로 적어도
+ * 되는 이유: cached values are normalised and rotated before they are cached, which is
+ * what bounds them by sqrt(512); the pages give no formula).
+ *
+ * Readings (the pages are silent; every operation is one fp32 rounding, no contraction):
+ *  - RMSNorm of a 512-channel token x (bf16):  S = sum of x_c^2 by a fixed pairwise order:
+ *    within each 16-channel block b, halving (element i += element i+8, then +4, +2, +1);
+ *    then over the 32 block sums, halving (b += b+16, then +8, +4, +2, +1).
+ *    m = S / 512;  r = 1 / sqrt(m + eps) as three rounded steps (add, sqrt, reciprocal);
+ *    n_c = x_c * r, then n_c * gamma_c when a gain is given.
+ *  - rotation of channel pairs (2i, 2i+1), i = 0..255, by the caller's tables at the
+ *    token's position p:  c = cos[p][i], s = sin[p][i];
+ *    y_2i = n_2i c - n_2i+1 s,  y_2i+1 = n_2i s + n_2i+1 c  (each product rounded).
+ *  - y is rounded to bf16 (nearest, ties to even), then packed exactly as orc_pack_kv
+ *    packs bf16 tokens (ratio 2: each token is normalised and rotated at its own
+ *    position, the pair mean is taken from the two bf16 results).  The indexer key is
+ *    packed from its own bf16 input unchanged.
+ * ------------------------------------------------------------------------------------ */
+
+/* Nearest bf16 (ties to even) of a finite fp32 value, as raw bits. */
+uint16_t orc_bf16_round(float v) {
+  uint32_t u;
+  memcpy(&u, &v, 4);
+  uint32_t lsb = (u >> 16) & 1u;
+  return (uint16_t)((u + 0x7FFFu + lsb) >> 16);
+}
+
+/* One token: x [512] bf16 bits -> y [512] fp32, normalised and rotated at position p
+ * (cos_p, sin_p: that position's 256-entry table rows; gamma may be NULL). */
+void orc_norm_rope_row(const uint16_t* x, const float* cos_p, const float* sin_p, const float* gamma,
+                       float eps, float* y) {
+  float v[ORC_D], blk[32];
+  for (int c = 0; c < ORC_D; ++c) v[c] = orc_bf16_value(x[c]);
+  for (int b = 0; b < 32; ++b) {
+    float t[16];
+    for (int i = 0; i < 16; ++i) t[i] = v[16 * b + i] * v[16 * b + i];
+    for (int h = 8; h >= 1; h /= 2)
+      for (int i = 0; i < h; ++i) t[i] = t[i] + t[i + h];
+    blk[b] = t[0];
+  }
+  for (int h = 16; h >= 1; h /= 2)
+    for (int b = 0; b < h; ++b) blk[b] = blk[b] + blk[b + h];
+  float m = blk[0] / 512.0f;
+  float r = 1.0f / sqrtf(m + eps);
+  float n[ORC_D];
+  for (int c = 0; c < ORC_D; ++c) {
+    n[c] = v[c] * r;
+    if (gamma) n[c] = n[c] * gamma[c];
+  }
+  for (int i = 0; i < ORC_D / 2; ++i) {
+    float c = cos_p[i], s = sin_p[i];
+    float a = n[2 * i], b = n[2 * i + 1];
+    float ac = a * c, bs = b * s, as = a * s, bc = b * c;
+    y[2 * i] = ac - bs;
+    y[2 * i + 1] = as + bc;
+  }
+}
+
+/* Producer: kv [T][512] raw bf16 tokens at positions pos[T] (indices into the tables,
+ * rope_cos/rope_sin [n_pos][256]), ik [T][128] bf16; writes T/ratio contiguous entries.
+ * A position outside [0, n_pos) leaves its entry all zero and returns nonzero. */
+int orc_pack_kv_normed(const uint16_t* kv, const uint16_t* ik, int64_t T, int ratio, const int64_t* pos,
+                       const float* rope_cos, const float* rope_sin, int64_t n_pos, const float* gamma,
+                       float eps, uint8_t* kv_out, uint8_t* ik_out) {
+  int64_t E = T / ratio;
+  int bad = 0;
+  uint16_t* tok = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(T > 0 ? T : 1) * ORC_D);
+#pragma omp parallel for schedule(static) reduction(| : bad)
+  for (int64_t t = 0; t < T; ++t) {
+    float y[ORC_D];
+    int64_t p = pos[t];
+    if (p < 0 || p >= n_pos) {
+      bad = 1;
+      for (int c = 0; c < ORC_D; ++c) tok[t * ORC_D + c] = 0;
+      continue;
+    }
+    orc_norm_rope_row(kv + t * ORC_D, rope_cos + p * (ORC_D / 2), rope_sin + p * (ORC_D / 2), gamma, eps, y);
+    for (int c = 0; c < ORC_D; ++c) tok[t * ORC_D + c] = orc_bf16_round(y[c]);
+  }
+  orc_pack_kv(tok, ik, T, ratio, kv_out, ik_out);
+  for (int64_t j = 0; j < E; ++j) {  /* entries with a bad position stay zero */
+    int zero = 0;
+    for (int k = 0; k < ratio; ++k) {
+      int64_t p = pos[j * ratio + k];
+      if (p < 0 || p >= n_pos) zero = 1;
+    }
+    if (zero) {
+      memset(kv_out + j * ORC_KV_BYTES, 0, ORC_KV_BYTES);
+      memset(ik_out + j * ORC_IK_BYTES, 0, ORC_IK_BYTES);
+    }
+  }
+  free(tok);
+  return bad;
+}
+
 /* Exact dequantisation (products of an E2M1 value and a scale are exact in double). */
 void orc_dequant_kv(const uint8_t* e, double* out /*[512]*/) {
   for (int c = 0; c < ORC_D; ++c) {

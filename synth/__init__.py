@@ -72,6 +72,29 @@ def swa_window(seed, B, S_w, device="cpu", stream="swa"):
     return x.to(torch.float8_e4m3fn).view(torch.uint8)
 
 
+def rope_tables(n_pos, device="cpu", base=10000.0):
+    """cos / sin input tables [n_pos, 256] fp32 for rotating channel pairs at positions
+    0..n_pos-1 with the usual rotary frequencies base^(-i/256) (the producer takes the
+    tables as inputs and does not compute them)."""
+    i = torch.arange(256, dtype=torch.float64)
+    inv = base ** (-i / 256.0)
+    ang = torch.arange(int(n_pos), dtype=torch.float64)[:, None] * inv[None, :]
+    return ang.cos().to(torch.float32).to(device), ang.sin().to(torch.float32).to(device)
+
+
+def raw_kv_tokens(seed, T, device="cpu", stream="raw"):
+    """Raw (pre-normalisation) bf16 main-KV tokens [T,512]: N(0,1) times a per-token
+    magnitude 2^U(-4,4), 0.1% of the elements scaled by 8; plus indexer keys [T,128]."""
+    T = int(T)
+    x = normal(seed, stream + ".main", (T, D), device)
+    u = torch.rand(T, D, generator=_gen(seed, stream + ".tail", device), device=device)
+    x = torch.where(u < 1e-3, x * 8.0, x)
+    mag = torch.rand(T, 1, generator=_gen(seed, stream + ".mag", device), device=device) * 8.0 - 4.0
+    x = x * torch.exp2(mag)
+    ik = normal(seed, stream + ".ik", (T, DI), device)
+    return x.to(torch.bfloat16), ik.to(torch.bfloat16)
+
+
 def queries(seed, B, Q, H, device="cpu", stream="q"):
     return normal(seed, stream, (B, Q, H, D), device)
 

@@ -98,6 +98,17 @@ MUTANTS = [
      "const uint8_t* row = swa + ((size_t)r) * ORC_D;"),
     ("entries ignore the sequence base", "orc_dequant_kv(kv_pool + (seq_base[b] + j) * ORC_KV_BYTES",
      "orc_dequant_kv(kv_pool + (j) * ORC_KV_BYTES"),
+    # producer: RMSNorm + rotation
+    ("norm sums half of each block", "for (int h = 8; h >= 1; h /= 2)", "for (int h = 4; h >= 1; h /= 2)"),
+    ("norm mean over 256 channels", "float m = blk[0] / 512.0f;", "float m = blk[0] / 256.0f;"),
+    ("norm without eps", "float r = 1.0f / sqrtf(m + eps);", "float r = 1.0f / sqrtf(m);"),
+    ("gain ignored", "if (gamma) n[c] = n[c] * gamma[c];", ""),
+    ("rotation sign", "y[2 * i] = ac - bs;", "y[2 * i] = ac + bs;"),
+    ("rotation pair crossed", "y[2 * i + 1] = as + bc;", "y[2 * i + 1] = bs + ac;"),
+    ("rotation table of the next position", "rope_cos + p * (ORC_D / 2), rope_sin + p * (ORC_D / 2)",
+     "rope_cos + (p + 1) * (ORC_D / 2), rope_sin + (p + 1) * (ORC_D / 2)"),
+    ("bf16 rounding truncates", "return (uint16_t)((u + 0x7FFFu + lsb) >> 16);", "return (uint16_t)(u >> 16);"),
+    ("bad position keeps its entry", "    if (zero) {\n      memset(kv_out", "    if (0) {\n      memset(kv_out"),
 ]
 
 

@@ -172,3 +172,113 @@ def test_dequant_reconstructs_within_half_step(orc):
     xi = ik.to(torch.float64).numpy()
     s = pi[:, 64:68].copy().view(np.float32)[:, 0].astype(np.float64)
     assert (np.abs(z - xi).max(axis=1) <= s + 1e-12).all()
+
+
+# ---- producer: RMSNorm + rotation, then the pack (P3 §4비트로 적어도 되는 이유) -----------------
+def _bits(x):
+    return torch.from_numpy(np.asarray(x, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+
+
+def _identity(n_pos=1):
+    return np.ones((n_pos, 256), np.float32), np.zeros((n_pos, 256), np.float32)
+
+
+def test_normed_constant_row_is_unit(orc):
+    """A row of equal values a normalises to exactly 1 (S = 512 a^2 exact, r = 1/|a|) and
+    then packs as a row of ones."""
+    c, s = _identity()
+    for a in (0.5, 2.0, -0.25, 3.0):
+        y = orc.norm_rope_row(_bits(np.full(512, a)), c[0], s[0], eps=0.0)
+        assert np.all(y == np.float32(np.sign(a))), a
+    kv, ik, bad = orc.pack_kv_normed(_bits(np.full((1, 512), 3.0)), _bits(np.zeros((1, 128))), 1,
+                                     np.zeros(1, np.int64), c, s, eps=0.0)
+    ones, _ = orc.pack_kv(_bits(np.ones((1, 512))), _bits(np.zeros((1, 128))), 1)
+    assert not bad and np.array_equal(kv, ones)
+
+
+def test_normed_mean_square_is_one(orc):
+    """Without eps the normalised row (identity rotation) has mean square 1 to fp32
+    accuracy, at any input scale (the RMS bound sqrt(512) on the L2 norm)."""
+    c, s = _identity()
+    x, _ = synth.raw_kv_tokens(40, 64)
+    xb = x.view(torch.int16).numpy().astype(np.uint16)
+    for t in range(64):
+        y = orc.norm_rope_row(xb[t], c[0], s[0], eps=0.0).astype(np.float64)
+        assert abs(np.mean(y * y) - 1.0) < 5e-6
+        assert np.linalg.norm(y) <= np.sqrt(512) * (1 + 5e-6)
+
+
+def test_normed_matches_float64_definition(orc):
+    """Against the definition evaluated in float64 (independent of the rounding order): a
+    wrong pair, sign, table row or gain index shows up far above 1e-5."""
+    x, _ = synth.raw_kv_tokens(41, 8)
+    xb = x.view(torch.int16).numpy().astype(np.uint16)
+    cos, sin = synth.rope_tables(50)
+    cos, sin = cos.numpy(), sin.numpy()
+    g = (np.arange(512) % 7 + 1).astype(np.float32) / 4
+    for t, p in enumerate((0, 1, 7, 49, 13, 2, 30, 31)):
+        xv = x[t].float().numpy().astype(np.float64)
+        n = xv / np.sqrt(np.mean(xv * xv) + 1e-6) * g
+        want = np.empty(512)
+        want[0::2] = n[0::2] * cos[p] - n[1::2] * sin[p]
+        want[1::2] = n[0::2] * sin[p] + n[1::2] * cos[p]
+        got = orc.norm_rope_row(xb[t], cos[p], sin[p], gamma=g, eps=1e-6)
+        assert np.max(np.abs(got - want)) <= 1e-5 * np.max(np.abs(want)), (t, p)
+
+
+def test_normed_quarter_turn_swaps_pairs(orc):
+    """cos = 0, sin = 1 rotates every pair by a quarter turn: (a, b) -> (-b, a) exactly."""
+    x, _ = synth.raw_kv_tokens(42, 1)
+    xb = x.view(torch.int16).numpy().astype(np.uint16)[0]
+    c0, s0 = _identity()
+    n = orc.norm_rope_row(xb, c0[0], s0[0])
+    y = orc.norm_rope_row(xb, np.zeros(256, np.float32), np.ones(256, np.float32))
+    assert np.array_equal(y[0::2], -n[1::2]) and np.array_equal(y[1::2], n[0::2])
+
+
+def test_normed_gain_is_per_channel(orc):
+    """A gain that doubles one channel changes that channel alone, by exactly 2."""
+    x, _ = synth.raw_kv_tokens(43, 1)
+    xb = x.view(torch.int16).numpy().astype(np.uint16)[0]
+    c, s = _identity()
+    g = np.ones(512, np.float32)
+    g[77] = 2.0
+    a = orc.norm_rope_row(xb, c[0], s[0])
+    b = orc.norm_rope_row(xb, c[0], s[0], gamma=g)
+    assert b[77] == 2 * a[77] and np.array_equal(np.delete(a, 77), np.delete(b, 77))
+
+
+def test_bf16_round_is_nearest_even(orc):
+    """bf16 rounding against torch's fp32 -> bf16 cast (a library routine) on values
+    that sit on, above and below the ties."""
+    vals = np.array([1.0, 1.00390625, 1.005859375, 1.0078125, -3.0117188, 1e-20, 65504.0, 0.1, -0.3333],
+                    np.float32)
+    rng = np.random.default_rng(5)
+    vals = np.concatenate([vals, rng.standard_normal(2000).astype(np.float32) * 10])
+    want = torch.from_numpy(vals).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+    got = np.array([orc.bf16_round(float(v)) for v in vals], np.uint16)
+    assert np.array_equal(got, want)
+
+
+def test_normed_pack_is_pack_of_rounded_rows(orc):
+    """The producer equals the plain pack of its bf16-rounded rows, at both ratios, each
+    token at its own position; a position past the tables empties its entry."""
+    T = 20
+    x, ik = synth.raw_kv_tokens(44, T)
+    xb = x.view(torch.int16).numpy().astype(np.uint16)
+    ib = ik.view(torch.int16).numpy().astype(np.uint16)
+    cos, sin = synth.rope_tables(64)
+    cos, sin = cos.numpy(), sin.numpy()
+    pos = np.arange(T, dtype=np.int64) * 3
+    rows = np.stack([np.array([orc.bf16_round(float(v)) for v in orc.norm_rope_row(xb[t], cos[pos[t]], sin[pos[t]])],
+                              np.uint16) for t in range(T)])
+    for ratio in (1, 2):
+        kv, ikp, bad = orc.pack_kv_normed(xb, ib, ratio, pos, cos, sin)
+        want_kv, want_ik = orc.pack_kv(rows, ib, ratio)
+        assert not bad and np.array_equal(kv, want_kv) and np.array_equal(ikp, want_ik)
+    pos2 = pos.copy()
+    pos2[5] = 64
+    kv, ikp, bad = orc.pack_kv_normed(xb, ib, 1, pos2, cos, sin)
+    want_kv, _ = orc.pack_kv(rows, ib, 1)
+    assert bad and not kv[5].any() and not ikp[5].any()
+    assert np.array_equal(np.delete(kv, 5, axis=0), np.delete(want_kv, 5, axis=0))
