@@ -559,7 +559,8 @@ def oracle_step(wl, st):
 def time_pack(steps, warmup, device):
     """FP4 pack throughput on 2^20 new tokens (512-channel main KV + 128-dim indexer key,
     bf16, resident in HBM) at 1:1 and 2:1: (bytes read + bytes written) / device time, L2
-    flushed between launches.  Inputs follow the pack workload's value recipe."""
+    flushed between launches.  Inputs follow the pack workload's value recipe.  The same
+    for the producer that normalises and rotates raw tokens before packing them."""
     import synth
     from sparse_attention_fp4_pack_b200 import csa2
     T = 1 << 20
@@ -584,7 +585,29 @@ def time_pack(steps, warmup, device):
         nbytes = T * 1280 + (T // ratio) * 356
         res[f"{ratio}:1"] = {"GB/s": round(nbytes / (ms * 1e-3) / 1e9, 1), "us": round(ms * 1e3, 1),
                              "bytes": nbytes}
-    del kv, ik, kvp, ikp, flush
+    # the producer (RMSNorm + rotation + pack) on raw tokens at positions 0..T-1: it also
+    # reads the token's position and its cos/sin table rows (8 + 2048 B per token)
+    del kv, ik
+    raw, rik = synth.raw_kv_tokens(1, T, device=device)
+    cos, sin = synth.rope_tables(T, device=device)
+    pos = torch.arange(T, dtype=torch.int64, device=device)
+    for ratio in (1, 2):
+        ms = 0.0
+        for i in range(warmup + steps):
+            flush.fill_(i)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            csa2.csa2_pack_kv_normed(raw, rik, ratio, pos, cos, sin, kvp, ikp)
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= warmup:
+                ms += e0.elapsed_time(e1)
+        ms /= steps
+        nbytes = T * (1280 + 8 + 2048) + (T // ratio) * 356
+        res[f"normed {ratio}:1"] = {"GB/s": round(nbytes / (ms * 1e-3) / 1e9, 1), "us": round(ms * 1e3, 1),
+                                    "bytes": nbytes}
+    del raw, rik, cos, sin, pos, kvp, ikp, flush
     torch.cuda.empty_cache()
     return res
 

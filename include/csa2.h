@@ -110,6 +110,36 @@ csa2_status csa2_pack_kv(const void* kv, const void* ik, int64_t T, int ratio,
                          uint8_t* ik_pool, uint32_t* dev_status, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * a1 producer: RMSNorm + rotary encoding + pack (P3 §4비트로 적어도 되는 이유: cached
+ * values are normalised and rotated before caching, which bounds them by sqrt(512);
+ * the pages give no formula, so the operations below are this library's reading).
+ *
+ *   kv   bf16 [T][512]  raw (not yet normalised) main-KV tokens
+ *   ik   bf16 [T][128]  indexer-key tokens (packed as csa2_pack_kv packs them)
+ *   pos  int64 [T]      row of the rotation tables for each token (its position)
+ *   rope_cos, rope_sin  fp32 [n_pos][256]: cosine and sine for channel pair i at each row
+ *   gamma fp32 [512] per-channel gain, or NULL for none;  eps >= 0
+ *   T, ratio, dst_entry, pool_entries, kv_pool, ik_pool: as csa2_pack_kv
+ *
+ * Per token, every operation rounded once in fp32 (no fused multiply-add):
+ *   S = sum of x_c^2, summed by halving within each 16-channel block (element i += i+8,
+ *       then +4, +2, +1), then by halving over the 32 block sums (+16, +8, +4, +2, +1);
+ *   r = 1 / sqrt(S / 512 + eps) (the add, the square root and the reciprocal each
+ *       correctly rounded);  n_c = x_c * r, then n_c * gamma_c;
+ *   channel pairs (2i, 2i+1) rotated with c = rope_cos[pos][i], s = rope_sin[pos][i]:
+ *       y_2i = n_2i c - n_2i+1 s,  y_2i+1 = n_2i s + n_2i+1 c;
+ *   y rounded to bf16 (nearest, ties to even), then encoded exactly as csa2_pack_kv
+ *   encodes a bf16 token (ratio 2: each token at its own position, then the pair mean).
+ * Output is bit-exact with that definition.  An entry whose destination or either
+ * position is out of range is skipped and flags CSA2_DEV_BAD_INDEX.
+ * --------------------------------------------------------------------------------- */
+csa2_status csa2_pack_kv_normed(const void* kv, const void* ik, int64_t T, int ratio, const int64_t* pos,
+                                const float* rope_cos, const float* rope_sin, int64_t n_pos,
+                                const float* gamma, float eps, const int64_t* dst_entry,
+                                int64_t pool_entries, uint8_t* kv_pool, uint8_t* ik_pool,
+                                uint32_t* dev_status, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * a2+a3  Full-mode indexer scan with flat Top-K (P1 §무엇과 다른가: a Full layer scores
  * the whole causally visible range with its own indexer Q and picks Top-K).
  *

@@ -47,6 +47,8 @@ def lib():
         L.csa2_version.restype = I32
         L.csa2_pack_kv.restype = I32
         L.csa2_pack_kv.argtypes = [P, P, I64, I32, P, I64, P, P, P, P]
+        L.csa2_pack_kv_normed.restype = I32
+        L.csa2_pack_kv_normed.argtypes = [P, P, I64, I32, P, P, P, I64, P, F32, P, I64, P, P, P, P]
         L.csa2_index_full_workspace_size.restype = SZ
         L.csa2_index_full_workspace_size.argtypes = [I32, I32, I32, I32, I64]
         L.csa2_index_full.restype = I32
@@ -162,6 +164,37 @@ def csa2_pack_kv(kv, ik, ratio, kv_pool, ik_pool, dst_entry=None, dev_status=Non
     _check(lib().csa2_pack_kv(_ptr(kv), _ptr(ik), T, int(ratio), _ptr(dst_entry), kv_pool.shape[0],
                               _ptr(kv_pool), _ptr(ik_pool), _ptr(dev_status), _stream(stream)),
            "csa2_pack_kv")
+
+
+def csa2_pack_kv_normed(kv, ik, ratio, pos, rope_cos, rope_sin, kv_pool, ik_pool, gamma=None, eps=1e-6,
+                        dst_entry=None, dev_status=None, stream=None):
+    """Raw kv bf16 [T,512] normalised and rotated (pos int64 [T] into rope_cos / rope_sin
+    f32 [n_pos,256]; gamma f32 [512] or None), then packed like csa2_pack_kv."""
+    _shape(kv, (None, D), "kv")
+    T = kv.shape[0]
+    _shape(ik, (T, DI), "ik")
+    _shape(pos, (T,), "pos")
+    _shape(rope_cos, (None, D // 2), "rope_cos")
+    _shape(rope_sin, (rope_cos.shape[0], D // 2), "rope_sin")
+    _shape(gamma, (D,), "gamma")
+    _shape(kv_pool, (None, KV_BYTES), "kv_pool")
+    _shape(ik_pool, (kv_pool.shape[0], IK_BYTES), "ik_pool")
+    if dst_entry is not None and (dst_entry.dim() != 1 or dst_entry.numel() != T // max(int(ratio), 1)):
+        raise ValueError("dst_entry must hold one slot per new entry (T // ratio)")
+    _need(kv, torch.bfloat16, "kv", 2)
+    _need(ik, torch.bfloat16, "ik", 2)
+    _need(pos, torch.int64, "pos", 1)
+    _need(rope_cos, torch.float32, "rope_cos", 2)
+    _need(rope_sin, torch.float32, "rope_sin", 2)
+    _need(gamma, torch.float32, "gamma", 1)
+    _need(kv_pool, torch.uint8, "kv_pool", 2)
+    _need(ik_pool, torch.uint8, "ik_pool", 2)
+    _need(dst_entry, torch.int64, "dst_entry", 1)
+    _status(dev_status)
+    _check(lib().csa2_pack_kv_normed(_ptr(kv), _ptr(ik), T, int(ratio), _ptr(pos), _ptr(rope_cos), _ptr(rope_sin),
+                                     rope_cos.shape[0], _ptr(gamma), float(eps), _ptr(dst_entry), kv_pool.shape[0],
+                                     _ptr(kv_pool), _ptr(ik_pool), _ptr(dev_status), _stream(stream)),
+           "csa2_pack_kv_normed")
 
 
 def _query_dims(q, w, ik_pool, seq_base, n_vis):

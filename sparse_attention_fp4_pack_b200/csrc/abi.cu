@@ -10,6 +10,10 @@ namespace csa2 {
 cudaError_t launch_pack_kv(const void* kv, const void* ik, int64_t T, int ratio,
                            const int64_t* dst, int64_t pool_entries, uint8_t* kv_pool,
                            uint8_t* ik_pool, uint32_t* status, cudaStream_t stream, int num_sms);
+cudaError_t launch_pack_kv_normed(const void* kv, const void* ik, int64_t T, int ratio, const int64_t* pos,
+                                  const float* rope_cos, const float* rope_sin, int64_t n_pos, const float* gamma,
+                                  float eps, const int64_t* dst, int64_t pool_entries, uint8_t* kv_pool,
+                                  uint8_t* ik_pool, uint32_t* status, cudaStream_t stream, int num_sms);
 cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t* ik_pool,
                          int64_t pool_entries, const int64_t* seq_base, const int32_t* n_vis,
                          const int32_t* blocks, int B, int Q, int HI, int n_blocks, int block,
@@ -109,6 +113,26 @@ csa2_status csa2_pack_kv(const void* kv, const void* ik, int64_t T, int ratio,
   if (dev_status && !aligned(dev_status, 4)) return CSA2_ERR_INVALID_ARG;
   return launched(csa2::launch_pack_kv(kv, ik, T, ratio, dst_entry, pool_entries, kv_pool,
                                        ik_pool, dev_status, stream, current_sm_count()));
+}
+
+csa2_status csa2_pack_kv_normed(const void* kv, const void* ik, int64_t T, int ratio, const int64_t* pos,
+                                const float* rope_cos, const float* rope_sin, int64_t n_pos, const float* gamma,
+                                float eps, const int64_t* dst_entry, int64_t pool_entries, uint8_t* kv_pool,
+                                uint8_t* ik_pool, uint32_t* dev_status, cudaStream_t stream) {
+  if (ratio != 1 && ratio != 2) return CSA2_ERR_UNSUPPORTED;
+  if (T < 0 || pool_entries < 0 || n_pos < 0 || T % ratio != 0) return CSA2_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !std::isfinite(eps)) return CSA2_ERR_INVALID_ARG;
+  if (T == 0) return CSA2_OK;
+  if (!kv || !ik || !pos || !rope_cos || !rope_sin || !kv_pool || !ik_pool) return CSA2_ERR_INVALID_ARG;
+  if (!aligned(kv, 16) || !aligned(ik, 16) || !aligned(kv_pool, 16) || !aligned(ik_pool, 16) ||
+      !aligned(pos, 8) || !aligned(rope_cos, 16) || !aligned(rope_sin, 16) || (gamma && !aligned(gamma, 16)))
+    return CSA2_ERR_INVALID_ARG;
+  if (dst_entry && !aligned(dst_entry, 8)) return CSA2_ERR_INVALID_ARG;
+  if (!dst_entry && T / ratio > pool_entries) return CSA2_ERR_INVALID_ARG;
+  if (dev_status && !aligned(dev_status, 4)) return CSA2_ERR_INVALID_ARG;
+  return launched(csa2::launch_pack_kv_normed(kv, ik, T, ratio, pos, rope_cos, rope_sin, n_pos, gamma, eps,
+                                              dst_entry, pool_entries, kv_pool, ik_pool, dev_status, stream,
+                                              current_sm_count()));
 }
 
 size_t csa2_index_full_workspace_size(int B, int Q, int HI, int K, int64_t max_n_vis) {

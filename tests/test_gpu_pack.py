@@ -196,3 +196,88 @@ def test_full_size_pack_sampled(orc, ratio):
     s_t = torch.from_numpy(sample).cuda()
     assert np.array_equal(np_u8(kvp[s_t]), o_kv)
     assert np.array_equal(np_u8(ikp[s_t]), o_ik)
+
+
+# ---- producer: RMSNorm + rotation + pack, bit-exact against the oracle -----------------------
+def _normed(kv, ik, ratio, pos, cos, sin, gamma=None, eps=1e-6, dst=None, pool=None):
+    E = kv.shape[0] // ratio
+    P = pool if pool is not None else E
+    kvp = torch.zeros(P, 288, dtype=torch.uint8, device="cuda")
+    ikp = torch.zeros(P, 68, dtype=torch.uint8, device="cuda")
+    st = csa2.status_word()
+    csa2.csa2_pack_kv_normed(kv.cuda(), ik.cuda(), ratio, torch.as_tensor(pos, dtype=torch.int64).cuda(), cos.cuda(),
+                             sin.cuda(), kvp, ikp, gamma=None if gamma is None else gamma.cuda(), eps=eps,
+                             dst_entry=None if dst is None else torch.as_tensor(dst, dtype=torch.int64).cuda(),
+                             dev_status=st)
+    torch.cuda.synchronize()
+    return np_u8(kvp), np_u8(ikp), int(st.item())
+
+
+@pytest.mark.parametrize("ratio,with_gain", [(1, False), (1, True), (2, False), (2, True)])
+def test_normed_pack_random(orc, ratio, with_gain):
+    """Raw tokens over eight binades of scale with heavy tails, random positions in a
+    4096-row table, with and without a per-channel gain: bit-exact entries."""
+    T = 6002
+    kv, ik = synth.raw_kv_tokens(200 + ratio, T)
+    cos, sin = synth.rope_tables(4096)
+    pos = torch.randint(0, 4096, (T,), generator=torch.Generator().manual_seed(7 + ratio)).numpy()
+    gamma = (torch.rand(512, generator=torch.Generator().manual_seed(9)) * 1.5 + 0.25) if with_gain else None
+    g_kv, g_ik, st = _normed(kv, ik, ratio, pos, cos, sin, gamma=gamma)
+    assert st == 0
+    o_kv, o_ik, bad = orc.pack_kv_normed(bf16_bits(kv), bf16_bits(ik), ratio, pos, cos.numpy(), sin.numpy(),
+                                         gamma=None if gamma is None else gamma.numpy())
+    assert not bad
+    assert np.array_equal(g_ik, o_ik)
+    mism = np.nonzero((g_kv != o_kv).any(axis=1))[0]
+    assert mism.size == 0, f"{mism.size} entries differ, first {mism[:5]}"
+
+
+def test_normed_pack_edges(orc):
+    """Constant rows, zero rows (eps keeps them finite), a quarter-turn table, scatter to
+    chosen slots, and an out-of-range position: the entry is skipped and flagged."""
+    T = 64
+    rows = torch.zeros(T, 512)
+    rows[0:8] = 3.0
+    rows[8:16] = -0.0078125
+    rows[16:24] = 0.0
+    rows[24:] = torch.randn(40, 512, generator=torch.Generator().manual_seed(3)) * 100
+    kv = rows.to(torch.bfloat16)
+    ik = torch.randn(T, 128, generator=torch.Generator().manual_seed(4)).to(torch.bfloat16)
+    cos, sin = synth.rope_tables(8)
+    cos[0], sin[0] = 0.0, 1.0  # row 0: a quarter turn
+    pos = np.arange(T, dtype=np.int64) % 8
+    dst = np.arange(T, dtype=np.int64)[::-1].copy()
+    g_kv, g_ik, st = _normed(kv, ik, 1, pos, cos, sin, eps=1e-5, dst=dst)
+    o_kv, o_ik, _ = orc.pack_kv_normed(bf16_bits(kv), bf16_bits(ik), 1, pos, cos.numpy(), sin.numpy(), eps=1e-5)
+    assert st == 0
+    assert np.array_equal(g_kv[::-1], o_kv) and np.array_equal(g_ik[::-1], o_ik)
+    pos_bad = pos.copy()
+    pos_bad[10] = 8
+    g_kv, g_ik, st = _normed(kv, ik, 2, pos_bad, cos, sin, eps=1e-5)
+    o_kv, o_ik, bad = orc.pack_kv_normed(bf16_bits(kv), bf16_bits(ik), 2, pos_bad, cos.numpy(), sin.numpy(), eps=1e-5)
+    assert bad and (st & csa2.DEV_BAD_INDEX)
+    assert not g_kv[5].any() and np.array_equal(g_kv, o_kv) and np.array_equal(g_ik, o_ik)
+
+
+def test_normed_pack_full_size_sampled(orc):
+    """2^20 raw tokens (the pack workload's size) at positions 0..2^20-1: sampled entries
+    equal the oracle's producer on those tokens."""
+    T = 1 << 20
+    kv, ik = synth.raw_kv_tokens(210, T, device="cuda")
+    cos, sin = synth.rope_tables(T, device="cuda")
+    pos = torch.arange(T, dtype=torch.int64, device="cuda")
+    for ratio in (1, 2):
+        E = T // ratio
+        kvp = torch.zeros(E, 288, dtype=torch.uint8, device="cuda")
+        ikp = torch.zeros(E, 68, dtype=torch.uint8, device="cuda")
+        st = csa2.status_word()
+        csa2.csa2_pack_kv_normed(kv, ik, ratio, pos, cos, sin, kvp, ikp, dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        sample = np.random.default_rng(ratio).choice(E, 300, replace=False)
+        toks = np.stack([np.arange(j * ratio, (j + 1) * ratio) for j in sample]).reshape(-1)
+        t = torch.from_numpy(toks).cuda()
+        o_kv, o_ik, _ = orc.pack_kv_normed(bf16_bits(kv[t]), bf16_bits(ik[t]), ratio, toks, cos.cpu().numpy(),
+                                           sin.cpu().numpy())
+        assert np.array_equal(np_u8(kvp[torch.from_numpy(sample).cuda()]), o_kv)
+        assert np.array_equal(np_u8(ikp[torch.from_numpy(sample).cuda()]), o_ik)
