@@ -43,6 +43,7 @@ WORKLOAD_TEXT = {
                 "layer, H=64 x 512, HI=8 x 128, W=128",
     "verify": "multi-query verify: B=8 x 128K entries (2:1 of 256K tokens), Q=64 drafts, Full + Reuse layer",
     "tiny": "tiny decode: 1 sequence, 4096 entries, H=16, HI=4, Top-512, W=128",
+    "hier256k": "hierarchical decoder at 256K context: B=4 x 262,144 FP4 entries, as hier1m (profiling size)",
     "prefill": "chunked prefill: 1 sequence of 256K tokens at 2:1 (128K entries), a chunk of 1024 new "
                "tokens as queries (own causal limits), Full + Reuse layer, H=64 x 512, HI=8 x 128, Top-512",
 }

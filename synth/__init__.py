@@ -16,6 +16,8 @@ Workload shapes follow the five decode configurations of the build's target:
   verify     B=8, 2^18 tokens at 2:1 = 2^17 entries, Q=64 drafts          (seed 4)
   prefill    B=1, 2^18 tokens at 2:1 = 2^17 entries, a chunk of Q=1024    (seed 5)
              new tokens, each a query with its own causal limit
+  hier256k   hier1m's decoder at B=4 x 2^18 entries (a small case with the   (seed 6)
+             same per-layer launch shapes, for profiling)
 """
 from dataclasses import dataclass, field
 import zlib
@@ -153,6 +155,9 @@ def workload(name: str) -> DecodeWorkload:
     if name == "verify":
         return DecodeWorkload("verify", 4, B=8, Q=64, H=64, HI=8, K=512, window=128, ratio=2,
                               lengths=[1 << 17] * 8, new_tokens=64)
+    if name == "hier256k":  # the hierarchical decoder at a quarter of the context (profiling)
+        return DecodeWorkload("hier256k", 6, B=4, Q=1, H=64, HI=8, K=512, window=128, ratio=1,
+                              lengths=[1 << 18] * 4, hier=True, n_layers=20)
     if name == "prefill":
         return DecodeWorkload("prefill", 5, B=1, Q=1024, H=64, HI=8, K=512, window=128, ratio=2,
                               lengths=[1 << 17], new_tokens=1024)
