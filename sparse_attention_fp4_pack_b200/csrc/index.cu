@@ -1254,8 +1254,16 @@ cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t
     e = launch_chained(select_kernel<2>, dim3((unsigned)s.csize, (unsigned)BQ), dim3(kSelThreads),
                        SelShape<2>::kSmem, stream, (unsigned)s.csize, s);
   } else {
-    const int64_t c = (items + SelShape<4>::kChunk - 1) / SelShape<4>::kChunk;
-    s.csize = (int)(c < 1 ? 1 : (c > kMaxCluster ? kMaxCluster : c));
+    // one CTA per 16,384 keys, up to a cluster of 8; when the queries alone fill the GPU
+    // for more than two waves, fewer CTAs per query (each walks several chunks), since a
+    // wide cluster then only adds waves and cluster barriers
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int64_t c = (items + SelShape<4>::kChunk - 1) / SelShape<4>::kChunk;
+    c = c < 1 ? 1 : (c > kMaxCluster ? kMaxCluster : c);
+    const int64_t fit = (2 * (int64_t)sms) / (BQ > 0 ? BQ : 1);  // CTAs per query in two waves
+    if (c > fit) c = fit < 1 ? 1 : (fit >= 8 ? 8 : (fit >= 4 ? 4 : (fit >= 2 ? 2 : 1)));
+    s.csize = (int)c;
     e = cudaFuncSetAttribute(select_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, SelShape<4>::kSmem);
     if (e != cudaSuccess) return e;
     e = launch_chained(select_kernel<4>, dim3((unsigned)s.csize, (unsigned)BQ), dim3(kSelThreads),
