@@ -298,8 +298,11 @@ CALL_KERNELS = {
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the call's
 # dominant kernel, from an ncu capture of that kernel as it is now, per workload; a kernel
-# that changes drops out of this table until it is captured again.
-NCU_DRAM_BYTES_PER_LAUNCH = {}
+# that changes drops out of this table until it is captured again.  The attention launch
+# of hier1m was captured on hier256k, whose attention launch is the same (4 queries, 512
+# entries + 128 window tokens each, the same grid): its traffic does not depend on the
+# context length.
+NCU_DRAM_BYTES_PER_LAUNCH = {("hier1m", "attn"): 1657856}
 
 
 def call_rooflines(wl, per_call, counts, steps, peaks):

@@ -314,6 +314,9 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t caddr, uint32_t x, uint32
                : "memory");
 }
 
+// NQ: the products' N (the CTA's heads rounded up to 16, 32 or 64), a template parameter
+// so each launch runs one compact code path.
+template <int NQ>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
   chain_enter();
   extern __shared__ uint8_t smem_raw[];
@@ -344,7 +347,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
   const int H = a.H;                                 // heads of the query (output layout)
   const int h_base = (blockIdx.y % a.hgroups) * a.hg_size;
   const int NH = min(a.hg_size, H - h_base);         // heads of this cluster, rows 0..NH-1
-  const int NQ = NH <= 16 ? 16 : (NH <= 32 ? 32 : kHeadsPad);  // the products' N
   const int T = rank < a.n_tiles ? (a.n_tiles - 1 - rank) / C + 1 : 0;  // tiles rank + k C
   const int r = tid >> 1, hf = tid & 1;              // worker: tile row and half
   const int64_t base = a.seq_base[b];
@@ -797,11 +799,11 @@ cudaError_t launch_sparse_attn(const float* q, const uint8_t* kv_pool, int64_t p
     }
   }
   a.hg_size = H / a.hgroups;
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  const int nq = a.hg_size <= 16 ? 16 : (a.hg_size <= 32 ? 32 : kHeadsPad);
+  auto* fn = nq == 16 ? attn_kernel<16> : (nq == 32 ? attn_kernel<32> : attn_kernel<kHeadsPad>);
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
-  if (e != cudaSuccess) return e;
-  e = launch_chained(attn_kernel, dim3((unsigned)a.csize, (unsigned)(BQ * a.hgroups)), dim3(kAttnThreads), kSmemBytes,
+  e = launch_chained(fn, dim3((unsigned)a.csize, (unsigned)(BQ * a.hgroups)), dim3(kAttnThreads), kSmemBytes,
                      stream, a.csize > 1 ? (unsigned)a.csize : 0u, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
