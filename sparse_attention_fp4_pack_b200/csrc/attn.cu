@@ -318,7 +318,7 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t caddr, uint32_t x, uint32
 // so each launch runs one compact code path.
 template <int NQ>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
-  chain_enter();
+  chain_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = tc::align_smem_1024(smem_raw);
   uint8_t* Ks = sm + kOffK;
@@ -349,10 +349,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
   const int NH = min(a.hg_size, H - h_base);         // heads of this cluster, rows 0..NH-1
   const int T = rank < a.n_tiles ? (a.n_tiles - 1 - rank) / C + 1 : 0;  // tiles rank + k C
   const int r = tid >> 1, hf = tid & 1;              // worker: tile row and half
-  const int64_t base = a.seq_base[b];
-  const int64_t tq = a.q_pos[bq];
-  const int64_t sws = a.S_w > 0 ? a.swa_start[b] : 0;
 
+  // set-up that touches no global memory runs while the predecessor finishes
   if (tid == 0) {
     tc::mbar_init(bar_q, 1);
     tc::mbar_init(bar_ka, kWorkers);
@@ -360,6 +358,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
     tc::mbar_init(bar_s, 1);
     tc::mbar_init(bar_p, kWorkers);
     tc::mbar_init(bar_pv, 1);
+  }
+  if (tid < kHeadsPad) {
+    m_run[tid] = -INFINITY;
+    l_run[tid] = 0.0f;
+  }
+  if (warp == 0) tc::tmem_alloc(tc::smem_u32(tmem_slot), kTmemCols);
+  chain_wait();
+  const int64_t base = a.seq_base[b];
+  const int64_t tq = a.q_pos[bq];
+  const int64_t sws = a.S_w > 0 ? a.swa_start[b] : 0;
+
+  if (tid == 0) {
     const uint32_t bytes = (uint32_t)NH * kD * 4;
     tc::mbar_arrive_expect_tx(bar_q, bytes);
     const uint8_t* src = reinterpret_cast<const uint8_t*>(a.q + ((int64_t)bq * H + h_base) * kD);
@@ -381,11 +391,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
     }
     tc::cp_async_commit();
   }
-  if (tid < kHeadsPad) {
-    m_run[tid] = -INFINITY;
-    l_run[tid] = 0.0f;
-  }
-  if (warp == 0) tc::tmem_alloc(tc::smem_u32(tmem_slot), kTmemCols);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();

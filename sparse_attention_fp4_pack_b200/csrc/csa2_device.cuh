@@ -29,6 +29,12 @@ __device__ __forceinline__ void chain_enter() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
+// The two halves of chain_enter, for kernels that first do set-up touching no global
+// memory (barrier initialisation, tensor-memory allocation) while the predecessor runs.
+__device__ __forceinline__ void chain_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void chain_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // Host side: launch `kernel` with programmatic stream serialization, plus a cluster of
 // cluster_x CTAs along x when cluster_x > 0.

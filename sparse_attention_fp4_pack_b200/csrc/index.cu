@@ -107,7 +107,7 @@ __device__ __forceinline__ uint2 codes_to_u8(uint32_t w) {
 // tile, staged by cp.async one tile ahead).
 template <int HIPAD>
 __global__ void __launch_bounds__(kScanThreads) reindex_scan_kernel(ScanArgs a) {
-  chain_enter();
+  chain_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = tc::align_smem_1024(smem_raw);
   uint8_t* As = sm;                                   // [128 rows x 128 B], 128 B swizzle
@@ -127,6 +127,10 @@ __global__ void __launch_bounds__(kScanThreads) reindex_scan_kernel(ScanArgs a) 
   if (item0 >= limit) return;
   const int64_t left_tiles = (limit - item0 + kRows - 1) / kRows;
   const int ntiles = (int)(left_tiles < a.tiles_per_cta ? left_tiles : a.tiles_per_cta);
+  // set-up that touches no global memory runs while the predecessor finishes
+  if (warp == 0) tc::tmem_alloc(tc::smem_u32(tmem_slot), a.tmem_cols);
+  if (tid == 32) tc::mbar_init(tc::smem_u32(mbar), 1);
+  chain_wait();
   const int64_t nvis = valid_count(a, b, bq, blockIdx.x == 0);  // 0 if the count is bad
 
   const uint8_t* seq = a.ik_pool + a.seq_base[b] * kIkBytes;
@@ -176,8 +180,6 @@ __global__ void __launch_bounds__(kScanThreads) reindex_scan_kernel(ScanArgs a) 
     }
   }
   load_tile(0);  // the first tile's copies overlap the set-up below
-  if (warp == 0) tc::tmem_alloc(tc::smem_u32(tmem_slot), a.tmem_cols);
-  if (tid == 32) tc::mbar_init(tc::smem_u32(mbar), 1);
 
   // ---- B operand: four int8 limbs of every head, plus epilogue constants ----------------
 #pragma unroll
@@ -764,7 +766,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
   constexpr int kSelChunk = SelShape<PS>::kChunk;
   constexpr int kKeyRow = SelShape<PS>::kKeyRow;
   constexpr int kKeyWords = SelShape<PS>::kKeyWords;
-  chain_enter();
+  chain_launch_dependents();
   // phase: started
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
@@ -784,6 +786,9 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
   const int bq = blockIdx.y;
   const int b = bq / a.Q;
   const int K = a.K;
+  for (int i = tid; i < kSubWords / 4; i += kSelThreads)  // counters start at zero
+    reinterpret_cast<uint4*>(sub)[i] = make_uint4(0u, 0u, 0u, 0u);
+  chain_wait();
   int32_t* out = a.out_idx + (int64_t)bq * K;
   float* out_s = a.out_score ? a.out_score + (int64_t)bq * K : nullptr;
   // shared::cluster address of `src` in CTA r
@@ -810,8 +815,6 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
 
   if (a.mode == kReindex)  // read back with the labels of the selected items (barriers follow)
     for (int i = tid; i < a.n_blocks; i += kSelThreads) blk[i] = a.blocks[(int64_t)bq * a.n_blocks + i];
-  for (int i = tid; i < kSubWords / 4; i += kSelThreads)  // counters start at zero
-    reinterpret_cast<uint4*>(sub)[i] = make_uint4(0u, 0u, 0u, 0u);
 
   // chunk ch of the slice -> ks (item lo + ch*kSelChunk + kPer*t + e is key e of thread t; 0 past hi)
   const uint32_t* mk = ks + tid * kKeyRow;
