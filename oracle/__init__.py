@@ -53,6 +53,8 @@ def lib():
         L.orc_reindex.argtypes = [c_p, c_p, c_p, c_p, c_p, c_p, i32, i32, i32, i32, i32, i32, c_p, c_p]
         L.orc_sparse_attn.argtypes = [c_p, c_p, c_p, c_p, i32, c_p, i32, c_p, c_p, i32, i32, i32, i32,
                                       dbl, c_p, c_p]
+        L.orc_topk_labeled.argtypes = [c_p, c_p, i64, i32, c_p, c_p]
+        L.orc_attn_combine.argtypes = [c_p, c_p, i32, i64, c_p, c_p]
         _lib = L
     return _lib
 
@@ -242,4 +244,31 @@ def sparse_attn(q, kv_pool, seq_base, topk_, swa, swa_start, q_pos, sm_scale, wi
     lse = np.zeros((B, Q, H), np.float64)
     lib().orc_sparse_attn(_p(q), _p(pool), _p(sb), _p(tk), K, _p(sw), S_w, _p(ss), _p(qp), window,
                           B, Q, H, float(sm_scale), _p(out), _p(lse))
+    return out, lse
+
+
+# ---- context-parallel decomposition ---------------------------------------------------
+def topk_labeled(scores, labels, K):
+    """Top-K of labeled candidates (descending score, then ascending label): scores [n]
+    float64, labels [n] int64 -> (labels [K] int32 with -1 past n, scores [K] float64)."""
+    s = _c(scores, np.float64)
+    lab = _c(labels, np.int64)
+    assert s.shape == lab.shape and s.ndim == 1
+    idx = np.zeros(K, np.int32)
+    sc = np.zeros(K, np.float64)
+    lib().orc_topk_labeled(_p(s), _p(lab), s.shape[0], K, _p(idx), _p(sc))
+    return idx, sc
+
+
+def attn_combine(out_parts, lse_parts):
+    """Attention over a union of disjoint key sets from the parts' results:
+    out_parts [C, ..., 512], lse_parts [C, ...] -> (out [..., 512], lse [...]) float64."""
+    o = _c(out_parts, np.float64)
+    l = _c(lse_parts, np.float64)
+    C = o.shape[0]
+    assert o.shape[:-1] == l.shape and o.shape[-1] == 512
+    N = int(np.prod(l.shape[1:], dtype=np.int64))
+    out = np.zeros(l.shape[1:] + (512,), np.float64)
+    lse = np.zeros(l.shape[1:], np.float64)
+    lib().orc_attn_combine(_p(o), _p(l), C, N, _p(out), _p(lse))
     return out, lse

@@ -541,3 +541,47 @@ void orc_sparse_attn(const float* q /*[B][Q][H][512]*/, const uint8_t* kv_pool, 
     free(keys);
   }
 }
+
+/* ------------------------------------------------------------------------------------
+ * Context-parallel decode: the entries of one sequence split over C parts (P1 §무엇과
+ * 다른가: a Full layer's Top-K is taken over everything the query sees; P3 §전역
+ * 어텐션과 지역 어텐션: one softmax over the selected entries together with the window).
+ * The pages describe a single device; splitting is this oracle's reading of how the same
+ * results decompose, and each function below is the plain definition of one step.
+ * ------------------------------------------------------------------------------------ */
+
+/* Top-K of n labeled candidates: the order above (descending score, then ascending label)
+ * over (scores[i], labels[i]); -1 fills the slots past n.  With every part's own Top-K as
+ * the candidates, this is the Top-K of the union. */
+void orc_topk_labeled(const double* scores, const int64_t* labels, int64_t n, int K, int32_t* idx_out,
+                      double* score_out) {
+  topk_labeled(scores, labels, n, K, idx_out, score_out);
+}
+
+/* Attention over the union of C disjoint key sets from each set's normalised output and
+ * log-sum-exp of its logits: with M = max_c lse_c,
+ *   lse = M + log(sum_c exp(lse_c - M)),   out = sum_c exp(lse_c - lse) * out_c.
+ * A part with lse_c = -inf (no keys) contributes nothing; all parts empty gives out = 0,
+ * lse = -inf.  out_parts [C][N][512], lse_parts [C][N]; out [N][512], lse [N]. */
+void orc_attn_combine(const double* out_parts, const double* lse_parts, int C, int64_t N, double* out,
+                      double* lse) {
+  for (int64_t r = 0; r < N; ++r) {
+    double mx = -HUGE_VAL;
+    for (int c = 0; c < C; ++c)
+      if (lse_parts[(int64_t)c * N + r] > mx) mx = lse_parts[(int64_t)c * N + r];
+    double* o = out + r * ORC_D;
+    for (int d = 0; d < ORC_D; ++d) o[d] = 0.0;
+    if (mx == -HUGE_VAL) {
+      lse[r] = -HUGE_VAL;
+      continue;
+    }
+    double l = 0.0;
+    for (int c = 0; c < C; ++c) {
+      double wc = exp(lse_parts[(int64_t)c * N + r] - mx);
+      l += wc;
+      for (int d = 0; d < ORC_D; ++d) o[d] += wc * out_parts[((int64_t)c * N + r) * ORC_D + d];
+    }
+    for (int d = 0; d < ORC_D; ++d) o[d] /= l;
+    lse[r] = mx + log(l);
+  }
+}

@@ -109,6 +109,15 @@ MUTANTS = [
      "rope_cos + (p + 1) * (ORC_D / 2), rope_sin + (p + 1) * (ORC_D / 2)"),
     ("bf16 rounding truncates", "return (uint16_t)((u + 0x7FFFu + lsb) >> 16);", "return (uint16_t)(u >> 16);"),
     ("bad position keeps its entry", "    if (zero) {\n      memset(kv_out", "    if (0) {\n      memset(kv_out"),
+    # context-parallel decomposition
+    ("labeled top-k drops the labels", "p[i].i = labels ? labels[i] : i;", "p[i].i = i;"),
+    ("combine without the max shift", "double wc = exp(lse_parts[(int64_t)c * N + r] - mx);",
+     "double wc = exp(lse_parts[(int64_t)c * N + r]);"),
+    ("combine unnormalised", "for (int d = 0; d < ORC_D; ++d) o[d] /= l;\n    lse[r] = mx + log(l);",
+     "lse[r] = mx + log(l);"),
+    ("combine lse without the max", "lse[r] = mx + log(l);", "lse[r] = log(l);"),
+    ("combine skips the last part", "for (int c = 0; c < C; ++c) {\n      double wc",
+     "for (int c = 0; c + 1 < C; ++c) {\n      double wc"),
 ]
 
 

@@ -134,3 +134,49 @@ def test_reuse_and_multi_query_batching(orc):
         o1, l1 = orc.sparse_attn(q[:, i:i + 1], kvp, np.zeros(1, np.int64), topk[:, i:i + 1], swa,
                                  start, q_pos[:, i:i + 1], SM)
         assert np.array_equal(out[:, i:i + 1], o1) and np.array_equal(lse[:, i:i + 1], l1)
+
+
+def test_combine_of_parts_equals_attention_over_union(orc):
+    """Attention over disjoint key sets, combined from each set's output and log-sum-exp,
+    equals attention over their union: Top-K entries split three ways (one part also holds
+    the window, one part is empty)."""
+    kvp, _ = _pool(7, 96)
+    rng = np.random.default_rng(5)
+    B, Q, H, S_w = 2, 2, 4, 24
+    q = (3 * rng.standard_normal((B, Q, H, 512))).astype(np.float32)
+    topk = np.stack([np.stack([rng.choice(90, 40, replace=False) for _ in range(Q)]) for _ in range(B)])
+    topk = topk.astype(np.int32)
+    seq_base = np.zeros(B, np.int64)
+    swa = synth.swa_window(3, B, S_w).numpy()
+    swa_start = np.array([100, 200], np.int64)
+    q_pos = np.array([[110, 123], [205, 223]], np.int64)
+    whole_o, whole_l = orc.sparse_attn(q, kvp, seq_base, topk, swa, swa_start, q_pos, SM)
+    parts = []
+    for lo, hi, win in ((0, 17, False), (17, 40, True), (40, 40, False)):
+        t = np.full_like(topk, -1)
+        t[..., :hi - lo] = topk[..., lo:hi]
+        parts.append(orc.sparse_attn(q, kvp, seq_base, t, swa if win else None, swa_start, q_pos, SM))
+    o, l = orc.attn_combine(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
+    assert np.isneginf(parts[2][1]).all()
+    assert np.allclose(o, whole_o, rtol=1e-12, atol=1e-12)
+    assert np.allclose(l, whole_l, rtol=1e-12, atol=1e-12)
+
+
+def test_combine_closed_forms(orc):
+    """Two parts with equal log-sum-exp: the mean, lse + log 2.  A part with lse = -inf adds
+    nothing; all parts empty gives out = 0, lse = -inf."""
+    rng = np.random.default_rng(6)
+    a = rng.standard_normal((1, 512))
+    b = rng.standard_normal((1, 512))
+    o, l = orc.attn_combine(np.stack([a, b]), np.array([[0.75], [0.75]]))
+    assert np.allclose(o, (a + b) / 2, rtol=1e-15, atol=1e-15)
+    assert abs(l[0] - (0.75 + math.log(2))) < 1e-15
+    # weights e^1 : e^3 -> 1/(1+e^2), e^2/(1+e^2)
+    o, l = orc.attn_combine(np.stack([a, b]), np.array([[1.0], [3.0]]))
+    w1 = 1 / (1 + math.e ** 2)
+    assert np.allclose(o, w1 * a + (1 - w1) * b, rtol=1e-14, atol=1e-14)
+    assert abs(l[0] - math.log(math.e + math.e ** 3)) < 1e-14
+    o, l = orc.attn_combine(np.stack([a, 7 * b]), np.array([[2.5], [-np.inf]]))
+    assert np.array_equal(o, a) and l[0] == 2.5
+    o, l = orc.attn_combine(np.stack([a, b]), np.full((2, 1), -np.inf))
+    assert (o == 0).all() and np.isneginf(l).all()

@@ -160,3 +160,39 @@ def test_reindex_skips_empty_slots_and_invisible(orc):
     sc = orc.index_scores(q[0, 0], w[0, 0], ik[:n])
     want = sorted(cand, key=lambda j: (-sc[j], j))
     assert t[0, 0, :13].tolist() == want and (t[0, 0, 13:] == -1).all()
+
+
+def test_topk_labeled_brute_force(orc):
+    """Labeled Top-K: descending score, then ascending label, over arbitrary distinct labels
+    (shuffled, far apart); -1 past the candidates."""
+    rng = np.random.default_rng(11)
+    n = 700
+    s = np.round(rng.standard_normal(n), 1)               # many exact ties
+    lab = rng.permutation(n).astype(np.int64) * 977 + 13   # distinct, not in slot order
+    idx, sc = orc.topk_labeled(s, lab, 64)
+    order = sorted(range(n), key=lambda i: (-s[i], lab[i]))[:64]
+    assert idx.tolist() == [int(lab[i]) for i in order]
+    assert np.array_equal(sc, s[order])
+    idx, sc = orc.topk_labeled(s[:20], lab[:20], 32)
+    assert idx[:20].tolist() == [int(lab[i]) for i in sorted(range(20), key=lambda i: (-s[i], lab[i]))]
+    assert (idx[20:] == -1).all() and np.isneginf(sc[20:]).all()
+
+
+def test_topk_of_shard_topks_is_topk_of_whole(orc):
+    """Splitting a sequence's entries into contiguous shards: the labeled Top-K over the
+    shards' own Top-K lists (labels = shard offset + local index) is the Top-K of the
+    whole, ties included (the decomposition a context-parallel Full layer uses)."""
+    rng = np.random.default_rng(12)
+    n, K = 1000, 96
+    s = np.round(rng.standard_normal(n), 1)
+    cuts = [0, 130, 131, 600, n]                          # ragged, one single-entry shard
+    cand_s, cand_l = [], []
+    for lo, hi in zip(cuts[:-1], cuts[1:]):
+        li, ls = orc.topk(s[lo:hi], K)
+        keep = li >= 0
+        cand_s.append(ls[keep])
+        cand_l.append(li[keep].astype(np.int64) + lo)
+    got, gs = orc.topk_labeled(np.concatenate(cand_s), np.concatenate(cand_l), K)
+    want, ws = orc.topk(s, K)
+    assert got.tolist() == want.tolist()
+    assert np.array_equal(gs, ws)
