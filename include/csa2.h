@@ -62,6 +62,7 @@ extern "C" {
 #define CSA2_MAX_HI 16           /* largest number of indexer heads */
 #define CSA2_MAX_WINDOW 1024     /* largest sliding window */
 #define CSA2_STATIC_SCRATCH_BYTES (4u << 20) /* device array behind csa2_reindex_static */
+#define CSA2_MAX_SHARDS 64       /* largest number of context-parallel shards per merge */
 
 typedef enum csa2_status {
   CSA2_OK = 0,
@@ -229,6 +230,79 @@ csa2_status csa2_sparse_attn(const float* q, const uint8_t* kv_pool, int64_t poo
                              const int64_t* q_pos, int window, int B, int Q, int H,
                              float sm_scale, float* out, float* lse, void* ws, size_t ws_bytes,
                              uint32_t* dev_status, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Context-parallel decode: one sequence's cached entries split over C GPUs (ranks).
+ * The pages describe one device; this decomposition is the library's reading of how
+ * the same results split (P1 §무엇과 다른가: a Full layer's Top-K is taken over every
+ * entry its query sees; P3 §전역 어텐션과 지역 어텐션: one softmax over the selected
+ * entries and the window).  Rank c holds entries [lo_c, lo_c + len_c) of each sequence
+ * in its own pool; the shards of a sequence are disjoint, contiguous and ordered by rank
+ * (lo_0 < lo_1 < ...).  One Full layer then runs, on every rank:
+ *   1. csa2_cp_shard_vis: the visible count inside the shard;
+ *   2. csa2_index_full (or csa2_index_hier with lo_c a multiple of the block) on the
+ *      rank's pool: its own Top-K with scores;
+ *   3. an all-gather of the (index, score) lists over the ranks (the caller's
+ *      collective, e.g. NCCL): [C][B][Q][K] each;
+ *   4. csa2_topk_merge: the global Top-K (exact: the Top-K of the whole is the Top-K of
+ *      the union of the shards' Top-K lists);
+ *   5. csa2_topk_localize: the rank's own entries of that list, in its pool's indices;
+ *   6. csa2_sparse_attn on them (the window on one rank only): out_c and lse_c;
+ *   7. an all-gather of (out_c, lse_c) and csa2_attn_combine: attention over the union.
+ * The library does not communicate; every call below is rank-local.
+ * --------------------------------------------------------------------------------- */
+
+/* n_vis_local[b][i] = clamp(n_vis[b][i] - shard_lo[b], 0, shard_len[b]).
+ * n_vis int32 [B][Q]; shard_lo, shard_len int64 [B] (this rank's shard of each
+ * sequence); n_vis_local int32 [B][Q].  A negative shard_lo or shard_len gives 0 and
+ * flags CSA2_DEV_BAD_INDEX; a negative n_vis gives 0 and flags CSA2_DEV_BAD_COUNT. */
+csa2_status csa2_cp_shard_vis(const int32_t* n_vis, const int64_t* shard_lo, const int64_t* shard_len, int B,
+                              int Q, int32_t* n_vis_local, uint32_t* dev_status, cudaStream_t stream);
+
+/* Merge of C candidate lists into the K best (P1 §무엇과 다른가, read as above).
+ *   cand int32 [C][B][Q][Kc]: candidate labels local to shard c, -1 = empty slot
+ *   cand_score fp32 [C][B][Q][Kc]: their scores
+ *   part_stride  elements from shard c's list to shard c+1's, in both arrays (0 means
+ *        B*Q*Kc, dense); a larger stride lets one gathered buffer per shard hold
+ *        [labels | scores], so a single all-gather moves both
+ *   shard_off int64 [C][B]: label offset of shard c in sequence b; the global label of
+ *        a candidate is shard_off[c][b] + cand and must fit int32
+ *   topk int32 [B][Q][K] out: global labels of the K best candidates (a set, -1 in
+ *        unused slots); topk_score fp32 [B][Q][K] may be NULL
+ * Order: larger score first (fp32 values compared exactly); equal scores prefer the
+ * lower shard, then the earlier slot, which with lists from csa2_index_full or
+ * csa2_index_hier over shards ordered by rank is the lower global label, as on one
+ * device.  Candidates below -1 or whose label overflows are skipped and flag
+ * CSA2_DEV_BAD_INDEX.  1 <= C <= CSA2_MAX_SHARDS, 1 <= Kc, K <= CSA2_MAX_K. */
+size_t csa2_topk_merge_workspace_size(int C, int B, int Q, int Kc);
+csa2_status csa2_topk_merge(const int32_t* cand, const float* cand_score, int64_t part_stride,
+                            const int64_t* shard_off, int C, int B, int Q, int Kc, int K, int32_t* topk,
+                            float* topk_score, void* ws, size_t ws_bytes, uint32_t* dev_status,
+                            cudaStream_t stream);
+
+/* This rank's part of a merged list: for every query, the labels t of topk int32
+ * [B][Q][K] with shard_off[b] <= t < shard_off[b] + shard_len[b], as t - shard_off[b],
+ * compacted to the front of topk_local int32 [B][Q][K] in slot order; -1 fills the
+ * rest.  shard_off, shard_len int64 [B] (entry units; block units for block lists).
+ * topk_local must not alias topk.  A negative offset or length gives an all-empty row
+ * and flags CSA2_DEV_BAD_INDEX. */
+csa2_status csa2_topk_localize(const int32_t* topk, int B, int Q, int K, const int64_t* shard_off,
+                               const int64_t* shard_len, int32_t* topk_local, uint32_t* dev_status,
+                               cudaStream_t stream);
+
+/* Attention over the union of C disjoint key sets from each set's csa2_sparse_attn
+ * result (P3 §전역 어텐션과 지역 어텐션: one softmax over all of a query's keys).
+ *   out_parts fp32 [C][B][Q][H][512], lse_parts fp32 [C][B][Q][H] (natural log)
+ *   out_part_stride  floats from part c to part c+1 of out_parts (0 means B*Q*H*512,
+ *        dense; else at least that and a multiple of 4); lse_part_stride likewise for
+ *        lse_parts (0 means B*Q*H): one gathered buffer per part can hold [out | lse]
+ *   out fp32 [B][Q][H][512], lse fp32 [B][Q][H]; must not overlap the parts
+ * With M = max_c lse_c: w_c = exp(lse_c - M), out = sum_c w_c out_c / sum_c w_c,
+ * lse = M + log(sum_c w_c), in fp32.  Parts with lse_c = -inf add nothing; all parts
+ * empty give out = 0, lse = -inf.  1 <= C <= CSA2_MAX_SHARDS. */
+csa2_status csa2_attn_combine(const float* out_parts, int64_t out_part_stride, const float* lse_parts,
+                              int64_t lse_part_stride, int C, int B, int Q, int H, float* out, float* lse,
+                              cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------------
  * csa2_reindex_static: csa2_reindex without a workspace argument.  The pages have no

@@ -73,6 +73,16 @@ def lib():
         L.csa2_sparse_attn.restype = I32
         L.csa2_sparse_attn.argtypes = [P, P, I64, P, P, I32, P, I32, P, P, I32, I32, I32, I32, F32, P, P, P,
                                        SZ, P, P]
+        L.csa2_cp_shard_vis.restype = I32
+        L.csa2_cp_shard_vis.argtypes = [P, P, P, I32, I32, P, P, P]
+        L.csa2_topk_merge_workspace_size.restype = SZ
+        L.csa2_topk_merge_workspace_size.argtypes = [I32, I32, I32, I32]
+        L.csa2_topk_merge.restype = I32
+        L.csa2_topk_merge.argtypes = [P, P, I64, P, I32, I32, I32, I32, I32, P, P, P, SZ, P, P]
+        L.csa2_topk_localize.restype = I32
+        L.csa2_topk_localize.argtypes = [P, I32, I32, I32, P, P, P, P, P]
+        L.csa2_attn_combine.restype = I32
+        L.csa2_attn_combine.argtypes = [P, I64, P, I64, I32, I32, I32, I32, P, P, P]
         _lib = L
     return _lib
 
@@ -385,3 +395,99 @@ def csa2_sparse_attn(q, kv_pool, seq_base, topk, swa, swa_start, q_pos, sm_scale
                                   float(sm_scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                                   _ptr(dev_status), _stream(stream)),
            "csa2_sparse_attn")
+
+
+# ---- context-parallel decode ------------------------------------------------------------
+def csa2_cp_shard_vis(n_vis, shard_lo, shard_len, n_vis_local, dev_status=None, stream=None):
+    """n_vis i32 [B,Q]; shard_lo, shard_len i64 [B] -> n_vis_local i32 [B,Q] (the visible
+    count inside this rank's shard)."""
+    _shape(n_vis, (None, None), "n_vis")
+    B, Q = n_vis.shape
+    _rows(shard_lo, B, "shard_lo")
+    _rows(shard_len, B, "shard_len")
+    _shape(n_vis_local, (B, Q), "n_vis_local")
+    _need(n_vis, torch.int32, "n_vis", 2)
+    _need(shard_lo, torch.int64, "shard_lo", 1)
+    _need(shard_len, torch.int64, "shard_len", 1)
+    _need(n_vis_local, torch.int32, "n_vis_local", 2)
+    _status(dev_status)
+    _check(lib().csa2_cp_shard_vis(_ptr(n_vis), _ptr(shard_lo), _ptr(shard_len), B, Q, _ptr(n_vis_local),
+                                   _ptr(dev_status), _stream(stream)), "csa2_cp_shard_vis")
+
+
+def csa2_topk_merge_workspace_size(C, B, Q, Kc):
+    return lib().csa2_topk_merge_workspace_size(C, B, Q, Kc)
+
+
+def _part_stride(t, name):
+    """Elements from one part to the next of a [C, ...] tensor whose parts are each
+    contiguous (0 for a single part: the library then takes the dense stride)."""
+    if t.dim() < 1 or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor with a leading part dimension")
+    if not t[0].is_contiguous():
+        raise ValueError(f"{name}: each part must be contiguous")
+    return t.stride(0) if t.shape[0] > 1 else 0
+
+
+def csa2_topk_merge(cand, cand_score, shard_off, K, topk, topk_score=None, ws=None, dev_status=None,
+                    stream=None):
+    """cand i32 [C,B,Q,Kc] (labels local to each shard, -1 empty), cand_score f32 [C,B,Q,Kc],
+    shard_off i64 [C,B] -> topk i32 [B,Q,K] global labels (+ topk_score f32 [B,Q,K]).
+    cand and cand_score may be strided views (parts each contiguous, same part stride),
+    e.g. the two halves of one gathered buffer per shard."""
+    _shape(cand, (None, None, None, None), "cand")
+    C, B, Q, Kc = cand.shape
+    _shape(cand_score, (C, B, Q, Kc), "cand_score")
+    _shape(shard_off, (C, B), "shard_off")
+    _shape(topk, (B, Q, K), "topk")
+    _shape(topk_score, (B, Q, K), "topk_score")
+    if cand.dtype != torch.int32 or cand_score.dtype != torch.float32:
+        raise TypeError("cand must be int32 and cand_score float32")
+    ps = _part_stride(cand, "cand")
+    if _part_stride(cand_score, "cand_score") != ps:
+        raise ValueError("cand and cand_score must have the same part stride")
+    _need(shard_off, torch.int64, "shard_off", 2)
+    _need(topk, torch.int32, "topk", 3)
+    _need(topk_score, torch.float32, "topk_score", 3)
+    _status(dev_status)
+    if ws is None:
+        ws = workspace(csa2_topk_merge_workspace_size(C, B, Q, Kc), cand.device)
+    _check(lib().csa2_topk_merge(_ptr(cand), _ptr(cand_score), int(ps), _ptr(shard_off), C, B, Q, Kc, int(K),
+                                 _ptr(topk), _ptr(topk_score), _ptr(ws), ws.numel(), _ptr(dev_status),
+                                 _stream(stream)), "csa2_topk_merge")
+
+
+def csa2_topk_localize(topk, shard_off, shard_len, topk_local, dev_status=None, stream=None):
+    """topk i32 [B,Q,K] global labels; shard_off, shard_len i64 [B] -> topk_local i32
+    [B,Q,K]: this shard's labels minus its offset, compacted, -1 after them."""
+    _shape(topk, (None, None, None), "topk")
+    B, Q, K = topk.shape
+    _rows(shard_off, B, "shard_off")
+    _rows(shard_len, B, "shard_len")
+    _shape(topk_local, (B, Q, K), "topk_local")
+    _need(topk, torch.int32, "topk", 3)
+    _need(shard_off, torch.int64, "shard_off", 1)
+    _need(shard_len, torch.int64, "shard_len", 1)
+    _need(topk_local, torch.int32, "topk_local", 3)
+    _status(dev_status)
+    _check(lib().csa2_topk_localize(_ptr(topk), B, Q, K, _ptr(shard_off), _ptr(shard_len), _ptr(topk_local),
+                                    _ptr(dev_status), _stream(stream)), "csa2_topk_localize")
+
+
+def csa2_attn_combine(out_parts, lse_parts, out, lse, stream=None):
+    """out_parts f32 [C,B,Q,H,512], lse_parts f32 [C,B,Q,H] (parts each contiguous; dense,
+    or views of one gathered [out | lse] buffer per part) -> out f32 [B,Q,H,512], lse f32
+    [B,Q,H]: attention over the union."""
+    _shape(out_parts, (None, None, None, None, D), "out_parts")
+    C, B, Q, H, _ = out_parts.shape
+    _shape(lse_parts, (C, B, Q, H), "lse_parts")
+    _shape(out, (B, Q, H, D), "out")
+    _shape(lse, (B, Q, H), "lse")
+    if out_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32:
+        raise TypeError("out_parts and lse_parts must be float32")
+    pso = _part_stride(out_parts, "out_parts")
+    psl = _part_stride(lse_parts, "lse_parts")
+    _need(out, torch.float32, "out", 4)
+    _need(lse, torch.float32, "lse", 3)
+    _check(lib().csa2_attn_combine(_ptr(out_parts), int(pso), _ptr(lse_parts), int(psl), C, B, Q, H, _ptr(out),
+                                   _ptr(lse), _stream(stream)), "csa2_attn_combine")

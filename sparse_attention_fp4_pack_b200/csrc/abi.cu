@@ -27,6 +27,15 @@ cudaError_t launch_sparse_attn(const float* q, const uint8_t* kv_pool, int64_t p
                                const int64_t* q_pos, int window, int B, int Q, int H,
                                float sm_scale, float* out, float* lse, void* ws,
                                uint32_t* status, cudaStream_t stream);
+cudaError_t launch_shard_vis(const int32_t* n_vis, const int64_t* lo, const int64_t* len, int B, int Q,
+                             int32_t* out, uint32_t* status, cudaStream_t stream);
+cudaError_t launch_topk_merge(const int32_t* cand, const float* score, int64_t part, const int64_t* shard_off,
+                              int C, int B, int Q, int Kc, int K, int32_t* topk, float* topk_score, uint32_t* keys,
+                              int32_t* labels, int64_t stride, uint32_t* status, cudaStream_t stream);
+cudaError_t launch_topk_localize(const int32_t* topk, int B, int Q, int K, const int64_t* off, const int64_t* len,
+                                 int32_t* out, uint32_t* status, cudaStream_t stream);
+cudaError_t launch_attn_combine(const float* out_parts, int64_t part_o, const float* lse_parts, int64_t part_l,
+                                int C, int64_t N, float* out, float* lse, cudaStream_t stream);
 }  // namespace csa2
 
 namespace {
@@ -272,6 +281,78 @@ csa2_status csa2_sparse_attn(const float* q, const uint8_t* kv_pool, int64_t poo
   return launched(csa2::launch_sparse_attn(q, kv_pool, pool_entries, seq_base, topk, K, swa, S_w,
                                            swa_start, q_pos, window, B, Q, H, sm_scale, out, lse,
                                            ws, dev_status, stream));
+}
+
+// ---- context-parallel decode -----------------------------------------------------------
+
+csa2_status csa2_cp_shard_vis(const int32_t* n_vis, const int64_t* shard_lo, const int64_t* shard_len, int B,
+                              int Q, int32_t* n_vis_local, uint32_t* dev_status, cudaStream_t stream) {
+  if (B < 0 || Q < 0) return CSA2_ERR_INVALID_ARG;
+  if ((int64_t)B * Q == 0) return CSA2_OK;
+  if (!n_vis || !shard_lo || !shard_len || !n_vis_local) return CSA2_ERR_INVALID_ARG;
+  if (!aligned(n_vis, 4) || !aligned(shard_lo, 8) || !aligned(shard_len, 8) || !aligned(n_vis_local, 4))
+    return CSA2_ERR_INVALID_ARG;
+  return launched(csa2::launch_shard_vis(n_vis, shard_lo, shard_len, B, Q, n_vis_local, dev_status, stream));
+}
+
+size_t csa2_topk_merge_workspace_size(int C, int B, int Q, int Kc) {
+  if (C <= 0 || B <= 0 || Q <= 0 || Kc <= 0) return 0;
+  const size_t row = (size_t)key_row((int64_t)C * Kc);
+  return 2 * round256((size_t)B * Q * row * sizeof(uint32_t));
+}
+
+csa2_status csa2_topk_merge(const int32_t* cand, const float* cand_score, int64_t part_stride,
+                            const int64_t* shard_off, int C, int B, int Q, int Kc, int K, int32_t* topk,
+                            float* topk_score, void* ws, size_t ws_bytes, uint32_t* dev_status,
+                            cudaStream_t stream) {
+  if (B < 0 || Q < 0 || part_stride < 0) return CSA2_ERR_INVALID_ARG;
+  if (C < 1 || C > CSA2_MAX_SHARDS || Kc < 1 || Kc > CSA2_MAX_K || K < 1 || K > CSA2_MAX_K)
+    return CSA2_ERR_UNSUPPORTED;
+  if ((int64_t)B * Q > kMaxQueries) return CSA2_ERR_UNSUPPORTED;
+  if ((int64_t)B * Q == 0) return CSA2_OK;
+  if (!cand || !cand_score || !shard_off || !topk) return CSA2_ERR_INVALID_ARG;
+  if (!aligned(cand, 4) || !aligned(cand_score, 4) || !aligned(shard_off, 8) || !aligned(topk, 4) ||
+      (topk_score && !aligned(topk_score, 4)))
+    return CSA2_ERR_INVALID_ARG;
+  const size_t need = csa2_topk_merge_workspace_size(C, B, Q, Kc);
+  csa2_status st = check_ws(ws, ws_bytes, need);
+  if (st != CSA2_OK) return st;
+  const int64_t part = part_stride > 0 ? part_stride : (int64_t)B * Q * Kc;
+  if (part < (int64_t)B * Q * Kc) return CSA2_ERR_INVALID_ARG;
+  const int64_t stride = key_row((int64_t)C * Kc);
+  uint32_t* keys = static_cast<uint32_t*>(ws);
+  int32_t* labels = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + need / 2);
+  return launched(csa2::launch_topk_merge(cand, cand_score, part, shard_off, C, B, Q, Kc, K, topk, topk_score, keys,
+                                          labels, stride, dev_status, stream));
+}
+
+csa2_status csa2_topk_localize(const int32_t* topk, int B, int Q, int K, const int64_t* shard_off,
+                               const int64_t* shard_len, int32_t* topk_local, uint32_t* dev_status,
+                               cudaStream_t stream) {
+  if (B < 0 || Q < 0 || K < 0) return CSA2_ERR_INVALID_ARG;
+  if ((int64_t)B * Q == 0 || K == 0) return CSA2_OK;
+  if (!topk || !shard_off || !shard_len || !topk_local) return CSA2_ERR_INVALID_ARG;
+  if (!aligned(topk, 4) || !aligned(shard_off, 8) || !aligned(shard_len, 8) || !aligned(topk_local, 4))
+    return CSA2_ERR_INVALID_ARG;
+  if (topk == topk_local) return CSA2_ERR_INVALID_ARG;
+  return launched(csa2::launch_topk_localize(topk, B, Q, K, shard_off, shard_len, topk_local, dev_status, stream));
+}
+
+csa2_status csa2_attn_combine(const float* out_parts, int64_t out_part_stride, const float* lse_parts,
+                              int64_t lse_part_stride, int C, int B, int Q, int H, float* out, float* lse,
+                              cudaStream_t stream) {
+  if (B < 0 || Q < 0 || H < 0 || out_part_stride < 0 || lse_part_stride < 0) return CSA2_ERR_INVALID_ARG;
+  if (C < 1 || C > CSA2_MAX_SHARDS) return CSA2_ERR_UNSUPPORTED;
+  const int64_t N = (int64_t)B * Q * H;
+  if (N == 0) return CSA2_OK;
+  if (N > ((int64_t)1 << 31)) return CSA2_ERR_UNSUPPORTED;
+  if (!out_parts || !lse_parts || !out || !lse) return CSA2_ERR_INVALID_ARG;
+  const int64_t part_o = out_part_stride > 0 ? out_part_stride : N * CSA2_D;
+  const int64_t part_l = lse_part_stride > 0 ? lse_part_stride : N;
+  if (part_o < N * CSA2_D || part_o % 4 != 0 || part_l < N) return CSA2_ERR_INVALID_ARG;
+  if (!aligned(out_parts, 16) || !aligned(lse_parts, 4) || !aligned(out, 16) || !aligned(lse, 4))
+    return CSA2_ERR_INVALID_ARG;
+  return launched(csa2::launch_attn_combine(out_parts, part_o, lse_parts, part_l, C, N, out, lse, stream));
 }
 
 }  // extern "C"

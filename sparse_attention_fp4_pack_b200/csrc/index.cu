@@ -37,7 +37,8 @@
 
 namespace csa2 {
 
-enum ScanMode : int { kFlat = 0, kHier = 1, kReindex = 2 };
+// kMerge: selection only, over caller-built keys and labels (the merge of several lists)
+enum ScanMode : int { kFlat = 0, kHier = 1, kReindex = 2, kMerge = 3 };
 
 constexpr int kRows = 128;               // entries per tile = UMMA M
 constexpr int kScanThreads = 128;
@@ -669,6 +670,8 @@ struct SelectArgs {
   const int32_t* n_vis;
   int64_t max_n_vis, pool_entries;
   const int32_t* blocks;
+  const int32_t* labels;     // kMerge: label of item i at labels[bq * key_stride + i]
+  int64_t n_items;           // kMerge: items per query
   int32_t* out_idx;
   float* out_score;
 };
@@ -680,6 +683,7 @@ __device__ __forceinline__ int64_t item_label(const SelectArgs& a, const int32_t
     const int32_t c = blk[i >> a.block_shift];
     return ((int64_t)c << a.block_shift) + (i & (a.block - 1));
   }
+  if (a.mode == kMerge) return a.labels[(int64_t)blockIdx.y * a.key_stride + i];
   return i;
 }
 
@@ -795,7 +799,9 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
   auto remote = [&](const uint32_t* src, int r) { return tc::mapa(tc::smem_u32(src), (uint32_t)r); };
 
   int64_t n;
-  {
+  if (a.mode == kMerge) {
+    n = a.n_items;
+  } else {
     const int64_t base = a.seq_base[b];
     int64_t nv = a.n_vis[bq];
     if (nv < 0 || nv > a.max_n_vis || base < 0 || base + nv > a.pool_entries) nv = 0;
@@ -1192,6 +1198,60 @@ static cudaError_t launch_stream(ScanArgs a, int64_t items, int B, cudaStream_t 
   return cudaGetLastError();
 }
 
+// Selection of the K best of `items` keys per query row (blockIdx.y = row).
+static cudaError_t launch_select(SelectArgs s, int64_t items, int BQ, cudaStream_t stream) {
+  // At most 4,096 keys: one CTA with 4 keys per thread.  Otherwise one CTA per 16,384 keys
+  // (16 per thread), up to 8.  (Splitting a 16,384-key list over a cluster of 4-key CTAs
+  // measured no faster: each radix level then waits on two cluster barriers and a
+  // remote histogram sum, which cost what the shorter count saves.)
+  cudaError_t e;
+  if (items <= SelShape<2>::kChunk) {
+    s.csize = 1;
+    e = cudaFuncSetAttribute(select_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, SelShape<2>::kSmem);
+    if (e != cudaSuccess) return e;
+    e = launch_chained(select_kernel<2>, dim3((unsigned)s.csize, (unsigned)BQ), dim3(kSelThreads),
+                       SelShape<2>::kSmem, stream, (unsigned)s.csize, s);
+  } else {
+    // one CTA per 16,384 keys, up to a cluster of 8; when the queries alone fill the GPU
+    // for more than two waves, fewer CTAs per query (each walks several chunks), since a
+    // wide cluster then only adds waves and cluster barriers
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int64_t c = (items + SelShape<4>::kChunk - 1) / SelShape<4>::kChunk;
+    c = c < 1 ? 1 : (c > kMaxCluster ? kMaxCluster : c);
+    const int64_t fit = (2 * (int64_t)sms) / (BQ > 0 ? BQ : 1);  // CTAs per query in two waves
+    if (c > fit) c = fit < 1 ? 1 : (fit >= 8 ? 8 : (fit >= 4 ? 4 : (fit >= 2 ? 2 : 1)));
+    s.csize = (int)c;
+    e = cudaFuncSetAttribute(select_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, SelShape<4>::kSmem);
+    if (e != cudaSuccess) return e;
+    e = launch_chained(select_kernel<4>, dim3((unsigned)s.csize, (unsigned)BQ), dim3(kSelThreads),
+                       SelShape<4>::kSmem, stream, (unsigned)s.csize, s);
+  }
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// Merge: the K best of n_items caller-built keys (0 = no candidate) per query row, each
+// item named by its label; keys and labels are rows of key_stride (a multiple of 4).
+cudaError_t launch_select_labeled(const uint32_t* keys, const int32_t* labels, int64_t key_stride,
+                                  int64_t n_items, int BQ, int K, int32_t* out_idx, float* out_score,
+                                  cudaStream_t stream) {
+  SelectArgs s = {};
+  s.keys = keys;
+  s.key_stride = key_stride;
+  s.mode = kMerge;
+  s.Q = 1;
+  s.block = 1;
+  s.block_shift = 0;
+  s.K = K;
+  s.labels = labels;
+  s.n_items = n_items;
+  s.out_idx = out_idx;
+  s.out_score = out_score;
+  if (BQ == 0) return cudaSuccess;
+  return launch_select(s, n_items, BQ, stream);
+}
+
 cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t* ik_pool,
                          int64_t pool_entries, const int64_t* seq_base, const int32_t* n_vis,
                          const int32_t* blocks, int B, int Q, int HI, int n_blocks, int block,
@@ -1241,39 +1301,14 @@ cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t
   s.max_n_vis = max_n_vis;
   s.pool_entries = pool_entries;
   s.blocks = blocks;
+  s.labels = nullptr;
+  s.n_items = 0;
   s.out_idx = out_idx;
   s.out_score = out_score;
   const int64_t items = mode == kFlat ? max_n_vis
                         : mode == kHier ? (max_n_vis + block - 1) / block
                                         : (int64_t)n_blocks * block;
-  // At most 4,096 keys: one CTA with 4 keys per thread.  Otherwise one CTA per 16,384 keys
-  // (16 per thread), up to 8.  (Splitting a 16,384-key list over a cluster of 4-key CTAs
-  // measured no faster: each radix level then waits on two cluster barriers and a
-  // remote histogram sum, which cost what the shorter count saves.)
-  if (items <= SelShape<2>::kChunk) {
-    s.csize = 1;
-    e = cudaFuncSetAttribute(select_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, SelShape<2>::kSmem);
-    if (e != cudaSuccess) return e;
-    e = launch_chained(select_kernel<2>, dim3((unsigned)s.csize, (unsigned)BQ), dim3(kSelThreads),
-                       SelShape<2>::kSmem, stream, (unsigned)s.csize, s);
-  } else {
-    // one CTA per 16,384 keys, up to a cluster of 8; when the queries alone fill the GPU
-    // for more than two waves, fewer CTAs per query (each walks several chunks), since a
-    // wide cluster then only adds waves and cluster barriers
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int64_t c = (items + SelShape<4>::kChunk - 1) / SelShape<4>::kChunk;
-    c = c < 1 ? 1 : (c > kMaxCluster ? kMaxCluster : c);
-    const int64_t fit = (2 * (int64_t)sms) / (BQ > 0 ? BQ : 1);  // CTAs per query in two waves
-    if (c > fit) c = fit < 1 ? 1 : (fit >= 8 ? 8 : (fit >= 4 ? 4 : (fit >= 2 ? 2 : 1)));
-    s.csize = (int)c;
-    e = cudaFuncSetAttribute(select_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, SelShape<4>::kSmem);
-    if (e != cudaSuccess) return e;
-    e = launch_chained(select_kernel<4>, dim3((unsigned)s.csize, (unsigned)BQ), dim3(kSelThreads),
-                       SelShape<4>::kSmem, stream, (unsigned)s.csize, s);
-  }
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  return launch_select(s, items, BQ, stream);
 }
 
 }  // namespace csa2

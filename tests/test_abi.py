@@ -57,6 +57,7 @@ def test_workspace_sizes(L):
 P = ctypes.c_void_p
 FAKE = P(0x10000)       # 16-aligned, never dereferenced: validation fails before any launch
 MIS = P(0x10004)        # misaligned
+MIS2 = P(0x10002)       # misaligned for 4-byte elements too
 
 
 def test_pack_rejects_bad_args(L):
@@ -100,6 +101,39 @@ def test_attn_rejects_bad_args(L):
     assert L.csa2_sparse_attn(*base(64, 512, 4096, 0.04, FAKE, 128)) == 2       # window too large
     assert L.csa2_sparse_attn(*base(64, 512, 128, float("nan"), FAKE, 128)) == 1  # scale
     assert L.csa2_sparse_attn(*base(64, 512, 128, 0.04, None, 128)) == 1        # window data missing
+
+
+def test_context_parallel_calls_reject_bad_args(L):
+    st = ctypes.c_void_p(0)
+    assert L.csa2_topk_merge_workspace_size(8, 4, 1, 512) == 2 * 4 * 4096 * 4
+    assert L.csa2_topk_merge_workspace_size(0, 4, 1, 512) == 0
+    merge = lambda ps, C, Kc, K, ws, wsb: (FAKE, FAKE, ps, FAKE, C, 2, 1, Kc, K, FAKE, None, ws, wsb, None, st)
+    big = 1 << 30
+    assert L.csa2_topk_merge(*merge(0, 0, 64, 64, FAKE, big)) == 2          # no shards
+    assert L.csa2_topk_merge(*merge(0, 65, 64, 64, FAKE, big)) == 2         # above CSA2_MAX_SHARDS
+    assert L.csa2_topk_merge(*merge(0, 8, 4096, 64, FAKE, big)) == 2        # Kc above 2048
+    assert L.csa2_topk_merge(*merge(0, 8, 64, 0, FAKE, big)) == 2           # K = 0
+    assert L.csa2_topk_merge(*merge(100, 8, 64, 64, FAKE, big)) == 1        # parts overlap (stride < B*Q*Kc)
+    assert L.csa2_topk_merge(*merge(-1, 8, 64, 64, FAKE, big)) == 1         # negative stride
+    assert L.csa2_topk_merge(*merge(0, 8, 64, 64, None, big)) == 1          # no workspace
+    assert L.csa2_topk_merge(*merge(0, 8, 64, 64, FAKE, 64)) == 1           # workspace too small
+    assert L.csa2_topk_merge(MIS2, FAKE, 0, FAKE, 8, 2, 1, 64, 64, FAKE, None, FAKE, big, None, st) == 1
+    assert L.csa2_topk_merge(FAKE, FAKE, 0, FAKE, 8, 0, 1, 64, 64, None, None, None, 0, None, st) == 0
+    assert L.csa2_topk_localize(FAKE, 2, 1, 64, FAKE, FAKE, FAKE, None, st) == 1   # output aliases input
+    assert L.csa2_topk_localize(FAKE, 2, 1, 64, None, FAKE, P(0x20000), None, st) == 1
+    assert L.csa2_topk_localize(FAKE, 0, 1, 64, None, None, None, None, st) == 0
+    assert L.csa2_cp_shard_vis(FAKE, None, FAKE, 2, 1, FAKE, None, st) == 1
+    assert L.csa2_cp_shard_vis(FAKE, FAKE, FAKE, 2, 1, MIS2, None, st) == 1
+    assert L.csa2_cp_shard_vis(None, None, None, 0, 1, None, None, st) == 0
+    comb = lambda pso, psl, C, op: (op, pso, FAKE, psl, C, 2, 1, 16, FAKE, FAKE, st)
+    assert L.csa2_attn_combine(*comb(0, 0, 0, FAKE)) == 2                   # no parts
+    assert L.csa2_attn_combine(*comb(0, 0, 65, FAKE)) == 2
+    assert L.csa2_attn_combine(*comb(32 * 512 + 2, 0, 3, FAKE)) == 1        # stride not a multiple of 4
+    assert L.csa2_attn_combine(*comb(100, 0, 3, FAKE)) == 1                 # output parts overlap
+    assert L.csa2_attn_combine(*comb(0, 31, 3, FAKE)) == 1                  # lse parts overlap
+    assert L.csa2_attn_combine(*comb(0, -1, 3, FAKE)) == 1
+    assert L.csa2_attn_combine(*comb(0, 0, 3, MIS)) == 1                    # misaligned parts
+    assert L.csa2_attn_combine(FAKE, 0, FAKE, 0, 3, 0, 1, 16, None, None, st) == 0
 
 
 def test_binding_checks_shapes_before_the_device():
