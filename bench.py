@@ -64,6 +64,8 @@ def parse_args():
                    help="time the step without the per-call events (no breakdown or roofline)")
     p.add_argument("--no-configs", action="store_true",
                    help="measure only --workload (by default hier1m also brings full128k, verify and prefill)")
+    p.add_argument("--cp-ranks", type=int, default=8,
+                   help="at N=1, also time hier1m split over this many context-parallel ranks (0: skip)")
     return p.parse_args()
 
 
@@ -456,6 +458,74 @@ def measure(name, steps, warmup, world, dev, call_timing=True, e2e=True):
     return res
 
 
+def measure_cp(name, ranks, steps, warmup, dev):
+    """Context parallelism over `ranks` ranks, emulated on this one GPU.  Every rank's step runs
+    once in lockstep (the ranks reading their shards in place from one shared pool) to record
+    what each exchange delivers.  Then each rank's step runs on its own in a CUDA graph, the
+    recorded buffers taking the place of the all-gathers, timed like the main step (L2 flushed
+    between steps).  The slowest rank's time is the step's compute critical path on `ranks`
+    GPUs; the all-gathers themselves (NCCL over NVLink) are not in it, so their count and
+    sizes are reported beside it."""
+    import synth
+    from sparse_attention_fp4_pack_b200.cp import CPDecodeStep, ShardLayout, run_lockstep, run_replay
+    from sparse_attention_fp4_pack_b200.workload import build_state
+
+    wl = synth.workload(name)
+    sched = synth.layer_schedule(wl)
+    qd = synth.step_queries(wl)
+    x = build_state(wl, lambda b: synth.seq_tokens(wl, b, device=dev), qd, device=dev)
+    lengths = [int(n) for n in wl.lengths]
+    cps = []
+    for c in range(ranks):
+        lay = ShardLayout.in_shared_pool(c, ranks, lengths, x.seq_base, dev, block=wl.block)
+        cps.append(CPDecodeStep(lay, B=wl.B, Q=wl.Q, H=wl.H, HI=wl.HI, K=wl.K, window=wl.window, ratio=wl.ratio,
+                                schedule=sched, hier=wl.hier, max_shard_len=int(lay.length.max()),
+                                n_blocks=wl.n_blocks, block=wl.block, device=dev))
+    rec = []
+    run_lockstep(cps, [x] * ranks, record=rec)
+    torch.cuda.synchronize()
+    for s_ in cps:
+        s_.check_status()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    per_rank = []
+    for c, st in enumerate(cps):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            run_replay(st, x, rec)
+        torch.cuda.current_stream().wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            run_replay(st, x, rec)
+        total = 0.0
+        for i in range(warmup + steps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            flush.fill_(1)
+            torch.cuda.synchronize()
+            if i >= warmup:
+                total += e0.elapsed_time(e1)
+        st.check_status()
+        per_rank.append(total / steps)
+        del g
+    sizes = [int(r[0].numel() * r[0].element_size()) for r in rec]
+    worst = max(per_rank)
+    out = {"workload": f"{name} split over {ranks} ranks (contiguous shards of every sequence), emulated on one GPU",
+           "ranks": ranks, "ms_per_step_per_rank": [round(v, 4) for v in per_rank],
+           "ms_per_step_slowest_rank": round(worst, 4),
+           "us_per_token_compute": round(worst * 1000.0 / (wl.B * wl.Q), 3), "unit": UNIT,
+           "exchanges_per_step": len(rec), "exchange_bytes_per_rank_per_step": sum(sizes),
+           "largest_exchange_bytes_per_rank": max(sizes),
+           "note": "device time of one rank's kernels, its exchanges' gathered buffers replayed from a recorded "
+                   "lockstep run; the all-gathers are not timed (one GPU)"}
+    del cps, x, rec, flush
+    torch.cuda.empty_cache()
+    return out
+
+
 def config_of(name, wl, sched, world, cache_bytes):
     return {"workload": f"{name}: {WORKLOAD_TEXT[name]}", "B": wl.B, "Q": wl.Q, "H": wl.H, "HI": wl.HI,
             "K": wl.K, "window": wl.window, "layers": len(sched), "entries_per_seq": max(wl.lengths),
@@ -499,6 +569,8 @@ def run_ours(args, world, rank, local):
                              "clocks": c["clocks"]}
     if configs:
         line["configs"] = configs
+    if not args.no_configs and args.workload == "hier1m" and args.cp_ranks > 1 and world == 1:
+        line["context_parallel"] = measure_cp(args.workload, args.cp_ranks, args.steps, args.warmup, dev)
     return line, wl
 
 

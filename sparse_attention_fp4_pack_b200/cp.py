@@ -26,7 +26,7 @@ ranks' generators in turn within one process, the gather being a stack of their 
 """
 from dataclasses import dataclass
 import math
-from typing import List, Sequence
+from typing import List, Optional, Sequence
 
 import torch
 
@@ -51,10 +51,9 @@ class ShardLayout:
         return int(self.lo.shape[0])
 
     @staticmethod
-    def contiguous(rank, world, seq_len: Sequence[int], device, block: int = 8, window_rank=None):
-        """Every sequence split into `world` near-equal contiguous shards (cut points rounded
-        down to a multiple of `block`, the last shard taking the rest); each rank's pools
-        hold its shards back to back in sequence order."""
+    def _cuts(world, seq_len, block):
+        """Near-equal contiguous shards: cut points rounded down to a multiple of `block`,
+        the last shard taking the rest.  (lo, length) int64 [world, B] on the host."""
         B = len(seq_len)
         lo = torch.zeros(world, B, dtype=torch.int64)
         ln = torch.zeros(world, B, dtype=torch.int64)
@@ -62,8 +61,25 @@ class ShardLayout:
             cuts = [0] + [(n * c // world) // block * block for c in range(1, world)] + [n]
             for c in range(world):
                 lo[c, b], ln[c, b] = cuts[c], cuts[c + 1] - cuts[c]
-        base = torch.zeros(B, dtype=torch.int64)
+        return lo, ln
+
+    @staticmethod
+    def contiguous(rank, world, seq_len: Sequence[int], device, block: int = 8, window_rank=None):
+        """Every sequence split into `world` near-equal contiguous shards; each rank's pools
+        hold its shards back to back in sequence order."""
+        lo, ln = ShardLayout._cuts(world, seq_len, block)
+        base = torch.zeros(len(seq_len), dtype=torch.int64)
         base[1:] = torch.cumsum(ln[rank], 0)[:-1]
+        return ShardLayout(rank, lo.to(device), ln.to(device), base.to(device),
+                           world - 1 if window_rank is None else window_rank)
+
+    @staticmethod
+    def in_shared_pool(rank, world, seq_len: Sequence[int], seq_base, device, block: int = 8, window_rank=None):
+        """The same shards, but read in place from one pool that holds every sequence whole
+        (sequence b from seq_base[b]): several ranks in one process share a single copy of
+        the cache, each reading only its shards' entries."""
+        lo, ln = ShardLayout._cuts(world, seq_len, block)
+        base = torch.as_tensor(seq_base, dtype=torch.int64).cpu() + lo[rank]
         return ShardLayout(rank, lo.to(device), ln.to(device), base.to(device),
                            world - 1 if window_rank is None else window_rank)
 
@@ -234,14 +250,17 @@ def run_distributed(step: CPDecodeStep, x, group=None):
         pass
 
 
-def run_lockstep(steps: Sequence[CPDecodeStep], xs):
+def run_lockstep(steps: Sequence[CPDecodeStep], xs, record: Optional[list] = None):
     """Run every rank's step in one process, in turn up to each exchange; the gather of an
     exchange is the stack of the ranks' send buffers (same device).  For checking the
-    decomposition where only one GPU is present: nothing here waits on another rank."""
+    decomposition where only one GPU is present: nothing here waits on another rank.  With
+    `record` (a list), each exchange's gathered buffer is appended to it."""
     gens = [s.steps(x) for s, x in zip(steps, xs)]
     sends = [next(g) for g in gens]
     while True:
         stacked = torch.stack(sends)
+        if record is not None:
+            record.append(stacked)
         nxt = []
         done = 0
         for g in gens:
@@ -253,3 +272,19 @@ def run_lockstep(steps: Sequence[CPDecodeStep], xs):
             assert done == len(gens), "ranks left the step at different exchanges"
             return
         sends = nxt
+
+
+def run_replay(step: CPDecodeStep, x, gathered: Sequence[torch.Tensor]):
+    """One rank's step with every exchange's gathered buffer given in advance (e.g. recorded
+    by run_lockstep): the rank's own kernels alone, in the order a real step issues them,
+    with no collective.  Used to time one rank's share of a step on its own."""
+    gen = step.steps(x)
+    send = next(gen)
+    for i, g in enumerate(gathered):
+        assert g.shape[1:] == send.shape, f"exchange {i}: recorded buffer does not fit"
+        try:
+            send = gen.send(g)
+        except StopIteration:
+            assert i == len(gathered) - 1, "the step ended before the recorded exchanges did"
+            return
+    raise AssertionError("the step has more exchanges than were recorded")

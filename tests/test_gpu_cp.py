@@ -260,3 +260,30 @@ def test_cp_rank_with_empty_shard(orc):
                               lengths=[40, 3000], n_layers=2)
     steps = _run_and_check(orc, wl, 6)
     assert any(int(s.length[0]) == 0 for s in steps)
+
+
+def test_cp_hier1m_eight_ranks_sampled(orc):
+    """The hier1m step (4 x 2^20 entries, 20 layers) split over eight ranks in lockstep, the
+    ranks reading their shards in place from one shared pool; sequence 2 against the oracle
+    as in the single-device full-size check."""
+    wl = synth.workload("hier1m")
+    sched = synth.layer_schedule(wl)
+    qd = synth.step_queries(wl)
+    x = build_state(wl, lambda b: synth.seq_tokens(wl, b, device="cuda"), qd)
+    lengths = [int(n) for n in wl.lengths]
+    steps = []
+    for c in range(8):
+        lay = ShardLayout.in_shared_pool(c, 8, lengths, x.seq_base, "cuda", block=wl.block)
+        steps.append(CPDecodeStep(lay, B=wl.B, Q=wl.Q, H=wl.H, HI=wl.HI, K=wl.K, window=wl.window, ratio=wl.ratio,
+                                  schedule=sched, hier=True, max_shard_len=int(lay.length.max()), n_blocks=2048,
+                                  block=wl.block))
+    run_lockstep(steps, [x] * 8)
+    torch.cuda.synchronize()
+    for s in steps:
+        s.check_status()
+    own = [l for l, m in enumerate(sched) if m != "reuse"]
+    for s in steps[1:]:
+        assert torch.equal(s.topk[own], steps[0].topk[own]) and torch.equal(s.out, steps[0].out)
+    m = steps[0]
+    single.check_hier1m_sampled(orc, wl, sched, qd, x.kv_pool, x.ik_pool, int(x.seq_base[2]), m.blocks, m.topk,
+                                m.layer_topk, m.out, m.lse)

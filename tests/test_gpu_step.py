@@ -162,17 +162,23 @@ def test_hier1m_step_graph_sampled(orc):
     step.replay()
     torch.cuda.synchronize()
     step.check_status()
-    b = 2
+    check_hier1m_sampled(orc, wl, sched, qd, x.kv_pool, x.ik_pool, int(x.seq_base[2]), step.blocks, step.topk,
+                         step.layer_topk, step.out, step.lse)
+
+
+def check_hier1m_sampled(orc, wl, sched, qd, kv_pool, ik_pool, base, blocks, topk, layer_topk, out, lse, b=2):
+    """Sequence b of a hier1m step against the oracle: its packed pool (from `base` in the
+    pools), the layer-0 block set, every layer's Top-512 and every layer's attention output
+    (the oracle attending with the GPU's list)."""
     N = int(wl.lengths[b])
-    base = int(x.seq_base[b])
     kv, ik = synth.seq_tokens(wl, b, device="cuda")
     o_kv, o_ik = orc.pack_kv(bf16_bits(kv), bf16_bits(ik), wl.ratio)
     del kv, ik
-    assert np.array_equal(np_u8(x.kv_pool[base:base + N]), o_kv)
-    assert np.array_equal(np_u8(x.ik_pool[base:base + N]), o_ik)
+    assert np.array_equal(np_u8(kv_pool[base:base + N]), o_kv)
+    assert np.array_equal(np_u8(ik_pool[base:base + N]), o_ik)
     one = lambda t: t[b:b + 1].numpy()
     n_vis = int(qd["n_vis"][b, 0])
-    g_blocks = step.blocks.cpu().numpy()[b, 0]
+    g_blocks = blocks.cpu().numpy()[b, 0]
     cand = np.sort((g_blocks[:, None] * wl.block + np.arange(wl.block)[None, :]).reshape(-1))
     cand = cand[cand < n_vis]
     for l, mode in enumerate(sched):
@@ -184,13 +190,12 @@ def test_hier1m_step_graph_sampled(orc):
         if mode in ("full", "reindex"):
             sl = orc.index_scores(qd["qi"][l][b, 0].numpy(), qd["w"][l][b, 0].numpy(), o_ik[cand])
             o_sel, _ = orc.topk(sl, wl.K)
-            assert_topk_set(step.topk[l].cpu().numpy()[b, 0], cand[o_sel], sl, wl.K, labels=cand,
-                            what=f"layer {l}")
-        g_topk = step.layer_topk(l).cpu().numpy()[b:b + 1]
+            assert_topk_set(topk[l].cpu().numpy()[b, 0], cand[o_sel], sl, wl.K, labels=cand, what=f"layer {l}")
+        g_topk = layer_topk(l).cpu().numpy()[b:b + 1]
         o_out, o_lse = orc.sparse_attn(one(qd["q"][l]), o_kv, np.zeros(1, np.int64), g_topk, one(qd["swa"][l]),
                                        one(qd["swa_start"]), one(qd["q_pos"]), SM, window=wl.window)
-        assert_attn_close(step.out[l].cpu().numpy()[b:b + 1], o_out, what=f"layer {l} ({mode})")
-        assert np.abs(step.lse[l].cpu().numpy()[b:b + 1] - o_lse).max() < 1e-2
+        assert_attn_close(out[l].cpu().numpy()[b:b + 1], o_out, what=f"layer {l} ({mode})")
+        assert np.abs(lse[l].cpu().numpy()[b:b + 1] - o_lse).max() < 1e-2
 
 
 def test_io_step_matches_device_step():
