@@ -296,11 +296,6 @@ __device__ __forceinline__ void tmem_scale_cols(uint32_t taddr, int NQ, const fl
   }
 }
 
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
 // Barrier over every thread of every CTA of the cluster; orders shared::cluster stores
 // before it with loads after it.
 __device__ __forceinline__ void cluster_sync_all() {
@@ -341,7 +336,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int C = a.csize;
-  const int rank = C > 1 ? (int)cluster_ctarank() : 0;
+  const int rank = C > 1 ? (int)tc::cluster_ctarank() : 0;
   const int bq = blockIdx.y / a.hgroups;
   const int b = bq / a.Q;
   const int H = a.H;                                 // heads of the query (output layout)

@@ -1084,6 +1084,279 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
   if (C > 1) cluster.sync();  // keep every CTA's shared memory alive until remote reads are done
 }
 
+// Selection of lists held in registers: a query's keys are split over a cluster of C CTAs
+// (C = 1 .. 8, the cluster's x dimension), CTA r holding keys [r * 1024 * KPT, (r + 1) * 1024 *
+// KPT), thread t of it KPT consecutive keys, so (rank, thread, slot) order is index order.
+// Same radix levels, tie rule and output order as select_kernel.  Per level: every CTA counts
+// its keys into one of two histograms, one cluster barrier, then each thread sums its bin over
+// the cluster (distributed shared memory) and clears the other histogram (the one the
+// cluster read on the level before, which every CTA has finished reading by this barrier),
+// and one warp finds the bin.  The key range and the output positions take one cluster
+// exchange each.
+template <int KPT>
+__global__ void __launch_bounds__(1024, 1) select_cl_kernel(SelectArgs a) {
+  static_assert(KPT % 4 == 0, "keys are loaded 16 bytes at a time");
+  constexpr int NT = 1024;
+  chain_launch_dependents();
+  __shared__ uint32_t hist[2][kBins];   // this CTA's counts, alternating per level
+  __shared__ uint32_t hsum[kBins];      // the cluster's counts of the current level
+  __shared__ uint32_t wred[3][32];      // per-warp min, max, count of valid keys
+  __shared__ uint32_t wsum[2][32];      // per-warp totals of taken / tied keys
+  __shared__ uint32_t xch[8];           // exported to the cluster: min, max, count; taken, tied
+  __shared__ uint32_t lvl[4];           // bin found, keys above it, keys in it
+  __shared__ int32_t blk[CSA2_MAX_K];   // Reindex block ids of the query
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int C = a.csize;
+  const int rank = C > 1 ? (int)tc::cluster_ctarank() : 0;
+  const int bq = blockIdx.y;
+  const int b = bq / a.Q;
+  const int K = a.K;
+  hist[0][tid] = 0u;
+  chain_wait();
+  auto cluster_sync = [&]() {
+    if (C > 1) {
+      asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    } else {
+      __syncthreads();
+    }
+  };
+  // word w of `arr` in CTA r of the cluster
+  auto remote = [&](const uint32_t* arr, int w, int r) {
+    return tc::ld_cluster_u32(tc::mapa(tc::smem_u32(arr + w), (uint32_t)r));
+  };
+
+  int n;  // keys of this query (at most C * 1024 * KPT, checked by the host)
+  if (a.mode == kMerge) {
+    n = (int)a.n_items;
+  } else {
+    const int64_t base = a.seq_base[b];
+    int64_t nv = a.n_vis[bq];
+    if (nv < 0 || nv > a.max_n_vis || base < 0 || base + nv > a.pool_entries) nv = 0;
+    if (a.mode == kFlat)
+      n = (int)nv;
+    else if (a.mode == kHier)
+      n = (int)((nv + a.block - 1) >> a.block_shift);
+    else
+      n = a.n_blocks * a.block;
+  }
+  if (a.mode == kReindex)
+    for (int i = tid; i < a.n_blocks; i += NT) blk[i] = a.blocks[(int64_t)bq * a.n_blocks + i];
+
+  // ---- keys into registers; the range of the valid (non-zero) keys ---------------------------
+  const uint32_t* keys = a.keys + (int64_t)bq * a.key_stride;
+  const int i0 = rank * NT * KPT + tid * KPT;
+  uint32_t k[KPT];
+#pragma unroll
+  for (int u = 0; u < KPT / 4; ++u) {
+    const int i = i0 + 4 * u;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (i + 4 <= n) {
+      v = *reinterpret_cast<const uint4*>(keys + i);
+    } else if (i < n) {
+      v.x = keys[i];
+      v.y = i + 1 < n ? keys[i + 1] : 0u;
+      v.z = i + 2 < n ? keys[i + 2] : 0u;
+    }
+    k[4 * u] = v.x;
+    k[4 * u + 1] = v.y;
+    k[4 * u + 2] = v.z;
+    k[4 * u + 3] = v.w;
+  }
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u, cnt = 0u;
+#pragma unroll
+  for (int e = 0; e < KPT; ++e) {
+    if (k[e] != 0u) {
+      kmin = min(kmin, k[e]);
+      kmax = max(kmax, k[e]);
+      ++cnt;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  }
+  if (lane == 0) {
+    wred[0][warp] = kmin;
+    wred[1][warp] = kmax;
+    wred[2][warp] = cnt;
+  }
+  __syncthreads();
+  // every warp reduces the warps' partials, lane w taking warp w's
+  uint32_t gmin = wred[0][lane], gmax = wred[1][lane], gcnt = wred[2][lane];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    gmin = min(gmin, __shfl_xor_sync(0xffffffffu, gmin, o));
+    gmax = max(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
+    gcnt += __shfl_xor_sync(0xffffffffu, gcnt, o);
+  }
+  if (C > 1) {  // the cluster's range: lane r < C reads CTA r's
+    if (tid == 0) {
+      xch[0] = gmin;
+      xch[1] = gmax;
+      xch[2] = gcnt;
+    }
+    cluster_sync();
+    uint32_t rmin = 0xFFFFFFFFu, rmax = 0u, rcnt = 0u;
+    if (lane < C) {
+      rmin = remote(xch, 0, lane);
+      rmax = remote(xch, 1, lane);
+      rcnt = remote(xch, 2, lane);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      rmin = min(rmin, __shfl_xor_sync(0xffffffffu, rmin, o));
+      rmax = max(rmax, __shfl_xor_sync(0xffffffffu, rmax, o));
+      rcnt += __shfl_xor_sync(0xffffffffu, rcnt, o);
+    }
+    gmin = rmin;
+    gmax = rmax;
+    gcnt = rcnt;
+  }
+
+  // ---- radix levels --------------------------------------------------------------------------
+  uint32_t prefix = 0u, mask = 0u, need = (uint32_t)K;
+  const bool all_valid = gcnt <= (uint32_t)K;
+  if (!all_valid) {
+    if (gmin == gmax) {
+      prefix = gmin;  // every valid key is equal: ties only
+      mask = 0xFFFFFFFFu;
+    } else {
+      int p = 31 - __clz(gmin ^ gmax);  // highest bit where keys differ
+      mask = p == 31 ? 0u : ~((2u << p) - 1u);
+      prefix = gmin & mask;
+      int cur = 0;
+      for (;;) {
+        const int sh = p >= kDigitBits - 1 ? p - (kDigitBits - 1) : 0;
+        const uint32_t nb = 1u << (p - sh + 1);
+        uint32_t* h = hist[cur];
+#pragma unroll
+        for (int e = 0; e < KPT; ++e) {
+          const uint32_t key = k[e];
+          if (key != 0u && (key & mask) == prefix) atomicAdd(&h[(key >> sh) & (nb - 1u)], 1u);
+        }
+        const uint32_t* hs = h;
+        if (C > 1) {
+          cluster_sync();  // every CTA's counts are in; the other histogram is read by no one
+          uint32_t sum = 0u;
+          if (tid < (int)nb) {
+            uint32_t v[kMaxCluster];
+#pragma unroll
+            for (int r = 0; r < kMaxCluster; ++r) v[r] = r < C ? remote(h, tid, r) : 0u;
+#pragma unroll
+            for (int r = 0; r < kMaxCluster; ++r) sum += v[r];
+          }
+          hsum[tid] = sum;
+          hs = hsum;
+        }
+        hist[cur ^ 1][tid] = 0u;  // the next level's counters
+        __syncthreads();
+        if (warp == 0) {
+          find_bin_warp(hs, (int)nb, need, &lvl[0], &lvl[1]);
+          __syncwarp();
+          if (lane == 0) lvl[2] = hs[lvl[0]];
+        }
+        __syncthreads();
+        const uint32_t T = lvl[0], inbin = lvl[2];
+        need -= lvl[1];
+        prefix |= T << sh;
+        mask |= (nb - 1u) << sh;
+        if (inbin == need || sh == 0) break;  // every key of the bin is taken, or keys are equal
+        p = sh - 1;
+        cur ^= 1;
+      }
+    }
+  }
+
+  // ---- output: taken keys in index order, then the first `need` keys tied at the cut --------
+  // a valid key is taken when key & mask > prefix (every valid key when all_valid) and tied
+  // at the cut when key & mask == prefix
+  uint32_t my_gt = 0u, my_eq = 0u;
+#pragma unroll
+  for (int e = 0; e < KPT; ++e) {
+    const uint32_t kp = k[e] & mask;
+    if (k[e] != 0u && (all_valid || kp >= prefix)) {
+      if (all_valid || kp > prefix) ++my_gt;
+      else ++my_eq;
+    }
+  }
+  // block scan: warp-inclusive sums, then a scan over the warps' totals (lane w: warp w)
+  uint32_t ig = my_gt, ie = my_eq;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t yg = __shfl_up_sync(0xffffffffu, ig, o);
+    const uint32_t ye = __shfl_up_sync(0xffffffffu, ie, o);
+    if (lane >= o) {
+      ig += yg;
+      ie += ye;
+    }
+  }
+  if (lane == 31) {
+    wsum[0][warp] = ig;
+    wsum[1][warp] = ie;
+  }
+  __syncthreads();
+  uint32_t sg = wsum[0][lane], se = wsum[1][lane];
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t yg = __shfl_up_sync(0xffffffffu, sg, o);
+    const uint32_t ye = __shfl_up_sync(0xffffffffu, se, o);
+    if (lane >= o) {
+      sg += yg;
+      se += ye;
+    }
+  }
+  const uint32_t cta_g = __shfl_sync(0xffffffffu, sg, 31), cta_e = __shfl_sync(0xffffffffu, se, 31);
+  uint32_t lg = (warp > 0 ? __shfl_sync(0xffffffffu, sg, (warp - 1) & 31) : 0u) + ig - my_gt;
+  uint32_t le = (warp > 0 ? __shfl_sync(0xffffffffu, se, (warp - 1) & 31) : 0u) + ie - my_eq;
+  uint32_t G = cta_g;  // taken keys of the whole query
+  if (C > 1) {  // this CTA's items follow those of the lower ranks
+    if (tid == 0) {
+      xch[4] = cta_g;
+      xch[5] = cta_e;
+    }
+    cluster_sync();
+    uint32_t rg = lane < C ? remote(xch, 4, lane) : 0u, re = lane < C ? remote(xch, 5, lane) : 0u;
+    const uint32_t below_g = lane < rank ? rg : 0u, below_e = lane < rank ? re : 0u;
+    uint32_t bg = below_g, be = below_e;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      bg += __shfl_xor_sync(0xffffffffu, bg, o);
+      be += __shfl_xor_sync(0xffffffffu, be, o);
+      rg += __shfl_xor_sync(0xffffffffu, rg, o);
+    }
+    lg += bg;
+    le += be;
+    G = rg;
+  }
+  const uint32_t tie0 = (uint32_t)K - need;  // first slot of the tied keys
+  int32_t* out = a.out_idx + (int64_t)bq * K;
+  float* out_s = a.out_score ? a.out_score + (int64_t)bq * K : nullptr;
+#pragma unroll
+  for (int e = 0; e < KPT; ++e) {
+    const uint32_t key = k[e];
+    const uint32_t kp = key & mask;
+    if (key != 0u && (all_valid || kp >= prefix)) {  // taken, or tied at the cut
+      const bool gt = all_valid || kp > prefix;
+      if (gt || le < need) {
+        const uint32_t slot = gt ? lg : tie0 + le;
+        out[slot] = (int32_t)item_label(a, blk, i0 + e);
+        if (out_s) out_s[slot] = key_score(key);
+      }
+      if (gt) ++lg;
+      else ++le;
+    }
+  }
+  if (all_valid && rank == 0) {
+    for (int i = (int)G + tid; i < K; i += NT) {
+      out[i] = -1;
+      if (out_s) out_s[i] = -INFINITY;
+    }
+  }
+  if (C > 1) cluster_sync();  // keep this CTA's shared memory until the cluster has read it
+}
+
 // ------------------------------------------------------------------------------------
 // host launchers
 // ------------------------------------------------------------------------------------
@@ -1200,11 +1473,33 @@ static cudaError_t launch_stream(ScanArgs a, int64_t items, int B, cudaStream_t 
 
 // Selection of the K best of `items` keys per query row (blockIdx.y = row).
 static cudaError_t launch_select(SelectArgs s, int64_t items, int BQ, cudaStream_t stream) {
-  // At most 4,096 keys: one CTA with 4 keys per thread.  Otherwise one CTA per 16,384 keys
-  // (16 per thread), up to 8.  (Splitting a 16,384-key list over a cluster of 4-key CTAs
-  // measured no faster: each radix level then waits on two cluster barriers and a
-  // remote histogram sum, which cost what the shorter count saves.)
   cudaError_t e;
+  // Lists whose keys fit the registers of a cluster of at most 8 CTAs, when the clusters of all
+  // queries fit two waves: the fewest keys per thread (the most CTAs) that do.  A cluster of
+  // 16-key CTAs (lists above 16,384 keys) measured slower than select_kernel (19.4 against
+  // 16.5 us for 131,072 keys: each level's cluster barrier and histogram sum cost about a
+  // microsecond), so those lists stay with select_kernel.
+  {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    for (int kpt = 4; kpt <= 16; kpt *= 2) {
+      const int64_t c = (items + 1024 * kpt - 1) / (1024 * kpt);
+      if (c > kMaxCluster || (c > 1 && (int64_t)BQ * c > 2 * (int64_t)sms) || (kpt == 16 && c > 1)) continue;
+      s.csize = (int)(c < 1 ? 1 : c);
+      const dim3 grid((unsigned)s.csize, (unsigned)BQ);
+      const unsigned cl = s.csize > 1 ? (unsigned)s.csize : 0u;
+      if (kpt == 4)
+        e = launch_chained(select_cl_kernel<4>, grid, dim3(1024), 0, stream, cl, s);
+      else if (kpt == 8)
+        e = launch_chained(select_cl_kernel<8>, grid, dim3(1024), 0, stream, cl, s);
+      else
+        e = launch_chained(select_cl_kernel<16>, grid, dim3(1024), 0, stream, cl, s);
+      if (e != cudaSuccess) return e;
+      return cudaGetLastError();
+    }
+  }
+  // Otherwise select_kernel, which stages chunks of keys in shared memory: one CTA for at most
+  // 4,096 keys, else one CTA per 16,384 keys, up to 8.
   if (items <= SelShape<2>::kChunk) {
     s.csize = 1;
     e = cudaFuncSetAttribute(select_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, SelShape<2>::kSmem);

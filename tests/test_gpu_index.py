@@ -348,3 +348,28 @@ def test_flat_1m_ties_prefer_lower_index(orc):
     assert np.array_equal(np_u8(ikp), o_ik)
     o_topk, _ = orc.index_full(q.numpy(), w.numpy(), o_ik, np.zeros(1, np.int64), np.array([[T]], np.int32), 300)
     assert sorted(o_topk[0, 0].tolist()) == want
+
+
+@pytest.mark.parametrize("T", [12000, 30000, 60000])
+def test_cluster_select_ties_across_ctas(orc, T):
+    """Lists held in the registers of a cluster of CTAs (3 to 8 CTAs of 4 or 8 keys per thread):
+    entries [0, 7000) score -128, 100 entries near the end score 128 and the rest 0, so the
+    Top-2048 is the 100 positive keys and the 1948 lowest-index zero keys, 7000..8947, which
+    cross the CTA boundary at 8192 (CTAs hold 4096 or 8192 keys)."""
+    kv = torch.zeros(T, 512, dtype=torch.bfloat16, device="cuda")
+    ik = torch.zeros(T, 128, dtype=torch.bfloat16, device="cuda")
+    ik[:7000] = -1.0
+    ik[T - 150:T - 50] = 1.0
+    kvp = torch.empty(T, 288, dtype=torch.uint8, device="cuda")
+    ikp = torch.zeros(T, 68, dtype=torch.uint8, device="cuda")
+    csa2.csa2_pack_kv(kv, ik, 1, kvp, ikp)
+    q = torch.stack([torch.ones(128), -torch.ones(128)]).reshape(1, 1, 2, 128)
+    w = torch.tensor([1.0, -1.0]).reshape(1, 1, 2)
+    topk, _, st = run_full(q.cuda(), w.cuda(), ikp, torch.zeros(1, dtype=torch.int64, device="cuda"),
+                           torch.tensor([[T]], dtype=torch.int32, device="cuda"), 2048, T)
+    assert st == 0
+    want = list(range(7000, 8948)) + list(range(T - 150, T - 50))
+    assert sorted(topk[0, 0].tolist()) == want
+    _, o_ik = orc.pack_kv(np.zeros((T, 512), np.uint16), bf16_bits(ik), 1)
+    o_topk, _ = orc.index_full(q.numpy(), w.numpy(), o_ik, np.zeros(1, np.int64), np.array([[T]], np.int32), 2048)
+    assert sorted(o_topk[0, 0].tolist()) == want
