@@ -1366,14 +1366,16 @@ static int pow2_at_least(int x) {
   return p;
 }
 
-// Reindex scan: one CTA row per (sequence, query), two 128-candidate tiles per CTA.
+// Reindex scan: one CTA row per (sequence, query), one 128-candidate tile per CTA (512 CTAs
+// for 4 queries of 16,384 candidates fit one wave; two tiles per CTA measured 4% slower on the
+// whole hier1m step, each CTA's chain then holding two build -> MMA -> epilogue rounds).
 static cudaError_t launch_reindex_scan(ScanArgs a, int64_t items, int BQ, cudaStream_t st) {
   a.hipad = a.HI <= 4 ? 4 : (a.HI <= 8 ? 8 : 16);
   a.G = 1;
   a.n_groups = a.Q;
   a.N = a.hipad * 4;
   a.tmem_cols = pow2_at_least(a.N);
-  a.tiles_per_cta = 2;
+  a.tiles_per_cta = 1;
   const int64_t per_cta = (int64_t)a.tiles_per_cta * kRows;
   const dim3 grid((unsigned)((items + per_cta - 1) / per_cta), (unsigned)BQ);
   if (grid.x == 0 || grid.y == 0) return cudaSuccess;
