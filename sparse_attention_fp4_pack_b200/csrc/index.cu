@@ -1514,14 +1514,15 @@ static cudaError_t launch_select(SelectArgs s, int64_t items, int BQ, cudaStream
     e = launch_chained(select_kernel<2>, dim3((unsigned)s.csize, (unsigned)BQ), dim3(kSelThreads),
                        SelShape<2>::kSmem, stream, (unsigned)s.csize, s);
   } else {
-    // one CTA per 16,384 keys, up to a cluster of 8; when the queries alone fill the GPU
-    // for more than two waves, fewer CTAs per query (each walks several chunks), since a
-    // wide cluster then only adds waves and cluster barriers
+    // one CTA per 16,384 keys, up to a cluster of 8; when the queries' clusters would not fit
+    // one wave (one CTA per SM), fewer CTAs per query, each walking several chunks: a second
+    // wave costs more than the longer walk (full128k, 32 queries of 131,072 keys: 4 CTAs per
+    // query measured 7% faster on the whole step than 8)
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int64_t c = (items + SelShape<4>::kChunk - 1) / SelShape<4>::kChunk;
     c = c < 1 ? 1 : (c > kMaxCluster ? kMaxCluster : c);
-    const int64_t fit = (2 * (int64_t)sms) / (BQ > 0 ? BQ : 1);  // CTAs per query in two waves
+    const int64_t fit = (int64_t)sms / (BQ > 0 ? BQ : 1);  // CTAs per query in one wave
     if (c > fit) c = fit < 1 ? 1 : (fit >= 8 ? 8 : (fit >= 4 ? 4 : (fit >= 2 ? 2 : 1)));
     s.csize = (int)c;
     e = cudaFuncSetAttribute(select_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, SelShape<4>::kSmem);
