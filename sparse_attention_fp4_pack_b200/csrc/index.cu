@@ -649,13 +649,14 @@ constexpr int kMaxCluster = 8;
 // A CTA holds at most 2^20 keys (the host caps max_n_vis at 2^23, a query gets up to 8
 // CTAs), so no 32-bit counter can overflow.
 constexpr int kSubWords = kBins > 2 * CSA2_MAX_K ? kBins : 2 * CSA2_MAX_K;
+constexpr int kCand = 4096;  // keys of the cut bin a multi-chunk CTA keeps in shared memory
 template <int PS>
 struct SelShape {
   static constexpr int kPer = 1 << PS;                  // keys per thread per chunk
   static constexpr int kChunk = kSelThreads * kPer;     // keys per CTA per chunk
   static constexpr int kKeyRow = kPer + 1;              // a thread's keys in shared memory, padded
   static constexpr int kKeyWords = kSelThreads * kKeyRow;
-  static constexpr int kSmem = (kSubWords + kKeyWords + 2 * kBins + 128 + 64 + CSA2_MAX_K) * 4;
+  static constexpr int kSmem = (kSubWords + kKeyWords + 2 * kBins + 128 + 64 + CSA2_MAX_K + (PS >= 4 ? 2 * kCand : 0)) * 4;
 };
 static_assert(2 * CSA2_MAX_K <= kSubWords, "selected items are staged in the counter area");
 
@@ -865,6 +866,161 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
     }
     __syncthreads();
   };
+  // ---- one CTA walking several chunks: two passes over the keys ------------------------------
+  // Pass 1 counts the top 10 bits (sign, exponent, one mantissa bit) of every valid key; the
+  // bin holding the K-th largest is the cut.  Pass 2 writes every key above that bin straight
+  // to its slot (index order, per-chunk block prefixes) and copies the bin's keys, with their
+  // item indices and in index order, into shared memory; the remaining radix levels and the
+  // tied keys are resolved on that list.  The bin's keys must fit the list (kCand); when they
+  // do not, the counters are cleared and the general path below runs instead.  Against the
+  // general path (a range pass, one pass per level, a counting pass and an output pass, each
+  // reloading every chunk) this reads the keys twice instead of about six times.
+  if (C == 1 && nchunks > 1) {
+    uint32_t* candk = reinterpret_cast<uint32_t*>(blk + CSA2_MAX_K);  // [kCand] keys of the cut bin
+    int32_t* candi = reinterpret_cast<int32_t*>(candk + kCand);        // [kCand] their item indices
+    uint32_t cnt = 0u;
+    for (int ch = 0; ch < nchunks; ++ch) {
+      load_chunk(ch, false);
+#pragma unroll 4
+      for (int e = 0; e < kPer; ++e) {
+        const uint32_t key = mk[e];
+        if (key != 0u) {
+          atomicAdd(&sub[key >> 22], 1u);
+          ++cnt;
+        }
+      }
+    }
+    uint64_t tot;
+    block_excl_scan64((uint64_t)cnt, scan_ws, &tot);  // also orders the counts before the search
+    const bool all_valid = tot <= (uint64_t)K;
+    uint32_t T1 = 0u, above1 = 0u, inbin1 = 0u;
+    if (!all_valid) {
+      if (tid < 32) {
+        find_bin_warp(sub, kBins, (uint32_t)K, &misc[0], &misc[1]);
+        __syncwarp();
+        if (tid == 0) misc[2] = sub[misc[0]];
+      }
+      __syncthreads();
+      T1 = misc[0];
+      above1 = misc[1];
+      inbin1 = misc[2];
+    }
+    if (all_valid || inbin1 <= (uint32_t)kCand) {
+      int32_t* out = a.out_idx + (int64_t)bq * K;
+      float* out_s = a.out_score ? a.out_score + (int64_t)bq * K : nullptr;
+      uint32_t base_g = 0u, base_c = 0u;
+      for (int ch = 0; ch < nchunks; ++ch) {
+        load_chunk(ch, false);
+        uint32_t cg = 0u, cc = 0u;
+#pragma unroll 4
+        for (int e = 0; e < kPer; ++e) {
+          const uint32_t key = mk[e];
+          if (key != 0u) {
+            const uint32_t d = key >> 22;
+            if (all_valid || d > T1) ++cg;
+            else if (d == T1) ++cc;
+          }
+        }
+        uint64_t ctot;
+        const uint64_t cm = block_excl_scan64((uint64_t)cg | ((uint64_t)cc << 32), scan_ws, &ctot);
+        uint32_t lg = base_g + (uint32_t)cm, lc = base_c + (uint32_t)(cm >> 32);
+        const int64_t i0 = lo + (int64_t)ch * kSelChunk + (int64_t)tid * kPer;
+#pragma unroll 2
+        for (int e = 0; e < kPer; ++e) {
+          const uint32_t key = mk[e];
+          if (key == 0u) continue;
+          const uint32_t d = key >> 22;
+          if (all_valid || d > T1) {
+            out[lg] = (int32_t)item_label(a, blk, i0 + e);
+            if (out_s) out_s[lg] = key_score(key);
+            ++lg;
+          } else if (d == T1) {
+            candk[lc] = key;
+            candi[lc] = (int32_t)(i0 + e);
+            ++lc;
+          }
+        }
+        base_g += (uint32_t)ctot;
+        base_c += (uint32_t)(ctot >> 32);
+      }
+      if (all_valid) {
+        for (int i = (int)base_g + tid; i < K; i += kSelThreads) {
+          out[i] = -1;
+          if (out_s) out_s[i] = -INFINITY;
+        }
+        return;
+      }
+      // the remaining levels on the cut bin's keys, in two alternating histograms
+      const int nc = (int)base_c;
+      uint32_t need = (uint32_t)K - above1;
+      uint32_t prefix = T1 << 22, mask = 0xFFC00000u;
+      for (int i = tid; i < kBins; i += kSelThreads) {
+        hist[i] = 0u;
+        hsum[i] = 0u;
+      }
+      __syncthreads();  // the list and the cleared counters are visible
+      int p = 21, cur = 0;
+      for (;;) {
+        const int sh = p >= kDigitBits - 1 ? p - (kDigitBits - 1) : 0;
+        const uint32_t nb = 1u << (p - sh + 1);
+        uint32_t* h = cur ? hsum : hist;
+        uint32_t* hn = cur ? hist : hsum;
+        for (int i = tid; i < nc; i += kSelThreads) {
+          const uint32_t key = candk[i];
+          if ((key & mask) == prefix) atomicAdd(&h[(key >> sh) & (nb - 1u)], 1u);
+        }
+        for (int i = tid; i < kBins; i += kSelThreads) hn[i] = 0u;  // last read on the level before
+        __syncthreads();
+        if (tid < 32) {
+          find_bin_warp(h, (int)nb, need, &misc[0], &misc[1]);
+          __syncwarp();
+          if (tid == 0) misc[2] = h[misc[0]];
+        }
+        __syncthreads();
+        const uint32_t T = misc[0], inbin = misc[2];
+        need -= misc[1];
+        prefix |= T << sh;
+        mask |= (nb - 1u) << sh;
+        if (inbin == need || sh == 0) break;
+        p = sh - 1;
+        cur ^= 1;
+      }
+      // the list's taken keys after the first pass's, then its first `need` tied keys; a
+      // thread takes a contiguous run of the list, so both stay in index order
+      const int per = (nc + kSelThreads - 1) / kSelThreads;
+      const int c0 = tid * per, c1 = min(nc, c0 + per);
+      uint32_t g2 = 0u, e2 = 0u;
+      for (int i = c0; i < c1; ++i) {
+        const uint32_t kp = candk[i] & mask;
+        if (kp > prefix) ++g2;
+        else if (kp == prefix) ++e2;
+      }
+      uint64_t t2;
+      const uint64_t m2 = block_excl_scan64((uint64_t)g2 | ((uint64_t)e2 << 32), scan_ws, &t2);
+      uint32_t lg = above1 + (uint32_t)m2, le = (uint32_t)(m2 >> 32);
+      const uint32_t tie0 = (uint32_t)K - need;
+      for (int i = c0; i < c1; ++i) {
+        const uint32_t key = candk[i], kp = key & mask;
+        if (kp > prefix) {
+          out[lg] = (int32_t)item_label(a, blk, candi[i]);
+          if (out_s) out_s[lg] = key_score(key);
+          ++lg;
+        } else if (kp == prefix) {
+          if (le < need) {
+            out[tie0 + le] = (int32_t)item_label(a, blk, candi[i]);
+            if (out_s) out_s[tie0 + le] = key_score(key);
+          }
+          ++le;
+        }
+      }
+      return;
+    }
+    __syncthreads();  // every thread has read the search's result before the counters clear
+    for (int i = tid; i < kSubWords / 4; i += kSelThreads)
+      reinterpret_cast<uint4*>(sub)[i] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+  }
+
   // ---- 0. cluster-wide min / max / count of valid keys, taken while loading -------------
   for (int ch = 0; ch < nchunks; ++ch) load_chunk(ch, true);  // a single chunk stays loaded
   // phase: keys loaded

@@ -373,3 +373,34 @@ def test_cluster_select_ties_across_ctas(orc, T):
     _, o_ik = orc.pack_kv(np.zeros((T, 512), np.uint16), bf16_bits(ik), 1)
     o_topk, _ = orc.index_full(q.numpy(), w.numpy(), o_ik, np.zeros(1, np.int64), np.array([[T]], np.int32), 2048)
     assert sorted(o_topk[0, 0].tolist()) == want
+
+
+@pytest.mark.parametrize("neg", [36000, 20000])
+def test_multichunk_select_ties(orc, neg):
+    """80 queries of 40,000 keys each: the selection runs one CTA per query walking three
+    16,384-key chunks.  Entries [0, neg) score -128, the last 100 score 128 and the rest 0,
+    so the Top-300 is the 100 positive keys and the 200 lowest-index zero keys.  With 3,900
+    zero keys the cut bin fits the two-pass path's shared-memory list; with 19,900 it does not
+    and the general path runs."""
+    T, Q = 40000, 80
+    kv = torch.zeros(T, 512, dtype=torch.bfloat16, device="cuda")
+    ik = torch.zeros(T, 128, dtype=torch.bfloat16, device="cuda")
+    ik[:neg] = -1.0
+    ik[T - 100:] = 1.0
+    kvp = torch.empty(T, 288, dtype=torch.uint8, device="cuda")
+    ikp = torch.zeros(T, 68, dtype=torch.uint8, device="cuda")
+    csa2.csa2_pack_kv(kv, ik, 1, kvp, ikp)
+    q = torch.stack([torch.ones(128), -torch.ones(128)]).reshape(1, 1, 2, 128).repeat(1, Q, 1, 1)
+    w = torch.tensor([1.0, -1.0]).reshape(1, 1, 2).repeat(1, Q, 1)
+    n_vis = torch.full((1, Q), T, dtype=torch.int32, device="cuda")
+    topk, score, st = run_full(q.cuda(), w.cuda(), ikp, torch.zeros(1, dtype=torch.int64, device="cuda"), n_vis,
+                               300, T)
+    assert st == 0
+    want = list(range(neg, neg + 200)) + list(range(T - 100, T))
+    for i in range(Q):
+        assert sorted(topk[0, i].tolist()) == want, f"query {i}"
+    assert set(np.unique(score[0, 0]).tolist()) == {0.0, 128.0}
+    _, o_ik = orc.pack_kv(np.zeros((T, 512), np.uint16), bf16_bits(ik), 1)
+    o_topk, _ = orc.index_full(q[:, :1].numpy(), w[:, :1].numpy(), o_ik, np.zeros(1, np.int64),
+                               np.array([[T]], np.int32), 300)
+    assert sorted(o_topk[0, 0].tolist()) == want
