@@ -1247,8 +1247,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
 // its keys into one of two histograms, one cluster barrier, then each thread sums its bin over
 // the cluster (distributed shared memory) and clears the other histogram (the one the
 // cluster read on the level before, which every CTA has finished reading by this barrier),
-// and one warp finds the bin.  The key range and the output positions take one cluster
-// exchange each.
+// and one warp finds the bin.  The output positions take one more cluster exchange.
 template <int KPT>
 __global__ void __launch_bounds__(1024, 1) select_cl_kernel(SelectArgs a) {
   static_assert(KPT % 4 == 0, "keys are loaded 16 bytes at a time");
@@ -1256,9 +1255,9 @@ __global__ void __launch_bounds__(1024, 1) select_cl_kernel(SelectArgs a) {
   chain_launch_dependents();
   __shared__ uint32_t hist[2][kBins];   // this CTA's counts, alternating per level
   __shared__ uint32_t hsum[kBins];      // the cluster's counts of the current level
-  __shared__ uint32_t wred[3][32];      // per-warp min, max, count of valid keys
+  __shared__ uint32_t wred[3][32];      // per-warp min, max, count of valid keys (one CTA)
   __shared__ uint32_t wsum[2][32];      // per-warp totals of taken / tied keys
-  __shared__ uint32_t xch[8];           // exported to the cluster: min, max, count; taken, tied
+  __shared__ uint32_t xch[8];           // exported to the cluster: [4] taken and [5] tied keys
   __shared__ uint32_t lvl[4];           // bin found, keys above it, keys in it
   __shared__ int32_t blk[CSA2_MAX_K];   // Reindex block ids of the query
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1318,110 +1317,116 @@ __global__ void __launch_bounds__(1024, 1) select_cl_kernel(SelectArgs a) {
     k[4 * u + 2] = v.z;
     k[4 * u + 3] = v.w;
   }
-  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u, cnt = 0u;
+  // One CTA: the range of the valid keys aims the first digit at the highest bit where they
+  // differ.  A cluster skips that exchange (about 1-2 us): its first digit is the top 10 bits,
+  // and the count of valid keys comes from that level's summed histogram.
+  uint32_t gmin = 0xFFFFFFFFu, gmax = 0u, gcnt = 0u;
+  if (C == 1) {
+    uint32_t cnt = 0u;
 #pragma unroll
-  for (int e = 0; e < KPT; ++e) {
-    if (k[e] != 0u) {
-      kmin = min(kmin, k[e]);
-      kmax = max(kmax, k[e]);
-      ++cnt;
+    for (int e = 0; e < KPT; ++e) {
+      if (k[e] != 0u) {
+        gmin = min(gmin, k[e]);
+        gmax = max(gmax, k[e]);
+        ++cnt;
+      }
     }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-    cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-  }
-  if (lane == 0) {
-    wred[0][warp] = kmin;
-    wred[1][warp] = kmax;
-    wred[2][warp] = cnt;
-  }
-  __syncthreads();
-  // every warp reduces the warps' partials, lane w taking warp w's
-  uint32_t gmin = wred[0][lane], gmax = wred[1][lane], gcnt = wred[2][lane];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    gmin = min(gmin, __shfl_xor_sync(0xffffffffu, gmin, o));
-    gmax = max(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
-    gcnt += __shfl_xor_sync(0xffffffffu, gcnt, o);
-  }
-  if (C > 1) {  // the cluster's range: lane r < C reads CTA r's
-    if (tid == 0) {
-      xch[0] = gmin;
-      xch[1] = gmax;
-      xch[2] = gcnt;
-    }
-    cluster_sync();
-    uint32_t rmin = 0xFFFFFFFFu, rmax = 0u, rcnt = 0u;
-    if (lane < C) {
-      rmin = remote(xch, 0, lane);
-      rmax = remote(xch, 1, lane);
-      rcnt = remote(xch, 2, lane);
-    }
+    gcnt = cnt;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      rmin = min(rmin, __shfl_xor_sync(0xffffffffu, rmin, o));
-      rmax = max(rmax, __shfl_xor_sync(0xffffffffu, rmax, o));
-      rcnt += __shfl_xor_sync(0xffffffffu, rcnt, o);
+      gmin = min(gmin, __shfl_xor_sync(0xffffffffu, gmin, o));
+      gmax = max(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
+      gcnt += __shfl_xor_sync(0xffffffffu, gcnt, o);
     }
-    gmin = rmin;
-    gmax = rmax;
-    gcnt = rcnt;
+    if (lane == 0) {
+      wred[0][warp] = gmin;
+      wred[1][warp] = gmax;
+      wred[2][warp] = gcnt;
+    }
+    __syncthreads();
+    // every warp reduces the warps' partials, lane w taking warp w's
+    gmin = wred[0][lane];
+    gmax = wred[1][lane];
+    gcnt = wred[2][lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      gmin = min(gmin, __shfl_xor_sync(0xffffffffu, gmin, o));
+      gmax = max(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
+      gcnt += __shfl_xor_sync(0xffffffffu, gcnt, o);
+    }
   }
 
   // ---- radix levels --------------------------------------------------------------------------
   uint32_t prefix = 0u, mask = 0u, need = (uint32_t)K;
-  const bool all_valid = gcnt <= (uint32_t)K;
-  if (!all_valid) {
+  bool all_valid = C == 1 && gcnt <= (uint32_t)K;
+  int p = 31;  // highest bit of the first digit; -1: no level
+  if (C == 1 && !all_valid) {
     if (gmin == gmax) {
       prefix = gmin;  // every valid key is equal: ties only
       mask = 0xFFFFFFFFu;
+      p = -1;
     } else {
-      int p = 31 - __clz(gmin ^ gmax);  // highest bit where keys differ
+      p = 31 - __clz(gmin ^ gmax);  // highest bit where keys differ
       mask = p == 31 ? 0u : ~((2u << p) - 1u);
       prefix = gmin & mask;
-      int cur = 0;
-      for (;;) {
-        const int sh = p >= kDigitBits - 1 ? p - (kDigitBits - 1) : 0;
-        const uint32_t nb = 1u << (p - sh + 1);
-        uint32_t* h = hist[cur];
+    }
+  }
+  if (!all_valid && p >= 0) {
+    int cur = 0;
+    for (int level = 0;; ++level) {
+      const int sh = p >= kDigitBits - 1 ? p - (kDigitBits - 1) : 0;
+      const uint32_t nb = 1u << (p - sh + 1);
+      uint32_t* h = hist[cur];
 #pragma unroll
-        for (int e = 0; e < KPT; ++e) {
-          const uint32_t key = k[e];
-          if (key != 0u && (key & mask) == prefix) atomicAdd(&h[(key >> sh) & (nb - 1u)], 1u);
+      for (int e = 0; e < KPT; ++e) {
+        const uint32_t key = k[e];
+        if (key != 0u && (key & mask) == prefix) atomicAdd(&h[(key >> sh) & (nb - 1u)], 1u);
+      }
+      const uint32_t* hs = h;
+      if (C > 1) {
+        cluster_sync();  // every CTA's counts are in; the other histogram is read by no one
+        uint32_t sum = 0u;
+        if (tid < (int)nb) {
+          uint32_t v[kMaxCluster];
+#pragma unroll
+          for (int r = 0; r < kMaxCluster; ++r) v[r] = r < C ? remote(h, tid, r) : 0u;
+#pragma unroll
+          for (int r = 0; r < kMaxCluster; ++r) sum += v[r];
         }
-        const uint32_t* hs = h;
-        if (C > 1) {
-          cluster_sync();  // every CTA's counts are in; the other histogram is read by no one
-          uint32_t sum = 0u;
-          if (tid < (int)nb) {
-            uint32_t v[kMaxCluster];
+        hsum[tid] = sum;
+        hs = hsum;
+      }
+      hist[cur ^ 1][tid] = 0u;  // the next level's counters
+      __syncthreads();
+      if (warp == 0) {
+        bool few = false;
+        if (C > 1 && level == 0) {  // the cluster's count of valid keys: every one sits in a bin
+          uint32_t t = 0u;
+#pragma unroll 8
+          for (int i = 0; i < kBins / 32; ++i) t += hs[lane + 32 * i];
 #pragma unroll
-            for (int r = 0; r < kMaxCluster; ++r) v[r] = r < C ? remote(h, tid, r) : 0u;
-#pragma unroll
-            for (int r = 0; r < kMaxCluster; ++r) sum += v[r];
-          }
-          hsum[tid] = sum;
-          hs = hsum;
+          for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+          few = t <= need;
+          if (lane == 0) lvl[3] = few ? 1u : 0u;
         }
-        hist[cur ^ 1][tid] = 0u;  // the next level's counters
-        __syncthreads();
-        if (warp == 0) {
+        if (!few) {
           find_bin_warp(hs, (int)nb, need, &lvl[0], &lvl[1]);
           __syncwarp();
           if (lane == 0) lvl[2] = hs[lvl[0]];
         }
-        __syncthreads();
-        const uint32_t T = lvl[0], inbin = lvl[2];
-        need -= lvl[1];
-        prefix |= T << sh;
-        mask |= (nb - 1u) << sh;
-        if (inbin == need || sh == 0) break;  // every key of the bin is taken, or keys are equal
-        p = sh - 1;
-        cur ^= 1;
       }
+      __syncthreads();
+      if (C > 1 && level == 0 && lvl[3] != 0u) {  // at most K valid keys: every one is taken
+        all_valid = true;
+        break;
+      }
+      const uint32_t T = lvl[0], inbin = lvl[2];
+      need -= lvl[1];
+      prefix |= T << sh;
+      mask |= (nb - 1u) << sh;
+      if (inbin == need || sh == 0) break;  // every key of the bin is taken, or keys are equal
+      p = sh - 1;
+      cur ^= 1;
     }
   }
 
