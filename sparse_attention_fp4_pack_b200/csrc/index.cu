@@ -1481,6 +1481,9 @@ __global__ void __launch_bounds__(1024, 1) select_cl_kernel(SelectArgs a) {
     uint32_t rg = lane < C ? remote(xch, 4, lane) : 0u, re = lane < C ? remote(xch, 5, lane) : 0u;
     const uint32_t below_g = lane < rank ? rg : 0u, below_e = lane < rank ? re : 0u;
     uint32_t bg = below_g, be = below_e;
+    // the last remote reads of this CTA are done: arrive now, wait just before exiting (the
+    // other CTAs may still be reading this one's exchange words until they arrive)
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       bg += __shfl_xor_sync(0xffffffffu, bg, o);
@@ -1515,7 +1518,7 @@ __global__ void __launch_bounds__(1024, 1) select_cl_kernel(SelectArgs a) {
       if (out_s) out_s[i] = -INFINITY;
     }
   }
-  if (C > 1) cluster_sync();  // keep this CTA's shared memory until the cluster has read it
+  if (C > 1) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");  // see the arrive above
 }
 
 // ------------------------------------------------------------------------------------
