@@ -222,6 +222,9 @@ csa2_status csa2_reindex(const float* q, const float* w, const uint8_t* ik_pool,
  * E4M3 window tokens are exact in f16; queries (times sm_scale*log2 e) and softmax
  * probabilities are rounded to f16, so |q| * sm_scale must stay below 4e4.  An empty
  * key set gives out = 0, lse = -inf.  H in {16, 32, 48, 64}.
+ * q is read while the previous library kernel in the stream may still be running (the
+ * call's kernels are launched to overlap their predecessor's tail): it must not be an
+ * output of a libcsa2 call, which no libcsa2 call ever produces.
  * --------------------------------------------------------------------------------- */
 size_t csa2_sparse_attn_workspace_size(int B, int Q, int H, int K, int window);
 csa2_status csa2_sparse_attn(const float* q, const uint8_t* kv_pool, int64_t pool_entries,

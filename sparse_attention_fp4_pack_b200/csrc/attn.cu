@@ -328,10 +328,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
   uint64_t* mbar = reinterpret_cast<uint64_t*>(valid_s + 128);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mbar + 8);
   int32_t* idx_s = reinterpret_cast<int32_t*>(sm + kOffIdx);  // [K] Top-K entry index per slot
-  const float* Qf = reinterpret_cast<const float*>(Ks);     // fp32 query staging [NH][512]
-  // barriers: queries landed; key-tile halves written (A: dims 0-255, B: 256-511); S^T
+  // barriers (mbar[0] unused): key-tile halves written (A: dims 0-255, B: 256-511); S^T
   // ready; P^T ready; PV done
-  const uint32_t bar_q = tc::smem_u32(&mbar[0]), bar_ka = tc::smem_u32(&mbar[1]), bar_kb = tc::smem_u32(&mbar[2]);
+  const uint32_t bar_ka = tc::smem_u32(&mbar[1]), bar_kb = tc::smem_u32(&mbar[2]);
   const uint32_t bar_s = tc::smem_u32(&mbar[3]), bar_p = tc::smem_u32(&mbar[4]), bar_pv = tc::smem_u32(&mbar[5]);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -347,7 +346,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
 
   // set-up that touches no global memory runs while the predecessor finishes
   if (tid == 0) {
-    tc::mbar_init(bar_q, 1);
     tc::mbar_init(bar_ka, kWorkers);
     tc::mbar_init(bar_kb, kWorkers);
     tc::mbar_init(bar_s, 1);
@@ -359,18 +357,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
     l_run[tid] = 0.0f;
   }
   if (warp == 0) tc::tmem_alloc(tc::smem_u32(tmem_slot), kTmemCols);
+  // The queries are a caller input that no library call writes, so they are staged while the
+  // predecessor finishes: fp32 -> f16 tile scaled by sm_scale * log2(e), rows past NH zero, 8
+  // channels per chunk.  (A library kernel starts early only behind another library kernel,
+  // and whatever produced the queries before that one has completed by then.)
+  if (T > 0) {
+    const float qscale = a.sm_scale * 1.4426950408889634f;
+    const float* qg = a.q + ((int64_t)bq * H + h_base) * kD;
+#pragma unroll 4
+    for (int i = tid; i < NQ * 64; i += kWorkers) {
+      const int h = i >> 6, ch = i & 63, db = ch >> 3, c = ch & 7;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (h < NH) {
+        const float4 x0 = __ldg(reinterpret_cast<const float4*>(qg + h * kD + ch * 8));
+        const float4 x1 = __ldg(reinterpret_cast<const float4*>(qg + h * kD + ch * 8 + 4));
+        v.x = half2_bits(x0.x * qscale, x0.y * qscale);
+        v.y = half2_bits(x0.z * qscale, x0.w * qscale);
+        v.z = half2_bits(x1.x * qscale, x1.y * qscale);
+        v.w = half2_bits(x1.z * qscale, x1.w * qscale);
+      }
+      *reinterpret_cast<uint4*>(Qs + db * 8192 + tc::sw128(h, c * 16)) = v;
+    }
+    tc::fence_async_smem();
+  }
   chain_wait();
   const int64_t base = a.seq_base[b];
   const int64_t tq = a.q_pos[bq];
   const int64_t sws = a.S_w > 0 ? a.swa_start[b] : 0;
 
-  if (tid == 0) {
-    const uint32_t bytes = (uint32_t)NH * kD * 4;
-    tc::mbar_arrive_expect_tx(bar_q, bytes);
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(a.q + ((int64_t)bq * H + h_base) * kD);
-    for (uint32_t off = 0; off < bytes; off += 32768)
-      tc::bulk_g2s(tc::smem_u32(Ks) + off, src + off, bytes - off < 32768 ? bytes - off : 32768, bar_q);
-  }
   // the first tile's gather depends on one index load only; the indices of the later
   // tiles are staged by asynchronous copies
   SlotRaw sr;
@@ -426,28 +440,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
 
   {
     // ---- workers --------------------------------------------------------------------------------
-    // queries: fp32 staging -> f16 tile (scaled), rows past NH zero, 8 channels per chunk
-    bool fail = T > 0 && !tc::mbar_wait(bar_q, 0, kMaxPolls);
-    if (T > 0) {
-      const float qscale = a.sm_scale * 1.4426950408889634f;
-#pragma unroll 4
-      for (int i = tid; i < NQ * 64; i += kWorkers) {
-        const int h = i >> 6, ch = i & 63, db = ch >> 3, c = ch & 7;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (h < NH && !fail) {
-          const float4 x0 = *reinterpret_cast<const float4*>(Qf + h * kD + ch * 8);
-          const float4 x1 = *reinterpret_cast<const float4*>(Qf + h * kD + ch * 8 + 4);
-          v.x = half2_bits(x0.x * qscale, x0.y * qscale);
-          v.y = half2_bits(x0.z * qscale, x0.w * qscale);
-          v.z = half2_bits(x1.x * qscale, x1.y * qscale);
-          v.w = half2_bits(x1.z * qscale, x1.w * qscale);
-        }
-        *reinterpret_cast<uint4*>(Qs + db * 8192 + tc::sw128(h, c * 16)) = v;
-      }
-      tc::fence_async_smem();
-    }
-    // the staging is read before any key row overwrites it
-    timed_out = tc::named_sync_or(kWorkerBar, kWorkers, fail);
+    bool fail = false;
 
     const int q4 = warp & 3, half = warp >> 2;
     const int key = q4 * 32 + lane;                   // this thread's TMEM lane (tile row)

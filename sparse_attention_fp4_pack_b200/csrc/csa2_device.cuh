@@ -23,8 +23,10 @@ constexpr int kIkBytes = CSA2_IK_ENTRY_BYTES;
 // stream serialization, so its CTAs may be scheduled while the previous kernel in the
 // stream is still running.  Each kernel starts with chain_enter: it lets its own successor
 // begin launching, then waits until its predecessor has completed and that kernel's
-// writes are visible, before it touches global memory.  What overlaps is the launch and
-// CTA scheduling, not any data access.
+// writes are visible, before it touches global memory that a library kernel writes.  What
+// overlaps is the launch, CTA scheduling and on-chip set-up, plus (attention) the staging
+// of the queries: a caller input that no library kernel writes, whose producer has always
+// completed by then (a kernel starts early only behind a library kernel).
 __device__ __forceinline__ void chain_enter() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
