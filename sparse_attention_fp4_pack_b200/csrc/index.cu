@@ -131,42 +131,8 @@ __global__ void __launch_bounds__(kScanThreads) reindex_scan_kernel(ScanArgs a) 
   // set-up that touches no global memory runs while the predecessor finishes
   if (warp == 0) tc::tmem_alloc(tc::smem_u32(tmem_slot), a.tmem_cols);
   if (tid == 32) tc::mbar_init(tc::smem_u32(mbar), 1);
-  chain_wait();
-  const int64_t nvis = valid_count(a, b, bq, blockIdx.x == 0);  // 0 if the count is bad
-
-  const uint8_t* seq = a.ik_pool + a.seq_base[b] * kIkBytes;
-  const uint32_t raw_a = tc::smem_u32(raw);
-  // a tile's 128 / block gathered blocks, each staged at seg_stride (a 16 B multiple)
-  const int seg_stride = ((a.block * kIkBytes + 16) + 15) & ~15;
-
-  // gathered tile loader: tile ti into buffer ti & 1; `block` threads copy each block
-  auto load_tile = [&](int ti) {
-    const int64_t i0 = item0 + (int64_t)ti * kRows;
-    const uint32_t dst = raw_a + (ti & 1) * kRawBytes;
-    const int s = tid >> a.block_shift, sub = tid & (a.block - 1);
-    const int64_t slot_blk = (i0 >> a.block_shift) + s;
-    int32_t c = -1;
-    if (slot_blk < a.n_blocks) c = a.blocks[(int64_t)bq * a.n_blocks + slot_blk];
-    if (sub == 0) {
-      segc[(ti & 1) * 128 + s] = c;
-      if (c < -1) flag(a.status, CSA2_DEV_BAD_INDEX);
-    }
-    int cnt = 0;
-    if (c >= 0) {
-      const int64_t rem = nvis - (int64_t)c * a.block;
-      cnt = rem <= 0 ? 0 : (int)(rem < a.block ? rem : a.block);
-    }
-    if (cnt > 0) {
-      // a block starts at its own address residue mod 16 unless block*68 is a 16 B multiple
-      const uint8_t* src = seq + (int64_t)c * a.block * kIkBytes;
-      const int smis = (int)(reinterpret_cast<uintptr_t>(src) & 15u);
-      stage_async(dst + s * seg_stride + smis, src, cnt * kIkBytes, sub, a.block);
-    }
-    tc::cp_async_commit();
-  };
-
-  // The B operand's query rows and weights are loaded first, so their latency overlaps the
-  // block-id loads the first tile's gather waits for; a warp takes HIPAD / 4 heads.
+  // The B operand (the indexer queries and head weights: caller inputs that no library call
+  // writes) is built while the predecessor finishes; a warp takes HIPAD / 4 heads.
   constexpr int kHeadsPerWarp = HIPAD / (kScanThreads / 32);
   float4 qpre[kHeadsPerWarp];
   float wpre[kHeadsPerWarp];
@@ -180,8 +146,6 @@ __global__ void __launch_bounds__(kScanThreads) reindex_scan_kernel(ScanArgs a) 
       wpre[k] = a.w[(int64_t)bq * a.HI + h];
     }
   }
-  load_tile(0);  // the first tile's copies overlap the set-up below
-
   // ---- B operand: four int8 limbs of every head, plus epilogue constants ----------------
 #pragma unroll
   for (int k = 0; k < kHeadsPerWarp; ++k) {
@@ -223,6 +187,43 @@ __global__ void __launch_bounds__(kScanThreads) reindex_scan_kernel(ScanArgs a) 
     }
     if (lane == 0) wq[h] = S > 0.f ? wpre[k] / (2.0f * S) : 0.f;
   }
+  tc::fence_async_smem();
+  chain_wait();
+  const int64_t nvis = valid_count(a, b, bq, blockIdx.x == 0);  // 0 if the count is bad
+
+  const uint8_t* seq = a.ik_pool + a.seq_base[b] * kIkBytes;
+  const uint32_t raw_a = tc::smem_u32(raw);
+  // a tile's 128 / block gathered blocks, each staged at seg_stride (a 16 B multiple)
+  const int seg_stride = ((a.block * kIkBytes + 16) + 15) & ~15;
+
+  // gathered tile loader: tile ti into buffer ti & 1; `block` threads copy each block
+  auto load_tile = [&](int ti) {
+    const int64_t i0 = item0 + (int64_t)ti * kRows;
+    const uint32_t dst = raw_a + (ti & 1) * kRawBytes;
+    const int s = tid >> a.block_shift, sub = tid & (a.block - 1);
+    const int64_t slot_blk = (i0 >> a.block_shift) + s;
+    int32_t c = -1;
+    if (slot_blk < a.n_blocks) c = a.blocks[(int64_t)bq * a.n_blocks + slot_blk];
+    if (sub == 0) {
+      segc[(ti & 1) * 128 + s] = c;
+      if (c < -1) flag(a.status, CSA2_DEV_BAD_INDEX);
+    }
+    int cnt = 0;
+    if (c >= 0) {
+      const int64_t rem = nvis - (int64_t)c * a.block;
+      cnt = rem <= 0 ? 0 : (int)(rem < a.block ? rem : a.block);
+    }
+    if (cnt > 0) {
+      // a block starts at its own address residue mod 16 unless block*68 is a 16 B multiple
+      const uint8_t* src = seq + (int64_t)c * a.block * kIkBytes;
+      const int smis = (int)(reinterpret_cast<uintptr_t>(src) & 15u);
+      stage_async(dst + s * seg_stride + smis, src, cnt * kIkBytes, sub, a.block);
+    }
+    tc::cp_async_commit();
+  };
+
+  load_tile(0);
+
   tc::fence_async_smem();
   tc::fence_before_sync();
   __syncthreads();
