@@ -130,6 +130,30 @@ __device__ __forceinline__ uint32_t e4m3_scale_f16x2(uint32_t byte) {
   return h;
 }
 
+// The same for 8 values per lane: 3 exchange steps within each group of 8 lanes leave lane i
+// with value i mod 8 reduced over its 8 lanes; two more exchanges add the other groups.
+template <bool kMax>
+__device__ __forceinline__ float xpose_reduce8(float (&v)[8], int lane) {
+#pragma unroll
+  for (int n = 4; n >= 1; n >>= 1) {
+    const bool upper = (lane & n) != 0;
+#pragma unroll
+    for (int j = 0; j < n; ++j) {
+      const float send = upper ? v[j] : v[j + n];
+      const float keep = upper ? v[j + n] : v[j];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, n);
+      v[j] = kMax ? fmaxf(keep, recv) : keep + recv;
+    }
+  }
+  float x = v[0];
+#pragma unroll
+  for (int o = 8; o <= 16; o <<= 1) {
+    const float other = __shfl_xor_sync(0xffffffffu, x, o);
+    x = kMax ? fmaxf(x, other) : x + other;
+  }
+  return x;
+}
+
 // Reduce 32 values per lane across the warp so that lane i ends with the reduction of
 // value i over all 32 lanes (5 halving exchange steps, 31 shuffles).
 template <bool kMax>
@@ -147,26 +171,6 @@ __device__ __forceinline__ float xpose_reduce(float (&v)[32], int lane) {
   }
   return v[0];
 }
-
-// The same for 16 values: 4 exchange steps within each half-warp leave lane i with value
-// i mod 16 reduced over its 16 lanes; one more exchange adds the other half-warp.
-template <bool kMax>
-__device__ __forceinline__ float xpose_reduce16(float (&v)[16], int lane) {
-#pragma unroll
-  for (int n = 8; n >= 1; n >>= 1) {
-    const bool upper = (lane & n) != 0;
-#pragma unroll
-    for (int j = 0; j < n; ++j) {
-      const float send = upper ? v[j] : v[j + n];
-      const float keep = upper ? v[j + n] : v[j];
-      const float recv = __shfl_xor_sync(0xffffffffu, send, n);
-      v[j] = kMax ? fmaxf(keep, recv) : keep + recv;
-    }
-  }
-  const float other = __shfl_xor_sync(0xffffffffu, v[0], 16);
-  return kMax ? fmaxf(v[0], other) : v[0] + other;
-}
-
 
 // One key slot's raw data for this thread's half of the 512 channels: dim-blocks
 // d_i = 2i + hf (i = 0..3) of 64 channels.  Entry: codes of block d_i in v[2i], v[2i+1]
@@ -445,8 +449,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
     const int q4 = warp & 3, half = warp >> 2;
     const int key = q4 * 32 + lane;                   // this thread's TMEM lane (tile row)
     const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
-    const bool s_cols = half * 32 < NQ;               // this warp holds S^T columns
-    const int ncols = NQ == 16 ? 16 : 32;             // of them, when it does
+    // S^T columns of this warp: with 16 heads, 8 in each half of the warps; else 32 per warp
+    // of the halves that hold any
+    const bool s_cols = NQ == 16 || half * 32 < NQ;
+    const int ncols = NQ == 16 ? 8 : 32;
+    const int col0 = NQ == 16 ? half * 8 : half * 32;
     for (int k = 0; k < T && !timed_out; ++k) {
       const uint32_t par = (uint32_t)k & 1u;
       const int tile = rank + k * C;
@@ -496,22 +503,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {  // the four partial sums of S^T
           uint32_t raw[32];
-          if (ncols == 16) tc::tmem_ld16(lane_base + kColS + 64 * i, raw);
-          else tc::tmem_ld32(lane_base + kColS + 64 * i + half * 32, raw);
+          if (NQ == 16) tc::tmem_ld8(lane_base + kColS + 64 * i + col0, raw);
+          else tc::tmem_ld32(lane_base + kColS + 64 * i + col0, raw);
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) s[jj] += jj < ncols ? __uint_as_float(raw[jj]) : 0.0f;
         }
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) {
-          s[jj] = (jj < ncols && kv && half * 32 + jj < NH) ? s[jj] : -INFINITY;
+          s[jj] = (jj < ncols && kv && col0 + jj < NH) ? s[jj] : -INFINITY;
           v[jj] = s[jj];
         }
-        if (ncols == 16) {
-          float v16[16];
+        if (NQ == 16) {
+          float v8[8];
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) v16[jj] = v[jj];
-          const float m16 = xpose_reduce16<true>(v16, lane);
-          if (lane < 16) red_max[q4 * 64 + lane] = m16;
+          for (int jj = 0; jj < 8; ++jj) v8[jj] = v[jj];
+          const float m8 = xpose_reduce8<true>(v8, lane);
+          if (lane < 8) red_max[q4 * 64 + col0 + lane] = m8;
         } else {
           red_max[q4 * 64 + half * 32 + lane] = xpose_reduce<true>(v, lane);
         }
@@ -538,7 +545,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
         uint32_t ph[16];
 #pragma unroll
         for (int jj = 0; jj < 32; jj += 2) {
-          const int c0 = half * 32 + jj;
+          const int c0 = col0 + jj;
           const float m0 = jj < ncols ? m_run[c0] : -INFINITY, m1 = jj < ncols ? m_run[c0 + 1] : -INFINITY;
           const float p0 = m0 == -INFINITY ? 0.0f : exp2f(s[jj] - m0);
           const float p1 = m1 == -INFINITY ? 0.0f : exp2f(s[jj + 1] - m1);
@@ -550,13 +557,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
         }
         // P^T rows of NQ heads (2 NQ bytes, the swizzle of that width)
         if (NQ == 16) {
-          *reinterpret_cast<uint4*>(Ps + tc::swz(key, 0, 32)) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
-          *reinterpret_cast<uint4*>(Ps + tc::swz(key, 16, 32)) = make_uint4(ph[4], ph[5], ph[6], ph[7]);
-          float v16[16];
+          *reinterpret_cast<uint4*>(Ps + tc::swz(key, half * 16, 32)) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+          float v8[8];
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) v16[jj] = v[jj];
-          const float s16 = xpose_reduce16<false>(v16, lane);
-          if (lane < 16) red_sum[q4 * 64 + lane] = s16;
+          for (int jj = 0; jj < 8; ++jj) v8[jj] = v[jj];
+          const float s8 = xpose_reduce8<false>(v8, lane);
+          if (lane < 8) red_sum[q4 * 64 + col0 + lane] = s8;
         } else {
           const uint32_t rbw = 2u * (uint32_t)NQ;
 #pragma unroll
