@@ -827,12 +827,11 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
   // chunk ch of the slice -> ks (item lo + ch*kSelChunk + kPer*t + e is key e of thread t; 0 past hi)
   const uint32_t* mk = ks + tid * kKeyRow;
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u, cnt = 0u;  // over the valid (non-zero) keys
-  auto load_chunk = [&](int ch, bool range) {
+  constexpr int kLoads = kSelChunk / 4 / kSelThreads;  // 16 B loads per thread, all in flight
+  // issue chunk ch's loads into registers (no wait)
+  auto fetch_chunk = [&](int ch, uint4 (&v)[kLoads]) {
     const int64_t c0 = lo + (int64_t)ch * kSelChunk;
     const int64_t cn = hi - c0 < kSelChunk ? hi - c0 : kSelChunk;
-    __syncthreads();  // earlier readers of ks are done
-    constexpr int kLoads = kSelChunk / 4 / kSelThreads;  // 16 B loads per thread, all in flight
-    uint4 v[kLoads];
 #pragma unroll
     for (int u = 0; u < kLoads; ++u) {
       const int i = 4 * (tid + u * kSelThreads);
@@ -845,6 +844,10 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
         v[u].z = i + 2 < cn ? keys[c0 + i + 2] : 0u;
       }
     }
+  };
+  // fetched keys -> ks, between barriers (earlier readers of ks are done; the rows are complete)
+  auto stash_chunk = [&](const uint4 (&v)[kLoads], bool range) {
+    __syncthreads();
 #pragma unroll
     for (int u = 0; u < kLoads; ++u) {
       const int i = 4 * (tid + u * kSelThreads);
@@ -867,7 +870,13 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
     }
     __syncthreads();
   };
+  auto load_chunk = [&](int ch, bool range) {
+    uint4 v[kLoads];
+    fetch_chunk(ch, v);
+    stash_chunk(v, range);
+  };
   // ---- one CTA walking several chunks: two passes over the keys ------------------------------
+  // Each pass fetches the next chunk into registers while the current one is processed.
   // Pass 1 counts the top 10 bits (sign, exponent, one mantissa bit) of every valid key; the
   // bin holding the K-th largest is the cut.  Pass 2 writes every key above that bin straight
   // to its slot (index order, per-chunk block prefixes) and copies the bin's keys, with their
@@ -880,8 +889,11 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
     uint32_t* candk = reinterpret_cast<uint32_t*>(blk + CSA2_MAX_K);  // [kCand] keys of the cut bin
     int32_t* candi = reinterpret_cast<int32_t*>(candk + kCand);        // [kCand] their item indices
     uint32_t cnt = 0u;
+    uint4 nxt[kLoads];  // the next chunk's keys, in flight while this one is counted
+    fetch_chunk(0, nxt);
     for (int ch = 0; ch < nchunks; ++ch) {
-      load_chunk(ch, false);
+      stash_chunk(nxt, false);
+      if (ch + 1 < nchunks) fetch_chunk(ch + 1, nxt);
 #pragma unroll 4
       for (int e = 0; e < kPer; ++e) {
         const uint32_t key = mk[e];
@@ -910,8 +922,10 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
       int32_t* out = a.out_idx + (int64_t)bq * K;
       float* out_s = a.out_score ? a.out_score + (int64_t)bq * K : nullptr;
       uint32_t base_g = 0u, base_c = 0u;
+      fetch_chunk(0, nxt);
       for (int ch = 0; ch < nchunks; ++ch) {
-        load_chunk(ch, false);
+        stash_chunk(nxt, false);
+        if (ch + 1 < nchunks) fetch_chunk(ch + 1, nxt);
         uint32_t cg = 0u, cc = 0u;
 #pragma unroll 4
         for (int e = 0; e < kPer; ++e) {
