@@ -898,7 +898,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
       for (int e = 0; e < kPer; ++e) {
         const uint32_t key = mk[e];
         if (key != 0u) {
-          atomicAdd(&sub[key >> 22], 1u);
+          atomicAdd(&sub[key >> 20], 1u);
           ++cnt;
         }
       }
@@ -907,16 +907,30 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
     block_excl_scan64((uint64_t)cnt, scan_ws, &tot);  // also orders the counts before the search
     const bool all_valid = tot <= (uint64_t)K;
     uint32_t T1 = 0u, above1 = 0u, inbin1 = 0u;
-    if (!all_valid) {
+    if (!all_valid) {  // the cut bin of 4096: its group of 4 among 1024 groups, then the bin
+      for (int g = tid; g < kBins; g += kSelThreads)
+        hist[g] = sub[4 * g] + sub[4 * g + 1] + sub[4 * g + 2] + sub[4 * g + 3];
+      __syncthreads();
       if (tid < 32) {
-        find_bin_warp(sub, kBins, (uint32_t)K, &misc[0], &misc[1]);
+        find_bin_warp(hist, kBins, (uint32_t)K, &misc[0], &misc[1]);
         __syncwarp();
-        if (tid == 0) misc[2] = sub[misc[0]];
+        if (tid == 0) {
+          uint32_t above = misc[1], need1 = (uint32_t)K - above, t = 4 * misc[0] + 3;
+          for (int jj = 3; jj > 0; --jj, --t) {  // bins of the group from the top
+            const uint32_t c = sub[t];
+            if (need1 <= c) break;
+            need1 -= c;
+            above += c;
+          }
+          misc[2] = t;
+          misc[3] = above;
+          misc[4] = sub[t];
+        }
       }
       __syncthreads();
-      T1 = misc[0];
-      above1 = misc[1];
-      inbin1 = misc[2];
+      T1 = misc[2];
+      above1 = misc[3];
+      inbin1 = misc[4];
     }
     if (all_valid || inbin1 <= (uint32_t)kCand) {
       int32_t* out = a.out_idx + (int64_t)bq * K;
@@ -931,7 +945,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
         for (int e = 0; e < kPer; ++e) {
           const uint32_t key = mk[e];
           if (key != 0u) {
-            const uint32_t d = key >> 22;
+            const uint32_t d = key >> 20;
             if (all_valid || d > T1) ++cg;
             else if (d == T1) ++cc;
           }
@@ -944,7 +958,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
         for (int e = 0; e < kPer; ++e) {
           const uint32_t key = mk[e];
           if (key == 0u) continue;
-          const uint32_t d = key >> 22;
+          const uint32_t d = key >> 20;
           if (all_valid || d > T1) {
             out[lg] = (int32_t)item_label(a, blk, i0 + e);
             if (out_s) out_s[lg] = key_score(key);
@@ -968,13 +982,13 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
       // the remaining levels on the cut bin's keys, in two alternating histograms
       const int nc = (int)base_c;
       uint32_t need = (uint32_t)K - above1;
-      uint32_t prefix = T1 << 22, mask = 0xFFC00000u;
+      uint32_t prefix = T1 << 20, mask = 0xFFF00000u;
       for (int i = tid; i < kBins; i += kSelThreads) {
         hist[i] = 0u;
         hsum[i] = 0u;
       }
       __syncthreads();  // the list and the cleared counters are visible
-      int p = 21, cur = 0;
+      int p = 19, cur = 0;
       for (;;) {
         const int sh = p >= kDigitBits - 1 ? p - (kDigitBits - 1) : 0;
         const uint32_t nb = 1u << (p - sh + 1);
