@@ -640,15 +640,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
     // CTA o receives recv[c][d][0..hpc) from every CTA c (its heads' partial O^T rows).
     const int hpc = (((NH + C - 1) / C) + 3) & ~3;
     const int h0 = rank * hpc, n_own = max(0, min(hpc, NH - h0));
-    float* recv = reinterpret_cast<float*>(sm + kOffRecv);  // [C][512][hpc] partial O of each CTA
     float* fac = reinterpret_cast<float*>(Ps);                // [C][64] merge factors
     float* linv = fac + kMaxCluster * kHeadsPad;              // [hpc]
+    // With 16 heads, a CTA's query tile uses 16 of the 64 rows of each 8 KB dim-block and its
+    // P tile 4 KB of 16: the received partials go to that spare space (rows 16-63 of the dim-
+    // blocks, then the P area past the tile, in 6 KB pieces), and the per-head max and sum to
+    // the tail of the misc area.  Nothing else reads or writes those bytes, so a CTA may push
+    // as soon as its own products are done: no cluster barrier first.  Otherwise the partials
+    // go over the key and query tiles, once every CTA of the cluster is done with them.
+    const bool spare = NQ == 16 && C * kD * hpc * 4 <= 10 * 6144;
+    auto recv_off = [&](uint32_t byte) -> uint32_t {  // shared-memory offset of a received byte
+      if (!spare) return kOffRecv + byte;
+      const uint32_t g = byte / 6144u, r = byte - g * 6144u;
+      return g < 8u ? kOffQ + g * 8192u + 2048u + r : kOffP + 4096u + (g - 8u) * 6144u + r;
+    };
+    float* rml = reinterpret_cast<float*>(sm + kOffMisc + 3584);  // spare: max [C][hpc], sum [C][hpc]
+    float* rmax = spare ? rml : red_max;
+    float* rsum = spare ? rml + C * hpc : red_sum;
     tc::fence_before_sync();
-    cluster_sync_all();  // every CTA has finished its products: key and query tiles are free
+    if (!spare) cluster_sync_all();  // every CTA has finished its products: key and query tiles are free
     {
       const int q4 = warp & 3, half = warp >> 2;
       const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
-      const uint32_t recv_a = tc::smem_u32(recv);
+      const uint32_t sm_a = tc::smem_u32(sm);
       tc::fence_after_sync();
       const int cw = NQ == 16 ? 16 : 32;
       const bool have = T > 0 && !timed_out;
@@ -667,7 +681,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
             const int h = c0 + 4 * j4;  // heads h..h+3 share an owner (hpc is a multiple of 4)
             if (4 * j4 < cw && h < NH) {
               const int o_rank = h / hpc, hl = h - o_rank * hpc;
-              const uint32_t dst = recv_a + (uint32_t)(((rank * kD + d) * hpc + hl) * 4);
+              const uint32_t dst = sm_a + recv_off((uint32_t)(((rank * kD + d) * hpc + hl) * 4));
               if (have)
                 st_cluster_v4(tc::mapa(dst, (uint32_t)o_rank), o[4 * j4], o[4 * j4 + 1], o[4 * j4 + 2], o[4 * j4 + 3]);
               else
@@ -679,9 +693,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
       if (tid < NH) {  // this CTA's max and sum of head tid, to its owner
         const int o_rank = tid / hpc, hl = tid - o_rank * hpc;
         const float l = l_run[tid];
-        st_cluster_f32(tc::mapa(tc::smem_u32(red_max + rank * hpc + hl), (uint32_t)o_rank),
+        st_cluster_f32(tc::mapa(tc::smem_u32(rmax + rank * hpc + hl), (uint32_t)o_rank),
                        l > 0.0f ? m_run[tid] : -INFINITY);
-        st_cluster_f32(tc::mapa(tc::smem_u32(red_sum + rank * hpc + hl), (uint32_t)o_rank), l);
+        st_cluster_f32(tc::mapa(tc::smem_u32(rsum + rank * hpc + hl), (uint32_t)o_rank), l);
       }
     }
     cluster_sync_all();  // every partial has arrived
@@ -689,11 +703,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
       if (tid < n_own) {
         float M = -INFINITY;
         for (int c = 0; c < C; ++c)
-          if (red_sum[c * hpc + tid] > 0.0f) M = fmaxf(M, red_max[c * hpc + tid]);
+          if (rsum[c * hpc + tid] > 0.0f) M = fmaxf(M, rmax[c * hpc + tid]);
         float L = 0.0f;
         for (int c = 0; c < C; ++c) {
-          const float lc = red_sum[c * hpc + tid];
-          const float f = lc > 0.0f ? exp2f(red_max[c * hpc + tid] - M) : 0.0f;
+          const float lc = rsum[c * hpc + tid];
+          const float f = lc > 0.0f ? exp2f(rmax[c * hpc + tid] - M) : 0.0f;
           fac[c * kHeadsPad + tid] = f;
           L = fmaf(lc, f, L);
         }
@@ -706,7 +720,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
         const int g4 = i / kD, d = i % kD;  // heads 4 g4 .. 4 g4 + 3 of this CTA
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int c = 0; c < C; ++c) {
-          const float4 x = *reinterpret_cast<const float4*>(recv + (c * kD + d) * hpc + 4 * g4);
+          const float4 x =
+              *reinterpret_cast<const float4*>(sm + recv_off((uint32_t)(((c * kD + d) * hpc + 4 * g4) * 4)));
           acc.x = fmaf(x.x, fac[c * kHeadsPad + 4 * g4 + 0], acc.x);
           acc.y = fmaf(x.y, fac[c * kHeadsPad + 4 * g4 + 1], acc.y);
           acc.z = fmaf(x.z, fac[c * kHeadsPad + 4 * g4 + 2], acc.z);
