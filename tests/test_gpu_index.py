@@ -404,3 +404,24 @@ def test_multichunk_select_ties(orc, neg):
     o_topk, _ = orc.index_full(q[:, :1].numpy(), w[:, :1].numpy(), o_ik, np.zeros(1, np.int64),
                                np.array([[T]], np.int32), 300)
     assert sorted(o_topk[0, 0].tolist()) == want
+
+
+@pytest.mark.parametrize("nv", [300, 512, 513, 16384])
+def test_cluster_select_few_valid_keys(orc, nv):
+    """A 16,384-key flat selection runs as a cluster of 4 register CTAs, which learns how many
+    keys are valid from its first level's summed histogram: at most K valid keys (300, 512)
+    are all taken, in index order, with -1 after them; one more (513) goes through the radix
+    levels.  Checked against the oracle at the tie band."""
+    T, K = 16384, 512
+    kv, ik = synth.kv_tokens(31, T, recipe="rmsnorm")
+    kvp, ikp, _, o_ik = pools_from_tokens(orc, kv.cuda(), ik.cuda())
+    q, w = synth.index_queries(32, 1, 1, 8)
+    n_vis = torch.tensor([[nv]], dtype=torch.int32, device="cuda")
+    topk, score, st = run_full(q.cuda(), w.cuda(), ikp, torch.zeros(1, dtype=torch.int64, device="cuda"), n_vis, K, T)
+    assert st == 0
+    o_topk, _ = orc.index_full(q.numpy(), w.numpy(), o_ik, np.zeros(1, np.int64), np.array([[nv]], np.int32), K)
+    s = orc.index_scores(q[0, 0].numpy(), w[0, 0].numpy(), o_ik[:nv])
+    assert_topk_set(topk[0, 0], o_topk[0, 0], s, K)
+    if nv <= K:
+        assert topk[0, 0, :nv].tolist() == list(range(nv))   # every key, in index order
+        assert (topk[0, 0, nv:] == -1).all()
