@@ -19,7 +19,8 @@ cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t
                          const int32_t* blocks, int B, int Q, int HI, int n_blocks, int block,
                          int K, int64_t max_n_vis, int32_t* out_idx, float* out_score,
                          uint32_t* keys, int64_t key_stride, uint32_t* status,
-                         cudaStream_t stream, int withheld_tile = -1);
+                         cudaStream_t stream, int withheld_tile = -1, uint32_t* gmax = nullptr,
+                         int64_t gstride = 0);
 size_t attn_workspace_bytes(int B, int Q, int H, int K, int window);
 cudaError_t launch_sparse_attn(const float* q, const uint8_t* kv_pool, int64_t pool_entries,
                                const int64_t* seq_base, const int32_t* topk, int K,
@@ -42,7 +43,7 @@ namespace {
 
 constexpr int64_t kMaxQueries = 65535;  // grid.y limit of the per-query kernels
 constexpr int64_t kMaxNVis = (int64_t)1 << 23;  // largest accepted visible count: a selection CTA then
-                                                // holds at most 2^20 keys (64 reloaded chunks)
+                                                // counts at most 2^23 keys in 32-bit counters
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -144,11 +145,19 @@ csa2_status csa2_pack_kv_normed(const void* kv, const void* ik, int64_t T, int r
                                               current_sm_count()));
 }
 
+// The flat index workspace: the keys [B*Q][key_row(max_n_vis)], then the largest key of every
+// 32 [B*Q][key_row(ceil(max_n_vis / 32))].
+size_t full_keys_bytes(int B, int Q, int64_t max_n_vis) {
+  return round256((size_t)B * Q * (size_t)key_row(max_n_vis) * sizeof(uint32_t));
+}
+int64_t full_gmax_row(int64_t max_n_vis) { return key_row((max_n_vis + 31) / 32); }
+
 size_t csa2_index_full_workspace_size(int B, int Q, int HI, int K, int64_t max_n_vis) {
   (void)HI;
   (void)K;
   if (B <= 0 || Q <= 0 || max_n_vis <= 0) return 0;
-  return round256((size_t)B * Q * (size_t)key_row(max_n_vis) * sizeof(uint32_t));
+  return full_keys_bytes(B, Q, max_n_vis) +
+         round256((size_t)B * Q * (size_t)full_gmax_row(max_n_vis) * sizeof(uint32_t));
 }
 
 csa2_status csa2_index_full(const float* q, const float* w, const uint8_t* ik_pool,
@@ -164,9 +173,11 @@ csa2_status csa2_index_full(const float* q, const float* w, const uint8_t* ik_po
   if (!topk || !aligned(topk, 4) || (topk_score && !aligned(topk_score, 4))) return CSA2_ERR_INVALID_ARG;
   const size_t need = csa2_index_full_workspace_size(B, Q, HI, K, max_n_vis);
   if ((st = check_ws(ws, ws_bytes, need)) != CSA2_OK) return st;
+  uint32_t* gmax = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + full_keys_bytes(B, Q, max_n_vis));
   return launched(csa2::launch_index(0, q, w, ik_pool, pool_entries, seq_base, n_vis, nullptr, B,
                                      Q, HI, 0, 1, K, max_n_vis, topk, topk_score,
-                                     static_cast<uint32_t*>(ws), key_row(max_n_vis), dev_status, stream));
+                                     static_cast<uint32_t*>(ws), key_row(max_n_vis), dev_status, stream, -1,
+                                     gmax, full_gmax_row(max_n_vis)));
 }
 
 csa2_status csa2_test_index_full_withheld_copy(const float* q, const float* w, const uint8_t* ik_pool,

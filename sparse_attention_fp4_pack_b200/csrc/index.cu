@@ -61,6 +61,8 @@ struct ScanArgs {
   int64_t max_n_vis;
   int64_t key_stride;
   uint32_t* keys;
+  uint32_t* gmax;         // flat, may be null: the largest key of every 32 keys, per query row
+  int64_t gstride;        // gmax words per query row
   uint32_t* status;
   int withheld_tile;      // test hook: the first CTA never copies this tile (-1: off)
 };
@@ -558,8 +560,12 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
         if (MODE == kHier) {
           for (int o = 1; o < a.block; o <<= 1) key = max(key, __shfl_xor_sync(0xffffffffu, key, o));
           if ((row & (a.block - 1)) == 0 && j < nqg) krow[j >> a.block_shift] = key;
-        } else if (j < limit) {
-          krow[j] = key;
+        } else {
+          if (j < limit) krow[j] = key;
+          if (a.gmax != nullptr) {  // the largest key of this warp's 32 rows
+            const uint32_t m = __reduce_max_sync(0xffffffffu, key);
+            if ((row & 31) == 0 && j < limit) a.gmax[((int64_t)b * a.Q + q0 + g) * a.gstride + (j >> 5)] = m;
+          }
         }
       }
       tc::fence_before_sync();
@@ -647,8 +653,8 @@ constexpr int kMaxCluster = 8;
 //   hist  [kBins] this CTA's histogram;  hsum [kBins] the cluster's
 //   scan scratch (32 x u64), cluster exchange words (16) and misc (8), padded to 64 words
 //   blk   [CSA2_MAX_K] the query's Reindex block ids
-// A CTA holds at most 2^20 keys (the host caps max_n_vis at 2^23, a query gets up to 8
-// CTAs), so no 32-bit counter can overflow.
+// A CTA counts at most 2^23 keys (the host caps max_n_vis at 2^23), so no 32-bit counter
+// can overflow.
 constexpr int kSubWords = kBins > 2 * CSA2_MAX_K ? kBins : 2 * CSA2_MAX_K;
 constexpr int kCand = 4096;  // keys of the cut bin a multi-chunk CTA keeps in shared memory
 template <int PS>
@@ -673,6 +679,8 @@ struct SelectArgs {
   int64_t max_n_vis, pool_entries;
   const int32_t* blocks;
   const int32_t* labels;     // kMerge: label of item i at labels[bq * key_stride + i]
+  const uint32_t* gmax;      // kFlat, may be null: the largest key of every 32, per query row
+  int64_t gstride;
   int64_t n_items;           // kMerge: items per query
   int32_t* out_idx;
   float* out_score;
@@ -885,9 +893,226 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
   // do not, the counters are cleared and the general path below runs instead.  Against the
   // general path (a range pass, one pass per level, a counting pass and an output pass, each
   // reloading every chunk) this reads the keys twice instead of about six times.
+  // Shared by the one-CTA paths below: the listed keys (candk/candi, nc of them, in index
+  // order; every one shares the bits of `mask` with `prefix`, the highest undecided bit being
+  // p) resolved into the slots from `base`: the remaining radix levels in two alternating
+  // histograms, then the taken keys in index order and the first `need` keys tied at the cut.
+  uint32_t* candk = reinterpret_cast<uint32_t*>(blk + CSA2_MAX_K);  // [kCand] listed keys
+  int32_t* candi = reinterpret_cast<int32_t*>(candk + kCand);        // [kCand] their item indices
+  auto finish_list = [&](int nc, uint32_t base, uint32_t need, uint32_t prefix, uint32_t mask, int p,
+                         int32_t* out, float* out_s) {
+
+    for (int i = tid; i < kBins; i += kSelThreads) {
+      hist[i] = 0u;
+      hsum[i] = 0u;
+    }
+    __syncthreads();  // the list and the cleared counters are visible
+    int cur = 0;
+    while (p >= 0) {
+      const int sh = p >= kDigitBits - 1 ? p - (kDigitBits - 1) : 0;
+      const uint32_t nb = 1u << (p - sh + 1);
+      uint32_t* h = cur ? hsum : hist;
+      uint32_t* hn = cur ? hist : hsum;
+      for (int i = tid; i < nc; i += kSelThreads) {
+        const uint32_t key = candk[i];
+        if ((key & mask) == prefix) atomicAdd(&h[(key >> sh) & (nb - 1u)], 1u);
+      }
+      for (int i = tid; i < kBins; i += kSelThreads) hn[i] = 0u;  // last read on the level before
+      __syncthreads();
+      if (tid < 32) {
+        find_bin_warp(h, (int)nb, need, &misc[0], &misc[1]);
+        __syncwarp();
+        if (tid == 0) misc[2] = h[misc[0]];
+      }
+      __syncthreads();
+      const uint32_t T = misc[0], inbin = misc[2];
+      need -= misc[1];
+      prefix |= T << sh;
+      mask |= (nb - 1u) << sh;
+      if (inbin == need || sh == 0) break;
+      p = sh - 1;
+      cur ^= 1;
+    }
+    // the list's taken keys after the first pass's, then its first `need` tied keys; a
+    // thread takes a contiguous run of the list, so both stay in index order
+    const int per = (nc + kSelThreads - 1) / kSelThreads;
+    const int c0 = tid * per, c1 = min(nc, c0 + per);
+    uint32_t g2 = 0u, e2 = 0u;
+    for (int i = c0; i < c1; ++i) {
+      const uint32_t kp = candk[i] & mask;
+      if (kp > prefix) ++g2;
+      else if (kp == prefix) ++e2;
+    }
+    uint64_t t2;
+    const uint64_t m2 = block_excl_scan64((uint64_t)g2 | ((uint64_t)e2 << 32), scan_ws, &t2);
+    uint32_t lg = base + (uint32_t)m2, le = (uint32_t)(m2 >> 32);
+    const uint32_t tie0 = (uint32_t)K - need;
+    for (int i = c0; i < c1; ++i) {
+      const uint32_t key = candk[i], kp = key & mask;
+      if (kp > prefix) {
+        out[lg] = (int32_t)item_label(a, blk, candi[i]);
+        if (out_s) out_s[lg] = key_score(key);
+        ++lg;
+      } else if (kp == prefix) {
+        if (le < need) {
+          out[tie0 + le] = (int32_t)item_label(a, blk, candi[i]);
+          if (out_s) out_s[tie0 + le] = key_score(key);
+        }
+        ++le;
+      }
+    }
+  };
+
+  // ---- one CTA, with the scan's group maxima: a threshold, then only the groups above it ----
+  // The flat scan also leaves the largest key of every 32 (gm).  At least K groups have a
+  // maximum at or above x, the K-th largest maximum cut to its top 22 bits, so at least K keys
+  // are >= x and the K best are among them.  Only the groups whose maximum reaches x are read
+  // (a warp per group): their keys >= x go, with their item indices and in index order, to the
+  // shared-memory list that the remaining radix levels resolve.  With fewer than K valid
+  // groups x = 1, every valid key.  When the groups above x (kGroupList) or their keys
+  // (kCand) do not fit, the counters are cleared and the two-pass path below runs instead.
+  if constexpr (PS >= 4) {
+    if (C == 1 && nchunks > 1 && a.gmax != nullptr) {
+      constexpr int kGroupList = 8192;
+      static_assert(2 * kGroupList <= kKeyWords, "the group list is kept where the chunks would be");
+      constexpr int kWarps = kSelThreads / 32, kU = 8;  // a warp reads kU groups at a time
+      const uint32_t* gm = a.gmax + (int64_t)bq * a.gstride;
+      const int ng = (int)((n + 31) >> 5);
+      uint32_t gc = 0u;
+      for (int g = tid; g < ng; g += kSelThreads) {
+        const uint32_t m = gm[g];
+        if (m != 0u) {
+          atomicAdd(&sub[m >> 20], 1u);
+          ++gc;
+        }
+      }
+      uint64_t gtot;
+      block_excl_scan64((uint64_t)gc, scan_ws, &gtot);  // also orders the counts before the search
+      uint32_t x = 1u;
+      if (gtot >= (uint64_t)K) {
+        // the 12-bit bin of the K-th largest maximum: its group of 4 among 1024, then the bin
+        for (int g = tid; g < kBins; g += kSelThreads) {
+          hist[g] = sub[4 * g] + sub[4 * g + 1] + sub[4 * g + 2] + sub[4 * g + 3];
+          hsum[g] = 0u;
+        }
+        __syncthreads();
+        if (tid < 32) {
+          find_bin_warp(hist, kBins, (uint32_t)K, &misc[0], &misc[1]);
+          __syncwarp();
+          if (tid == 0) {
+            uint32_t above = misc[1], need1 = (uint32_t)K - above, t = 4 * misc[0] + 3;
+            for (int jj = 3; jj > 0; --jj, --t) {  // bins of the group from the top
+              const uint32_t c = sub[t];
+              if (need1 <= c) break;
+              need1 -= c;
+              above += c;
+            }
+            misc[2] = t;
+            misc[3] = above;
+          }
+        }
+        __syncthreads();
+        const uint32_t T1 = misc[2], above1 = misc[3];
+        // the next 10 bits, among the maxima in that bin
+        for (int g = tid; g < ng; g += kSelThreads) {
+          const uint32_t m = gm[g];
+          if ((m >> 20) == T1) atomicAdd(&hsum[(m >> 10) & (kBins - 1)], 1u);
+        }
+        __syncthreads();
+        if (tid < 32) find_bin_warp(hsum, kBins, (uint32_t)K - above1, &misc[4], &misc[5]);
+        __syncthreads();
+        x = max((T1 << 20) | (misc[4] << 10), 1u);
+      }
+      // the groups whose maximum reaches x, in index order (a thread takes a contiguous run)
+      uint32_t* gl = ks;                // [kGroupList] their group numbers
+      uint32_t* goff = ks + kGroupList;  // [kGroupList] their keys >= x, then their first list slots
+      const int per = (ng + kSelThreads - 1) / kSelThreads;
+      const int g0 = tid * per, g1 = min(ng, g0 + per);
+      uint32_t sc = 0u;
+      for (int g = g0; g < g1; ++g) sc += gm[g] >= x ? 1u : 0u;
+      uint64_t stot;
+      uint32_t so = (uint32_t)block_excl_scan64((uint64_t)sc, scan_ws, &stot);
+      const int S = (int)stot;
+      if (S <= kGroupList) {
+        for (int g = g0; g < g1; ++g)
+          if (gm[g] >= x) gl[so++] = (uint32_t)g;
+        __syncthreads();
+        const int warp = tid >> 5;
+        // the keys of kU listed groups of this warp (0 past the list and past n)
+        auto group_keys = [&](int s0, uint32_t (&kk)[kU]) {
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const int sidx = s0 + u * kWarps;
+            kk[u] = 0u;
+            if (sidx < S) {
+              const int64_t i = (int64_t)gl[sidx] * 32 + lane;
+              if (i < n) kk[u] = keys[i];
+            }
+          }
+        };
+        for (int s0 = warp; s0 < S; s0 += kWarps * kU) {
+          uint32_t kk[kU];
+          group_keys(s0, kk);
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const uint32_t m = __ballot_sync(0xffffffffu, kk[u] >= x);
+            if (lane == 0 && s0 + u * kWarps < S) goff[s0 + u * kWarps] = (uint32_t)__popc(m);
+          }
+        }
+        __syncthreads();
+        const int per2 = (S + kSelThreads - 1) / kSelThreads;
+        const int s0 = tid * per2, s1 = min(S, s0 + per2);
+        uint32_t cc = 0u;
+        for (int si = s0; si < s1; ++si) cc += goff[si];
+        uint64_t ctot;
+        uint32_t co = (uint32_t)block_excl_scan64((uint64_t)cc, scan_ws, &ctot);
+        const int nc = (int)ctot;
+        if (nc <= kCand) {
+          for (int si = s0; si < s1; ++si) {
+            const uint32_t c = goff[si];
+            goff[si] = co;
+            co += c;
+          }
+          __syncthreads();
+          for (int sw = warp; sw < S; sw += kWarps * kU) {
+            uint32_t kk[kU];
+            group_keys(sw, kk);
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+              const uint32_t m = __ballot_sync(0xffffffffu, kk[u] >= x);
+              if (kk[u] >= x) {
+                const int sidx = sw + u * kWarps;
+                const uint32_t pos = goff[sidx] + (uint32_t)__popc(m & ((1u << lane) - 1u));
+                candk[pos] = kk[u];
+                candi[pos] = (int32_t)(gl[sidx] * 32u + (uint32_t)lane);
+              }
+            }
+          }
+          if (nc <= K) {  // every valid key (fewer than K groups), in index order, then -1
+            __syncthreads();
+            for (int i = tid; i < K; i += kSelThreads) {
+              if (i < nc) {
+                out[i] = (int32_t)item_label(a, blk, candi[i]);
+                if (out_s) out_s[i] = key_score(candk[i]);
+              } else {
+                out[i] = -1;
+                if (out_s) out_s[i] = -INFINITY;
+              }
+            }
+            return;
+          }
+          finish_list(nc, 0u, (uint32_t)K, 0u, 0u, 31, out, out_s);
+          return;
+        }
+      }
+      __syncthreads();  // every thread has left the counters and the list
+      for (int i = tid; i < kSubWords / 4; i += kSelThreads)
+        reinterpret_cast<uint4*>(sub)[i] = make_uint4(0u, 0u, 0u, 0u);
+      __syncthreads();
+    }
+  }
+
   if (C == 1 && nchunks > 1) {
-    uint32_t* candk = reinterpret_cast<uint32_t*>(blk + CSA2_MAX_K);  // [kCand] keys of the cut bin
-    int32_t* candi = reinterpret_cast<int32_t*>(candk + kCand);        // [kCand] their item indices
     uint32_t cnt = 0u;
     uint4 nxt[kLoads];  // the next chunk's keys, in flight while this one is counted
     fetch_chunk(0, nxt);
@@ -979,69 +1204,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
         }
         return;
       }
-      // the remaining levels on the cut bin's keys, in two alternating histograms
-      const int nc = (int)base_c;
-      uint32_t need = (uint32_t)K - above1;
-      uint32_t prefix = T1 << 20, mask = 0xFFF00000u;
-      for (int i = tid; i < kBins; i += kSelThreads) {
-        hist[i] = 0u;
-        hsum[i] = 0u;
-      }
-      __syncthreads();  // the list and the cleared counters are visible
-      int p = 19, cur = 0;
-      for (;;) {
-        const int sh = p >= kDigitBits - 1 ? p - (kDigitBits - 1) : 0;
-        const uint32_t nb = 1u << (p - sh + 1);
-        uint32_t* h = cur ? hsum : hist;
-        uint32_t* hn = cur ? hist : hsum;
-        for (int i = tid; i < nc; i += kSelThreads) {
-          const uint32_t key = candk[i];
-          if ((key & mask) == prefix) atomicAdd(&h[(key >> sh) & (nb - 1u)], 1u);
-        }
-        for (int i = tid; i < kBins; i += kSelThreads) hn[i] = 0u;  // last read on the level before
-        __syncthreads();
-        if (tid < 32) {
-          find_bin_warp(h, (int)nb, need, &misc[0], &misc[1]);
-          __syncwarp();
-          if (tid == 0) misc[2] = h[misc[0]];
-        }
-        __syncthreads();
-        const uint32_t T = misc[0], inbin = misc[2];
-        need -= misc[1];
-        prefix |= T << sh;
-        mask |= (nb - 1u) << sh;
-        if (inbin == need || sh == 0) break;
-        p = sh - 1;
-        cur ^= 1;
-      }
-      // the list's taken keys after the first pass's, then its first `need` tied keys; a
-      // thread takes a contiguous run of the list, so both stay in index order
-      const int per = (nc + kSelThreads - 1) / kSelThreads;
-      const int c0 = tid * per, c1 = min(nc, c0 + per);
-      uint32_t g2 = 0u, e2 = 0u;
-      for (int i = c0; i < c1; ++i) {
-        const uint32_t kp = candk[i] & mask;
-        if (kp > prefix) ++g2;
-        else if (kp == prefix) ++e2;
-      }
-      uint64_t t2;
-      const uint64_t m2 = block_excl_scan64((uint64_t)g2 | ((uint64_t)e2 << 32), scan_ws, &t2);
-      uint32_t lg = above1 + (uint32_t)m2, le = (uint32_t)(m2 >> 32);
-      const uint32_t tie0 = (uint32_t)K - need;
-      for (int i = c0; i < c1; ++i) {
-        const uint32_t key = candk[i], kp = key & mask;
-        if (kp > prefix) {
-          out[lg] = (int32_t)item_label(a, blk, candi[i]);
-          if (out_s) out_s[lg] = key_score(key);
-          ++lg;
-        } else if (kp == prefix) {
-          if (le < need) {
-            out[tie0 + le] = (int32_t)item_label(a, blk, candi[i]);
-            if (out_s) out_s[tie0 + le] = key_score(key);
-          }
-          ++le;
-        }
-      }
+      finish_list((int)base_c, above1, (uint32_t)K - above1, T1 << 20, 0xFFF00000u, 19, out, out_s);
       return;
     }
     __syncthreads();  // every thread has read the search's result before the counters clear
@@ -1715,6 +1878,10 @@ static cudaError_t launch_select(SelectArgs s, int64_t items, int BQ, cudaStream
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int64_t c = (items + SelShape<4>::kChunk - 1) / SelShape<4>::kChunk;
     c = c < 1 ? 1 : (c > kMaxCluster ? kMaxCluster : c);
+    // with the scan's group maxima one CTA reads little more than the groups above the
+    // threshold (full128k, 32 queries of up to 131,072 keys: 10% faster on the whole step than
+    // 4 CTAs walking the keys)
+    if (s.gmax != nullptr) c = 1;
     const int64_t fit = (int64_t)sms / (BQ > 0 ? BQ : 1);  // CTAs per query in one wave
     if (c > fit) c = fit < 1 ? 1 : (fit >= 8 ? 8 : (fit >= 4 ? 4 : (fit >= 2 ? 2 : 1)));
     s.csize = (int)c;
@@ -1753,9 +1920,11 @@ cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t
                          const int32_t* blocks, int B, int Q, int HI, int n_blocks, int block,
                          int K, int64_t max_n_vis, int32_t* out_idx, float* out_score,
                          uint32_t* keys, int64_t key_stride, uint32_t* status,
-                         cudaStream_t stream, int withheld_tile) {
+                         cudaStream_t stream, int withheld_tile, uint32_t* gmax, int64_t gstride) {
   ScanArgs a;
   a.withheld_tile = withheld_tile;
+  a.gmax = mode == kFlat ? gmax : nullptr;
+  a.gstride = gstride;
   a.q = q;
   a.w = w;
   a.ik_pool = ik_pool;
@@ -1799,6 +1968,8 @@ cudaError_t launch_index(int mode, const float* q, const float* w, const uint8_t
   s.blocks = blocks;
   s.labels = nullptr;
   s.n_items = 0;
+  s.gmax = mode == kFlat ? gmax : nullptr;
+  s.gstride = gstride;
   s.out_idx = out_idx;
   s.out_score = out_score;
   const int64_t items = mode == kFlat ? max_n_vis

@@ -375,13 +375,15 @@ def test_cluster_select_ties_across_ctas(orc, T):
     assert sorted(o_topk[0, 0].tolist()) == want
 
 
-@pytest.mark.parametrize("neg", [36000, 20000])
-def test_multichunk_select_ties(orc, neg):
-    """80 queries of 40,000 keys each: the selection runs one CTA per query walking three
-    16,384-key chunks.  Entries [0, neg) score -128, the last 100 score 128 and the rest 0,
-    so the Top-300 is the 100 positive keys and the 200 lowest-index zero keys.  With 3,900
-    zero keys the cut bin fits the two-pass path's shared-memory list; with 19,900 it does not
-    and the general path runs."""
+@pytest.mark.parametrize("neg,K", [(36000, 120), (36000, 300), (20000, 300)])
+def test_multichunk_select_ties(orc, neg, K):
+    """80 queries of 40,000 keys each: the selection runs one CTA per query.  Entries [0, neg)
+    score -128, the last 100 score 128 and the rest 0, so the Top-K is the 100 positive keys
+    and the K - 100 lowest-index zero keys.  With 3,900 zero keys and K = 120 the 121 groups of
+    32 zero keys and the 4 positive groups hold the K-th largest group maximum, and their 4,000
+    keys fit the list of the group-maxima path; with K = 300 the threshold falls to the
+    negative groups and the two-pass path takes over, its cut bin (3,900 zero keys) fitting its
+    list; with 19,900 zero keys neither list fits and the general path runs."""
     T, Q = 40000, 80
     kv = torch.zeros(T, 512, dtype=torch.bfloat16, device="cuda")
     ik = torch.zeros(T, 128, dtype=torch.bfloat16, device="cuda")
@@ -394,16 +396,38 @@ def test_multichunk_select_ties(orc, neg):
     w = torch.tensor([1.0, -1.0]).reshape(1, 1, 2).repeat(1, Q, 1)
     n_vis = torch.full((1, Q), T, dtype=torch.int32, device="cuda")
     topk, score, st = run_full(q.cuda(), w.cuda(), ikp, torch.zeros(1, dtype=torch.int64, device="cuda"), n_vis,
-                               300, T)
+                               K, T)
     assert st == 0
-    want = list(range(neg, neg + 200)) + list(range(T - 100, T))
+    want = list(range(neg, neg + K - 100)) + list(range(T - 100, T))
     for i in range(Q):
         assert sorted(topk[0, i].tolist()) == want, f"query {i}"
     assert set(np.unique(score[0, 0]).tolist()) == {0.0, 128.0}
     _, o_ik = orc.pack_kv(np.zeros((T, 512), np.uint16), bf16_bits(ik), 1)
     o_topk, _ = orc.index_full(q[:, :1].numpy(), w[:, :1].numpy(), o_ik, np.zeros(1, np.int64),
-                               np.array([[T]], np.int32), 300)
+                               np.array([[T]], np.int32), K)
     assert sorted(o_topk[0, 0].tolist()) == want
+
+
+@pytest.mark.parametrize("K", [512, 2048])
+def test_group_select_ragged(orc, K):
+    """96 queries of one sequence, each with its own visible count between 16,385 and 40,000
+    (most not a multiple of 32): one CTA per query takes its threshold from the scan's maxima of
+    32 keys and reads only the groups that reach it.  Every query is checked against the
+    oracle."""
+    T, Q = 40000, 96
+    kv, ik = synth.kv_tokens(41, T, recipe="rmsnorm")
+    kvp, ikp, _, o_ik = pools_from_tokens(orc, kv.cuda(), ik.cuda())
+    q, w = synth.index_queries(42, 1, Q, 8)
+    g = torch.Generator().manual_seed(43)
+    n_vis = torch.randint(16385, T + 1, (1, Q), generator=g).to(torch.int32)
+    n_vis[0, :3] = torch.tensor([T, 16385, 32 * 700], dtype=torch.int32)
+    topk, _, st = run_full(q.cuda(), w.cuda(), ikp, torch.zeros(1, dtype=torch.int64, device="cuda"),
+                           n_vis.cuda(), K, T)
+    assert st == 0
+    for i in range(Q):
+        s = orc.index_scores(q[0, i].numpy(), w[0, i].numpy(), o_ik)[: int(n_vis[0, i])]
+        o_topk, _ = orc.topk(s, K)
+        assert_topk_set(topk[0, i], o_topk, s, K, what=f"query {i}")
 
 
 @pytest.mark.parametrize("nv", [300, 512, 513, 16384])
