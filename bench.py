@@ -349,8 +349,9 @@ def dominant_roofline(wl, calls, peaks):
     return roof
 
 
-# arithmetic of the path: int8 x int8 -> int32 indexer dots (tcgen05 kind::i8) and
-# f16 x f16 -> fp32 attention (tcgen05 kind::f16), fp32 epilogues; FP4/FP8 storage
+# arithmetic of the path: f16 x f16 -> fp32 Full / hierarchical indexer dots and attention
+# (tcgen05 kind::f16), int8 x int8 -> int32 Reindex dots (kind::i8), fp32 epilogues; FP4/FP8
+# storage
 DTYPE = "f16+i8"
 
 

@@ -152,10 +152,10 @@ csa2_status csa2_pack_kv_normed(const void* kv, const void* ik, int64_t T, int r
  *        seq_base), -1 in unused slots; topk_score fp32 [B][Q][K] (may be NULL)
  *
  * score_j = sum_h w_h * max(0, q_h . k_j) over dequantised keys k_j.  Arithmetic: each
- * query head is scaled by a power of two and split into four int8 limbs (representing
- * it to 2^-21 of its largest element); the dot products of the limbs with the key's E2M1
- * codes are exact int32 sums on the tensor cores; fp32 is used only to combine the four
- * limbs, apply the ReLU, the head weights and the key's scale.  The result is a SET
+ * query head is scaled by a power of two and split into two f16 parts, hi + lo, which
+ * represent it to 2^-22 of each element; the key's E2M1 values are exact in f16; the
+ * tensor cores form every product exactly and sum both parts' products in fp32; fp32 then
+ * applies the ReLU, the head weights and the key's scale.  The result is a SET
  * (slot order unspecified); equal scores at the cut prefer lower indices.
  * 1 <= K <= 2048, 1 <= HI <= 16.
  * --------------------------------------------------------------------------------- */
@@ -192,8 +192,11 @@ csa2_status csa2_index_hier(const float* q, const float* w, const uint8_t* ik_po
  *
  * blocks int32 [B][Q][n_blocks] (from csa2_index_hier; ids distinct, -1 = empty).  The
  * candidates are the visible entries of those blocks; the result is the Top-K of them
- * by the layer's own q/w, exactly as csa2_index_full would rank them.  Block ids past
- * the pool are skipped and flag CSA2_DEV_BAD_INDEX.
+ * by the layer's own q/w, under csa2_index_full's score and tie rule.  Arithmetic: each
+ * query head is split into four int8 limbs (to 2^-22 of its largest element), the dot
+ * products with the codes are exact int32 sums on the tensor cores and fp32 combines the
+ * limbs (a K = 32 MMA step keeps this one-tile-per-CTA kernel's chain short).  Block ids
+ * past the pool are skipped and flag CSA2_DEV_BAD_INDEX.
  * --------------------------------------------------------------------------------- */
 size_t csa2_reindex_workspace_size(int B, int Q, int HI, int n_blocks, int block, int K);
 csa2_status csa2_reindex(const float* q, const float* w, const uint8_t* ik_pool,

@@ -93,20 +93,12 @@ __device__ __forceinline__ uint32_t half2_bits(float lo, float hi) {
 
 // 8 E2M1 codes (one 32-bit word, code i in bits 4i..4i+3) times an f16x2 scale -> 8 f16.
 __device__ __forceinline__ uint4 e2m1x8_to_f16(uint32_t w, uint32_t scale2) {
-  uint32_t h0, h1, h2, h3;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-      : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
-      : "r"(w));
+  const uint4 h = e2m1x8_f16(w);
   uint4 o;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o.x) : "r"(h0), "r"(scale2));
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o.y) : "r"(h1), "r"(scale2));
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o.z) : "r"(h2), "r"(scale2));
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o.w) : "r"(h3), "r"(scale2));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o.x) : "r"(h.x), "r"(scale2));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o.y) : "r"(h.y), "r"(scale2));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o.z) : "r"(h.z), "r"(scale2));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o.w) : "r"(h.w), "r"(scale2));
   return o;
 }
 

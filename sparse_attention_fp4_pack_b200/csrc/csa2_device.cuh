@@ -85,6 +85,21 @@ __device__ __forceinline__ uint32_t e2m1x2_rn_sat(float lo, float hi) {
   return r & 0xFFu;
 }
 
+// 8 E2M1 codes (one 32-bit word, code i in bits 4i..4i+3) -> 8 f16, exact (E2M1 values are
+// f16 values); code i lands in half i of the result, so the words keep the codes' order.
+__device__ __forceinline__ uint4 e2m1x8_f16(uint32_t w) {
+  uint4 o;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(o.x), "=r"(o.y), "=r"(o.z), "=r"(o.w)
+      : "r"(w));
+  return o;
+}
+
 // Non-negative fp32 -> E4M3 byte, round to nearest even, saturating at 448.
 __device__ __forceinline__ uint32_t e4m3_rn_sat(float x) {
   uint16_t r;

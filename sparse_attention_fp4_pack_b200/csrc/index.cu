@@ -12,12 +12,23 @@
 // Score of entry j for one query:  score_j = s_j * sum_h w_h * max(0, q_h . c_j)
 // (c_j the key's E2M1 values, s_j >= 0 its fp32 scale, so the ReLU commutes with s_j).
 //
-// Both scan kernels (stream_scan_kernel for the flat and hierarchical scans,
-// reindex_scan_kernel for Reindex) compute the dot products exactly on the tensor cores
-// (tcgen05.mma kind::i8, int32 accumulation):
-//   * A (128 entries x 128 dims, u8): u = 2c + 12 in [0, 24] — the E2M1 value doubled and
-//     offset to be non-negative; two byte-permutes per 4 codes build it (sign-replicate
-//     selects the positive or negative table).
+// The streaming scan (stream_scan_kernel: flat and hierarchical) computes the dot products
+// on the tensor cores as tcgen05.mma kind::f16 (f16 operands, fp32 accumulation):
+//   * A (128 entries x 128 dims, f16, in tensor memory): the key's E2M1 values themselves,
+//     which f16 holds exactly (the hardware's e2m1x2 -> f16x2 conversion, 8 codes per four
+//     instructions); each thread stores its entry's row into its own lane.
+//   * B (N rows x 128 dims, f16, twice): each query head h is scaled by the power of two
+//     S_h = 2^(14 - exponent(max|q_h|)), so x = q*S_h is exact with |x| < 2^15, and split
+//     into hi = f16(x) and lo = f16(x - hi), which represent x to 2^-22 of each element.
+//   * D (128 x N, fp32): the MMAs of hi and lo accumulate into the same columns, so D holds
+//     sum_d c_d (hi_d + lo_d) = S_h (q_h . c_j) with every product exact (2 x 11 significant
+//     bits) and fp32 sums; the epilogue applies the ReLU, the weights w_h / S_h and the key's
+//     scale.
+// The Reindex scan (reindex_scan_kernel: one tile per CTA, so its MMA chain is on the
+// critical path) uses tcgen05.mma kind::i8, whose K = 32 per instruction halves that chain:
+//   * A (128 entries x 128 dims, u8, shared memory): u = 2c + 12 in [0, 24] — the E2M1 value
+//     doubled and offset to be non-negative; two byte-permutes per 4 codes build it
+//     (sign-replicate selects the positive or negative table).
 //   * B (N rows x 128 dims, s8): each query head h is scaled by the power of two
 //     S_h = 2^(5 - exponent(max|q_h|)), so x = q*S_h is exact with |x| < 64, and split into
 //     four int8 limbs x = L0 + L1/128 + L2/128^2 + L3/128^3 (error below 2^-22).
@@ -27,10 +38,11 @@
 // One thread owns one tile row (entry) end to end: it builds the row's A operand, and
 // after the MMA reads the same TMEM lane and writes the entry's order-preserving uint32
 // key (hierarchical mode: the max over `block` neighbouring lanes).  The streaming scan
-// takes a group of up to 8 queries of one sequence per CTA (multi-query verify), so the A
-// operand is built once for the group.
+// takes a group of queries of one sequence per CTA (multi-query verify and prefill: 4 of
+// 8 heads), so the A operand is built once for the group.
 #include <algorithm>
 #include <cooperative_groups.h>
+#include <cuda_fp16.h>
 
 #include "csa2_device.cuh"
 #include "tc.cuh"
@@ -55,7 +67,7 @@ struct ScanArgs {
   const int32_t* blocks;  // reindex only
   int Q, HI, hipad, G, n_groups, n_blocks, block;
   int block_shift;        // log2(block)
-  int N;                  // MMA N = G * hipad * 4
+  int N;                  // MMA N = G * hipad rounded up to 16
   int tmem_cols;
   int tiles_per_cta;
   int64_t max_n_vis;
@@ -91,6 +103,86 @@ __device__ __forceinline__ void stage_async(uint32_t dst, const uint8_t* src, in
     tc::cp_async4(dst + head + body + 4 * i, src + head + body + 4 * i);
 }
 
+constexpr int kATmemCols = 64;       // an A tile in tensor memory: 128 f16 per lane, two per column
+
+// Row n of the B operands for one query head, from the head's 128 fp32 elements (lane l holds
+// elements 4l..4l+3; zeros for a padding row).  x = q*S with S = 2^(14 - exponent(max|q|)),
+// so |x| < 2^15 and the scaling is exact; hi = f16(x) and lo = f16(x - hi) (x - hi is exact in
+// fp32) represent x to 2^-22 of each element.  The hi operand sits at Bs and the lo operand at
+// Bs + 2*npad*128, each as two 128-byte-swizzled K-halves of npad rows (elements 0..63 and
+// 64..127).  Returns 1/S (0 for a head whose largest element is below 1e-30).
+__device__ __forceinline__ float build_b_head(uint8_t* Bs, int npad, int n, float4 v) {
+  const int lane = threadIdx.x & 31;
+  float m = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float S = 0.f, inv = 0.f;
+  if (m > 1e-30f) {
+    const int E = (int)((__float_as_uint(m) >> 23) & 0xFFu) - 127;
+    S = __uint_as_float((uint32_t)(127 + 14 - E) << 23);
+    inv = __uint_as_float((uint32_t)(127 - 14 + E) << 23);
+  }
+  const float x[4] = {v.x * S, v.y * S, v.z * S, v.w * S};
+  uint32_t hw[2], lw[2];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const __half2 h = __floats2half2_rn(x[2 * e], x[2 * e + 1]);
+    const float2 hf = __half22float2(h);
+    const __half2 l = __floats2half2_rn(x[2 * e] - hf.x, x[2 * e + 1] - hf.y);
+    hw[e] = *reinterpret_cast<const uint32_t*>(&h);
+    lw[e] = *reinterpret_cast<const uint32_t*>(&l);
+  }
+  const uint32_t off = (uint32_t)(lane >> 4) * (uint32_t)npad * 128u + tc::sw128((uint32_t)n, (uint32_t)(lane & 15) * 8u);
+  *reinterpret_cast<uint2*>(Bs + off) = make_uint2(hw[0], hw[1]);
+  *reinterpret_cast<uint2*>(Bs + 2u * (uint32_t)npad * 128u + off) = make_uint2(lw[0], lw[1]);
+  return inv;
+}
+
+// The 16 MMAs of one tile: A (its 128 x 128 f16 in tensor memory, 64 columns from a_tmem)
+// times the hi and then the lo B operand (each two swizzled K-halves of npad rows at b_addr),
+// all accumulating into the npad columns at d.
+__device__ __forceinline__ void issue_tile_mma(uint32_t d, uint32_t a_tmem, uint32_t b_addr, int npad,
+                                               uint32_t idesc) {
+  const uint32_t bh = (uint32_t)npad * 128u;  // one K-half of one B operand
+#pragma unroll
+  for (int p = 0; p < 2; ++p)
+#pragma unroll
+    for (int kh = 0; kh < 2; ++kh)
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)  // 16 elements per MMA: 8 columns of A, 32 B of a B row
+        tc::mma_f16_ts(d, a_tmem + (uint32_t)(kh * 32 + ks * 8),
+                       tc::smem_desc_sw128(b_addr + (uint32_t)(2 * p + kh) * bh + (uint32_t)ks * 32u, 16, 1024), idesc,
+                       (p | kh | ks) ? 1u : 0u);
+}
+
+// One entry's A row: its 128 E2M1 codes (16 words at ea in shared memory; zeros when !valid)
+// as f16 pairs into 64 columns of this thread's tensor-memory lane from taddr, then the wait
+// for the stores.  Warp-wide: every lane of the warp calls it.
+__device__ __forceinline__ void build_a_row(uint32_t taddr, uint32_t ea, bool valid) {
+  uint32_t cw[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) cw[i] = valid ? tc::ld_shared_u32(ea + 4u * (uint32_t)i) : 0u;
+  uint32_t o0[32], o1[32];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint4 h0 = e2m1x8_f16(cw[i]), h1 = e2m1x8_f16(cw[8 + i]);
+    o0[4 * i] = h0.x;
+    o0[4 * i + 1] = h0.y;
+    o0[4 * i + 2] = h0.z;
+    o0[4 * i + 3] = h0.w;
+    o1[4 * i] = h1.x;
+    o1[4 * i + 1] = h1.y;
+    o1[4 * i + 2] = h1.z;
+    o1[4 * i + 3] = h1.w;
+  }
+  tc::tmem_st32_nowait(taddr, o0);
+  tc::tmem_st32_nowait(taddr + 32u, o1);
+  tc::tmem_wait_st();
+}
+
+// Reindex scan: one CTA row per (sequence, query), each CTA scoring kRows-candidate tiles
+// gathered from the query's block list (128 / block blocks of `block` consecutive keys per
+// tile, staged by cp.async one tile ahead).
 // 8 E2M1 codes (one word) -> 8 bytes u = 2c + 12.
 __device__ __forceinline__ uint2 codes_to_u8(uint32_t w) {
   // tables indexed by the 3-bit magnitude m: 12 + 2|c| and 12 - 2|c|
@@ -105,9 +197,6 @@ __device__ __forceinline__ uint2 codes_to_u8(uint32_t w) {
   return make_uint2(p0 | n0, p1 | n1);
 }
 
-// Reindex scan: one CTA row per (sequence, query), each CTA scoring kRows-candidate tiles
-// gathered from the query's block list (128 / block blocks of `block` consecutive keys per
-// tile, staged by cp.async one tile ahead).
 template <int HIPAD>
 __global__ void __launch_bounds__(kScanThreads) reindex_scan_kernel(ScanArgs a) {
   chain_launch_dependents();
@@ -332,18 +421,17 @@ constexpr int kStreamThreads = kStreamWorkers + 32;       // plus the copy warp
 constexpr int kStages = 2;                                // raw tiles in flight per CTA
 constexpr int kRawTile = kRows * kIkBytes + 16;           // one tile plus its lead, 16 B multiple
 constexpr int kWorkerBar = 1;                             // named barrier of the workers
+constexpr int kStreamN = 32;                              // largest MMA N: G * HIPAD, rounded up to 16
 
 template <int MODE, int HIPAD>
 __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs a) {
   chain_enter();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = tc::align_smem_1024(smem_raw);
-  uint8_t* As = sm;                                   // 2 x [128 rows x 128 B], 128 B swizzle
-  uint8_t* Bs = As + 2 * kRows * 128;                 // [N rows x 128 B]
-  uint8_t* raw = Bs + a.N * 128;                      // kStages x kRawTile
-  int32_t* corr = reinterpret_cast<int32_t*>(raw + kStages * kRawTile);  // [N]
-  float* wq = reinterpret_cast<float*>(corr + a.N);                      // [G * HIPAD]
-  int64_t* nq = reinterpret_cast<int64_t*>(wq + a.G * HIPAD);            // [G] visible count per query
+  uint8_t* Bs = sm;                                   // hi, lo x 2 K-halves x [N rows x 128 B]
+  uint8_t* raw = Bs + 4 * a.N * 128;                  // kStages x kRawTile
+  float* wq = reinterpret_cast<float*>(raw + kStages * kRawTile);        // [N] head weight / S
+  int64_t* nq = reinterpret_cast<int64_t*>(wq + a.N);                    // [G] visible count per query
   uint64_t* full = reinterpret_cast<uint64_t*>(nq + a.G);                // [kStages] raw tile landed
   uint64_t* empty = full + kStages;                                      // [kStages] raw tile consumed
   uint64_t* dfull = empty + kStages;                                     // [2] accumulator ready
@@ -382,53 +470,19 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
     tc::mbar_init(dfull_a + 8, 1);
   }
 
-  // ---- B operand: four int8 limbs of every (query, head), plus epilogue constants ---------
-  for (int gh = warp; gh < a.G * HIPAD; gh += kStreamThreads / 32) {
+  // ---- B operands: hi and lo f16 rows of every (query, head), zero padding rows ----------
+  for (int gh = warp; gh < a.N; gh += kStreamThreads / 32) {
     const int g = gh / HIPAD, h = gh % HIPAD;
     const bool live = g < G && h < a.HI;
-    float x[4] = {0.f, 0.f, 0.f, 0.f};
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     float wv = 0.f;
     if (live) {
       const int64_t bq = (int64_t)b * a.Q + q0 + g;
-      const float4 v = reinterpret_cast<const float4*>(a.q + (bq * a.HI + h) * kDI)[lane];
-      x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+      v = reinterpret_cast<const float4*>(a.q + (bq * a.HI + h) * kDI)[lane];
       wv = a.w[bq * a.HI + h];
     }
-    float m = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    // power-of-two scale S = 2^(5 - exponent(m)): x = q*S is exact and |x| < 64, so the
-    // first limb never leaves int8 and the limbs represent x to 2^-21 (heads whose max is
-    // below 1e-30 count as zero)
-    float S = 0.f;
-    if (m > 1e-30f) {
-      const int E = (int)((__float_as_uint(m) >> 23) & 0xFFu) - 127;
-      S = __uint_as_float((uint32_t)(127 + 5 - E) << 23);
-    }
-    uint32_t limb[4] = {0u, 0u, 0u, 0u};
-    int lsum[4] = {0, 0, 0, 0};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float r = x[e] * S;
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const float L = rintf(r);
-        const int li = (int)L;
-        limb[p] |= ((uint32_t)(li & 0xFF)) << (8 * e);
-        lsum[p] += li;
-        r = (r - L) * 128.0f;
-      }
-    }
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const int n = gh * 4 + p;
-      *reinterpret_cast<uint32_t*>(Bs + tc::sw128(n, lane * 4)) = limb[p];
-      int t = lsum[p];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-      if (lane == 0) corr[n] = 0x4B400000 - 12 * t;
-    }
-    if (lane == 0) wq[gh] = S > 0.f ? wv / (2.0f * S) : 0.f;
+    const float inv = build_b_head(Bs, a.N, gh, v);
+    if (lane == 0) wq[gh] = wv * inv;
   }
   tc::fence_async_smem();
   tc::fence_before_sync();
@@ -475,83 +529,57 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
   } else {
     // ---- workers ----------------------------------------------------------------------------
     const int row = tid;
-    const uint32_t idesc = tc::idesc_i8(kRows, a.N, false, true);
+    const uint32_t idesc = tc::idesc_f16(kRows, a.N, false, false);
+    // tensor memory: the A tile in columns [0, 64), accumulator u in [64 + u*N, 64 + (u+1)*N)
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-    const uint32_t corr_a = tc::smem_u32(corr), wq_a = tc::smem_u32(wq), nq_a = tc::smem_u32(nq);
+    const uint32_t wq_a = tc::smem_u32(wq), nq_a = tc::smem_u32(nq);
 
-    // build tile t's A row (buffer t & 1) from its raw buffer; false if the copy never landed
+    // build tile t's A row from its raw buffer (the previous tile's MMAs have completed);
+    // false if the copy never landed
     auto build = [&](int t, float& sj, bool& valid) -> bool {
       const int s = t % kStages;
       const bool ok = tc::mbar_wait(full_a + 8 * s, (uint32_t)(t / kStages) & 1u, kScanPolls);
       const int64_t j = item0 + (int64_t)t * kRows + row;
       valid = ok && j < limit;
-      sj = 0.f;
-      if (valid) {
-        const uint32_t ea = raw_a + s * kRawTile + lead + row * kIkBytes;
-        const uint32_t a_row = tc::smem_u32(As) + (uint32_t)(t & 1) * (kRows * 128u) + (uint32_t)row * 128u;
-        uint32_t cw[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) cw[i] = tc::ld_shared_u32(ea + 4 * i);
-        sj = __uint_as_float(tc::ld_shared_u32(ea + 64));
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {  // 16 codes -> one 16 B chunk of the A row
-          const uint2 lo = codes_to_u8(cw[2 * c8]);
-          const uint2 hi = codes_to_u8(cw[2 * c8 + 1]);
-          tc::st_shared_v4(a_row + (((uint32_t)c8 ^ (row & 7u)) << 4), make_uint4(lo.x, lo.y, hi.x, hi.y));
-        }
-      }
+      const uint32_t ea = raw_a + s * kRawTile + lead + row * kIkBytes;
+      build_a_row(lane_addr, ea, valid);
+      sj = valid ? __uint_as_float(tc::ld_shared_u32(ea + 64)) : 0.f;
       if (ok) tc::mbar_arrive(empty_a + 8 * s);
-      tc::fence_async_smem();
       tc::fence_before_sync();
       return ok;
     };
-    // tile t: A buffer t & 1 -> accumulator t & 1 (columns (t & 1) * N), completion on dfull[t & 1]
+    // tile t: the A tile -> accumulator t & 1, completion on dfull[t & 1]
     auto issue = [&](int t) {
       if (tid == 0) {
         tc::fence_after_sync();
-        const uint32_t ab = tc::smem_u32(As) + (uint32_t)(t & 1) * (kRows * 128u), bb = tc::smem_u32(Bs);
-        const uint32_t d = tmem + (uint32_t)((t & 1) * a.N);
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)  // K = 128 dims in steps of 32
-          tc::mma_i8(d, tc::smem_desc_sw128(ab + ks * 32, 16, 1024), tc::smem_desc_sw128(bb + ks * 32, 16, 1024),
-                     idesc, ks > 0 ? 1u : 0u);
+        issue_tile_mma(tmem + (uint32_t)(kATmemCols + (t & 1) * a.N), tmem, tc::smem_u32(Bs), a.N, idesc);
         tc::commit(dfull_a + 8u * (uint32_t)(t & 1));
       }
     };
-    // limbs -> fp32 dot products -> ReLU-weighted score -> order-preserving keys of tile t
+    // dot products -> ReLU-weighted score -> order-preserving keys of tile t
     auto epilogue = [&](int t, float sj, bool valid) -> bool {
       const bool ok = tc::mbar_wait(dfull_a + 8u * (uint32_t)(t & 1), (uint32_t)(t >> 1) & 1u, kScanPolls);
       tc::fence_after_sync();
       const int64_t j = item0 + (int64_t)t * kRows + row;
-      const uint32_t acc = lane_addr + (uint32_t)((t & 1) * a.N);
+      const uint32_t acc = lane_addr + (uint32_t)(kATmemCols + (t & 1) * a.N);
+      uint32_t r[kStreamN];
+      if (a.N == 16)
+        tc::tmem_ld16(acc, r);
+      else
+        tc::tmem_ld32(acc, r);
+      constexpr int kGmax = kStreamN / HIPAD;
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {
+      for (int g = 0; g < kGmax; ++g) {
         if (g >= G) break;
-        uint32_t r[HIPAD * 4];
-        const uint32_t ta = acc + (uint32_t)(g * HIPAD * 4);
-        if (HIPAD == 4) {
-          tc::tmem_ld16(ta, r);
-        } else {
-#pragma unroll
-          for (int c = 0; c < HIPAD * 4; c += 32) tc::tmem_ld32(ta + c, *reinterpret_cast<uint32_t(*)[32]>(r + c));
-        }
         float tot = 0.f;
 #pragma unroll
         for (int h4 = 0; h4 < HIPAD / 4; ++h4) {
           const uint4 w4 = tc::ld_shared_v4(wq_a + (uint32_t)(g * HIPAD + h4 * 4) * 4u);
-          const float wh[4] = {__uint_as_float(w4.x), __uint_as_float(w4.y), __uint_as_float(w4.z),
-                               __uint_as_float(w4.w)};
-#pragma unroll
-          for (int hh = 0; hh < 4; ++hh) {
-            const int h = h4 * 4 + hh;
-            const uint4 c = tc::ld_shared_v4(corr_a + (uint32_t)(g * HIPAD + h) * 16u);
-            const float f0 = __int_as_float((int)(r[h * 4 + 0] + c.x)) - 12582912.0f;
-            const float f1 = __int_as_float((int)(r[h * 4 + 1] + c.y)) - 12582912.0f;
-            const float f2 = __int_as_float((int)(r[h * 4 + 2] + c.z)) - 12582912.0f;
-            const float f3 = __int_as_float((int)(r[h * 4 + 3] + c.w)) - 12582912.0f;
-            const float z = fmaf(fmaf(fmaf(f3, 0.0078125f, f2), 0.0078125f, f1), 0.0078125f, f0);
-            tot = fmaf(wh[hh], fmaxf(z, 0.f), tot);
-          }
+          const int c = g * HIPAD + h4 * 4;
+          tot = fmaf(__uint_as_float(w4.x), fmaxf(__uint_as_float(r[c + 0]), 0.f), tot);
+          tot = fmaf(__uint_as_float(w4.y), fmaxf(__uint_as_float(r[c + 1]), 0.f), tot);
+          tot = fmaf(__uint_as_float(w4.z), fmaxf(__uint_as_float(r[c + 2]), 0.f), tot);
+          tot = fmaf(__uint_as_float(w4.w), fmaxf(__uint_as_float(r[c + 3]), 0.f), tot);
         }
         const int64_t nqg = (int64_t)tc::ld_shared_u64(nq_a + 8u * (uint32_t)g);
         const bool vis = valid && j < nqg;
@@ -572,8 +600,8 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
       return ok;
     };
 
-    // step t: build and issue tile t+1, then the epilogue of tile t (whose MMA was issued
-    // one step earlier and has had the whole build to complete)
+    // step t: once tile t's MMAs have completed (they free the A tile), build and issue tile
+    // t+1, then run the epilogue of tile t while tile t+1's MMAs run
     float sj = 0.f, sj_nxt = 0.f;
     bool v = false, v_nxt = false;
     int issued = 0;  // tiles whose MMA was issued (their raw buffers were consumed)
@@ -585,7 +613,10 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
     bool pend = false;  // a failed accumulator wait, voted on at the next barrier
     for (int t = 0; t < ntiles && !bad; ++t) {
       if (t + 1 < ntiles) {
-        const bool fail = !build(t + 1, sj_nxt, v_nxt) || pend;
+        const bool mok = tc::mbar_wait(dfull_a + 8u * (uint32_t)(t & 1), (uint32_t)(t >> 1) & 1u, kScanPolls);
+        tc::fence_after_sync();
+        const bool bok = build(t + 1, sj_nxt, v_nxt);  // warp-wide: every worker builds
+        const bool fail = !mok || !bok || pend;
         bad = tc::named_sync_or(kWorkerBar, kStreamWorkers, fail);
         if (bad) break;
         issue(t + 1);
@@ -1784,16 +1815,18 @@ static cudaError_t resident_ctas(F fn, int dev, int threads, size_t dyn_smem, in
 template <int MODE>
 static cudaError_t launch_stream(ScanArgs a, int64_t items, int B, cudaStream_t st) {
   a.hipad = a.HI <= 4 ? 4 : (a.HI <= 8 ? 8 : 16);
-  // accumulator pairs of 2N <= 256 columns, so two CTAs' tensor memory fits an SM
-  a.G = max(1, min(a.Q, 128 / (a.hipad * 4)));
+  // G queries of hipad heads per CTA, N = G * hipad <= 32 columns rounded up to 16 (the
+  // smallest N of an M = 128 MMA); the A tile and the accumulator pair take 64 + 2N <= 128
+  // columns, so four CTAs' tensor memory fits an SM
+  a.G = max(1, min(a.Q, kStreamN / a.hipad));
   a.n_groups = (a.Q + a.G - 1) / a.G;
-  a.N = a.G * a.hipad * 4;
-  a.tmem_cols = pow2_at_least(2 * a.N);
+  a.N = (a.G * a.hipad + 15) / 16 * 16;
+  a.tmem_cols = pow2_at_least(kATmemCols + 2 * a.N);
   const int64_t tiles = (items + kRows - 1) / kRows;
   const int64_t rows = (int64_t)B * a.n_groups;
   if (tiles == 0 || rows == 0) return cudaSuccess;
-  const size_t smem = 1024 + 2 * (size_t)kRows * 128 + (size_t)a.N * 128 + (size_t)kStages * kRawTile +
-                      (size_t)a.N * 4 + (size_t)a.G * a.hipad * 4 + (size_t)a.G * 8 + (2 * kStages + 2) * 8 + 16;
+  const size_t smem = 1024 + 4 * (size_t)a.N * 128 + (size_t)kStages * kRawTile +
+                      (size_t)a.N * 4 + (size_t)a.G * 8 + (2 * kStages + 2) * 8 + 16;
   // Runs of tiles sized for about `waves` waves of CTAs: 2 when few query rows share the
   // sequence walk, 8 when many do (multi-query verify and prefill, 128 and 256 rows of 4
   // queries), whose longer runs per CTA otherwise leave a tail (8 waves measured 5-7% faster

@@ -430,6 +430,29 @@ def test_group_select_ragged(orc, K):
         assert_topk_set(topk[0, i], o_topk, s, K, what=f"query {i}")
 
 
+@pytest.mark.parametrize("HI", [8, 16])
+def test_score_precision(orc, HI):
+    """The scores the scan reports for its Top-K against the oracle's fp64 scores of the same
+    entries: the query heads' two f16 parts carry 22 significant bits and the products are
+    exact, so only the fp32 sums round; every reported score is within 1e-6 relative."""
+    T, Q, K = 40000, 8, 512
+    kv, ik = synth.kv_tokens(51, T, recipe="rmsnorm")
+    kvp, ikp, _, o_ik = pools_from_tokens(orc, kv.cuda(), ik.cuda())
+    q, w = synth.index_queries(52, 1, Q, HI)
+    n_vis = torch.full((1, Q), T, dtype=torch.int32)
+    topk, score, st = run_full(q.cuda(), w.cuda(), ikp, torch.zeros(1, dtype=torch.int64, device="cuda"),
+                               n_vis.cuda(), K, T)
+    assert st == 0
+    worst = 0.0
+    for i in range(Q):
+        s = orc.index_scores(q[0, i].numpy(), w[0, i].numpy(), o_ik)
+        sel = topk[0, i]
+        assert (sel >= 0).all()
+        rel = np.abs(score[0, i].astype(np.float64) - s[sel]) / np.abs(s[sel])
+        worst = max(worst, float(rel.max()))
+    assert worst <= 1e-6, f"largest relative score error {worst:.3e}"
+
+
 @pytest.mark.parametrize("nv", [300, 512, 513, 16384])
 def test_cluster_select_few_valid_keys(orc, nv):
     """A 16,384-key flat selection runs as a cluster of 4 register CTAs, which learns how many
