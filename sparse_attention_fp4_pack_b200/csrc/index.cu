@@ -105,13 +105,14 @@ __device__ __forceinline__ void stage_async(uint32_t dst, const uint8_t* src, in
 
 constexpr int kATmemCols = 64;       // an A tile in tensor memory: 128 f16 per lane, two per column
 
-// Row n of the B operands for one query head, from the head's 128 fp32 elements (lane l holds
-// elements 4l..4l+3; zeros for a padding row).  x = q*S with S = 2^(14 - exponent(max|q|)),
-// so |x| < 2^15 and the scaling is exact; hi = f16(x) and lo = f16(x - hi) (x - hi is exact in
-// fp32) represent x to 2^-22 of each element.  The hi operand sits at Bs and the lo operand at
-// Bs + 2*npad*128, each as two 128-byte-swizzled K-halves of npad rows (elements 0..63 and
-// 64..127).  Returns 1/S (0 for a head whose largest element is below 1e-30).
-__device__ __forceinline__ float build_b_head(uint8_t* Bs, int npad, int n, float4 v) {
+// The B rows of one query head, from the head's 128 fp32 elements (lane l holds elements
+// 4l..4l+3; zeros for a padding row).  x = q*S with S = 2^(14 - exponent(max|q|)), so
+// |x| < 2^15 and the scaling is exact; hi = f16(x) and lo = f16(x - hi) (x - hi is exact in
+// fp32) represent x to 2^-22 of each element.  hi goes to row n of the operand at Bs and lo to
+// row n_lo of the operand at Blo (the same operand when the two are stacked along N); an
+// operand is two 128-byte-swizzled K-halves of npad rows (elements 0..63 and 64..127).
+// Returns 1/S (0 for a head whose largest element is below 1e-30).
+__device__ __forceinline__ float build_b_head(uint8_t* Bs, uint8_t* Blo, int npad, int n, int n_lo, float4 v) {
   const int lane = threadIdx.x & 31;
   float m = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
 #pragma unroll
@@ -132,20 +133,19 @@ __device__ __forceinline__ float build_b_head(uint8_t* Bs, int npad, int n, floa
     hw[e] = *reinterpret_cast<const uint32_t*>(&h);
     lw[e] = *reinterpret_cast<const uint32_t*>(&l);
   }
-  const uint32_t off = (uint32_t)(lane >> 4) * (uint32_t)npad * 128u + tc::sw128((uint32_t)n, (uint32_t)(lane & 15) * 8u);
-  *reinterpret_cast<uint2*>(Bs + off) = make_uint2(hw[0], hw[1]);
-  *reinterpret_cast<uint2*>(Bs + 2u * (uint32_t)npad * 128u + off) = make_uint2(lw[0], lw[1]);
+  const uint32_t kh = (uint32_t)(lane >> 4) * (uint32_t)npad * 128u, byte = (uint32_t)(lane & 15) * 8u;
+  *reinterpret_cast<uint2*>(Bs + kh + tc::sw128((uint32_t)n, byte)) = make_uint2(hw[0], hw[1]);
+  *reinterpret_cast<uint2*>(Blo + kh + tc::sw128((uint32_t)n_lo, byte)) = make_uint2(lw[0], lw[1]);
   return inv;
 }
 
-// The 16 MMAs of one tile: A (its 128 x 128 f16 in tensor memory, 64 columns from a_tmem)
-// times the hi and then the lo B operand (each two swizzled K-halves of npad rows at b_addr),
-// all accumulating into the npad columns at d.
-__device__ __forceinline__ void issue_tile_mma(uint32_t d, uint32_t a_tmem, uint32_t b_addr, int npad,
+// The MMAs of one tile: A (its 128 x 128 f16 in tensor memory, 64 columns from a_tmem) times
+// `parts` B operands at b_addr (each two swizzled K-halves of npad rows: hi and then lo, or one
+// operand holding both), all accumulating into the npad columns at d; 8 MMAs per operand.
+__device__ __forceinline__ void issue_tile_mma(uint32_t d, uint32_t a_tmem, uint32_t b_addr, int npad, int parts,
                                                uint32_t idesc) {
   const uint32_t bh = (uint32_t)npad * 128u;  // one K-half of one B operand
-#pragma unroll
-  for (int p = 0; p < 2; ++p)
+  for (int p = 0; p < parts; ++p)
 #pragma unroll
     for (int kh = 0; kh < 2; ++kh)
 #pragma unroll
@@ -471,7 +471,11 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
   }
 
   // ---- B operands: hi and lo f16 rows of every (query, head), zero padding rows ----------
-  for (int gh = warp; gh < a.N; gh += kStreamThreads / 32) {
+  // One query (G = 1): hi in rows [0, HIPAD) and lo in rows [HIPAD, 2 HIPAD) of one operand,
+  // filling N's padding, so a tile takes 8 MMAs; else the hi and lo operands, 16 MMAs.
+  const bool stacked = a.G == 1;
+  const int nb = stacked ? HIPAD : a.N;  // B rows built from heads
+  for (int gh = warp; gh < nb; gh += kStreamThreads / 32) {
     const int g = gh / HIPAD, h = gh % HIPAD;
     const bool live = g < G && h < a.HI;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -481,9 +485,15 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
       v = reinterpret_cast<const float4*>(a.q + (bq * a.HI + h) * kDI)[lane];
       wv = a.w[bq * a.HI + h];
     }
-    const float inv = build_b_head(Bs, a.N, gh, v);
+    const float inv = stacked ? build_b_head(Bs, Bs, a.N, gh, HIPAD + gh, v)
+                              : build_b_head(Bs, Bs + 2 * a.N * 128, a.N, gh, gh, v);
     if (lane == 0) wq[gh] = wv * inv;
   }
+  if (stacked)  // rows [2 HIPAD, N) of both K-halves are zero
+    for (int i = tid; i < 2 * (a.N - 2 * HIPAD) * 32; i += kStreamThreads) {
+      const int kh = i / ((a.N - 2 * HIPAD) * 32), rest = i % ((a.N - 2 * HIPAD) * 32);
+      *reinterpret_cast<uint32_t*>(Bs + kh * a.N * 128 + (2 * HIPAD + rest / 32) * 128 + (rest % 32) * 4) = 0u;
+    }
   tc::fence_async_smem();
   tc::fence_before_sync();
   __syncthreads();
@@ -552,7 +562,8 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
     auto issue = [&](int t) {
       if (tid == 0) {
         tc::fence_after_sync();
-        issue_tile_mma(tmem + (uint32_t)(kATmemCols + (t & 1) * a.N), tmem, tc::smem_u32(Bs), a.N, idesc);
+        issue_tile_mma(tmem + (uint32_t)(kATmemCols + (t & 1) * a.N), tmem, tc::smem_u32(Bs), a.N,
+                       stacked ? 1 : 2, idesc);
         tc::commit(dfull_a + 8u * (uint32_t)(t & 1));
       }
     };
@@ -572,14 +583,30 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
       for (int g = 0; g < kGmax; ++g) {
         if (g >= G) break;
         float tot = 0.f;
+        if (stacked) {  // one query: head h's hi sum in column h, its lo sum in column HIPAD + h
 #pragma unroll
-        for (int h4 = 0; h4 < HIPAD / 4; ++h4) {
-          const uint4 w4 = tc::ld_shared_v4(wq_a + (uint32_t)(g * HIPAD + h4 * 4) * 4u);
-          const int c = g * HIPAD + h4 * 4;
-          tot = fmaf(__uint_as_float(w4.x), fmaxf(__uint_as_float(r[c + 0]), 0.f), tot);
-          tot = fmaf(__uint_as_float(w4.y), fmaxf(__uint_as_float(r[c + 1]), 0.f), tot);
-          tot = fmaf(__uint_as_float(w4.z), fmaxf(__uint_as_float(r[c + 2]), 0.f), tot);
-          tot = fmaf(__uint_as_float(w4.w), fmaxf(__uint_as_float(r[c + 3]), 0.f), tot);
+          for (int h4 = 0; h4 < HIPAD / 4; ++h4) {
+            const uint4 w4 = tc::ld_shared_v4(wq_a + (uint32_t)(h4 * 4) * 4u);
+            const int c = h4 * 4;
+            const float z0 = __uint_as_float(r[c + 0]) + __uint_as_float(r[HIPAD + c + 0]);
+            const float z1 = __uint_as_float(r[c + 1]) + __uint_as_float(r[HIPAD + c + 1]);
+            const float z2 = __uint_as_float(r[c + 2]) + __uint_as_float(r[HIPAD + c + 2]);
+            const float z3 = __uint_as_float(r[c + 3]) + __uint_as_float(r[HIPAD + c + 3]);
+            tot = fmaf(__uint_as_float(w4.x), fmaxf(z0, 0.f), tot);
+            tot = fmaf(__uint_as_float(w4.y), fmaxf(z1, 0.f), tot);
+            tot = fmaf(__uint_as_float(w4.z), fmaxf(z2, 0.f), tot);
+            tot = fmaf(__uint_as_float(w4.w), fmaxf(z3, 0.f), tot);
+          }
+        } else {
+#pragma unroll
+          for (int h4 = 0; h4 < HIPAD / 4; ++h4) {
+            const uint4 w4 = tc::ld_shared_v4(wq_a + (uint32_t)(g * HIPAD + h4 * 4) * 4u);
+            const int c = g * HIPAD + h4 * 4;
+            tot = fmaf(__uint_as_float(w4.x), fmaxf(__uint_as_float(r[c + 0]), 0.f), tot);
+            tot = fmaf(__uint_as_float(w4.y), fmaxf(__uint_as_float(r[c + 1]), 0.f), tot);
+            tot = fmaf(__uint_as_float(w4.z), fmaxf(__uint_as_float(r[c + 2]), 0.f), tot);
+            tot = fmaf(__uint_as_float(w4.w), fmaxf(__uint_as_float(r[c + 3]), 0.f), tot);
+          }
         }
         const int64_t nqg = (int64_t)tc::ld_shared_u64(nq_a + 8u * (uint32_t)g);
         const bool vis = valid && j < nqg;
@@ -1820,7 +1847,8 @@ static cudaError_t launch_stream(ScanArgs a, int64_t items, int B, cudaStream_t 
   // columns, so four CTAs' tensor memory fits an SM
   a.G = max(1, min(a.Q, kStreamN / a.hipad));
   a.n_groups = (a.Q + a.G - 1) / a.G;
-  a.N = (a.G * a.hipad + 15) / 16 * 16;
+  // one query stacks its hi and lo rows in one operand of 2 * hipad rows
+  a.N = ((a.G == 1 ? 2 : a.G) * a.hipad + 15) / 16 * 16;
   a.tmem_cols = pow2_at_least(kATmemCols + 2 * a.N);
   const int64_t tiles = (items + kRows - 1) / kRows;
   const int64_t rows = (int64_t)B * a.n_groups;
