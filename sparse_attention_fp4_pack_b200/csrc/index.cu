@@ -406,19 +406,20 @@ __global__ void __launch_bounds__(kScanThreads) reindex_scan_kernel(ScanArgs a) 
 //     copy into a ring of kStages raw buffers, up to kStages tiles ahead of the math; the
 //     copy starts at the 16 B boundary at or below the tile's first key (that lead,
 //     0..12 bytes, is the same for every tile of a sequence) and is rounded up to 16 B,
-//     falling back to word copies when the rounded copy would run past the pool;
-//   * the four worker warps own one tile row each.  The A operand and the accumulator are
-//     doubled: the workers build tile t+1's A rows, thread 0 issues its MMA into the other
-//     accumulator, and only then do they run tile t's epilogue, whose MMA finished during
-//     the previous step, so the MMA round trip never waits on the chain.
-// The CTA is small (about 56 KB of shared memory, 160 threads), so four of them share an
-// SM and hide each other's copy latency.  Every wait is bounded; the workers
-// agree on giving up through a reducing barrier, and the copy warp waits for its
-// outstanding copies before the CTA exits.
+//     falling back to word copies when the rounded copy would run past the pool.  It also
+//     issues each tile's MMAs once the workers report the tile's A rows built;
+//   * the four worker warps own one tile row each.  The accumulator is doubled: once tile
+//     t's MMAs have completed (they free the A tile in tensor memory), the workers build
+//     tile t+1's rows and report them, then run tile t's epilogue while tile t+1's MMAs run.
+//     No worker issues MMAs, so none lags the others at the per-tile vote.
+// Four CTAs share an SM (tensor memory: the A tile and the accumulator pair, at most 128
+// columns).  Every wait is bounded; the workers agree on giving up through a reducing
+// barrier and tell the copy warp, and the copy warp waits for its outstanding copies and
+// MMAs before the CTA exits.
 // ------------------------------------------------------------------------------------
 constexpr int kStreamWorkers = 128;                       // one tile row per thread
 constexpr int kStreamThreads = kStreamWorkers + 32;       // plus the copy warp
-constexpr int kStages = 2;                                // raw tiles in flight per CTA
+constexpr int kStages = 4;                                // raw tiles in flight per CTA
 constexpr int kRawTile = kRows * kIkBytes + 16;           // one tile plus its lead, 16 B multiple
 constexpr int kWorkerBar = 1;                             // named barrier of the workers
 constexpr int kStreamN = 32;                              // largest MMA N: G * HIPAD, rounded up to 16
@@ -435,7 +436,8 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
   uint64_t* full = reinterpret_cast<uint64_t*>(nq + a.G);                // [kStages] raw tile landed
   uint64_t* empty = full + kStages;                                      // [kStages] raw tile consumed
   uint64_t* dfull = empty + kStages;                                     // [2] accumulator ready
-  uint32_t* misc = reinterpret_cast<uint32_t*>(dfull + 2);               // tmem base, tiles built, issued
+  uint64_t* built = dfull + 2;                                           // the A tile is built
+  uint32_t* misc = reinterpret_cast<uint32_t*>(built + 1);  // tmem base, tiles consumed, copied, stop, issued
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b = blockIdx.y / a.n_groups;
@@ -468,6 +470,7 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
     }
     tc::mbar_init(dfull_a, 1);
     tc::mbar_init(dfull_a + 8, 1);
+    tc::mbar_init(tc::smem_u32(built), 1);
   }
 
   // ---- B operands: hi and lo f16 rows of every (query, head), zero padding rows ----------
@@ -500,20 +503,23 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
   tc::fence_after_sync();
   const uint32_t tmem = misc[0];
 
+  const uint32_t built_a = tc::smem_u32(built);
+  const uint32_t idesc = tc::idesc_f16(kRows, a.N, false, false);
   if (warp == kStreamWorkers / 32) {
-    // ---- copy warp ------------------------------------------------------------------------
+    // ---- copy and MMA warp ------------------------------------------------------------------
+    // Tile t's MMAs go out once the workers report its A tile built; that report also frees
+    // its raw buffer, so tile t + kStages is copied right after.
     const uint8_t* pool_end = a.ik_pool + a.pool_entries * kIkBytes;
-    int issued = 0;
-    bool ok = true;
-    for (int t = 0; t < ntiles; ++t) {
+    int copied = 0, mma_issued = 0;
+    bool ok = true, withheld = false;
+    auto copy_tile = [&](int t) -> bool {
       // test hook: stop copying, so the workers' wait for this tile runs out
-      if (t == a.withheld_tile && blockIdx.x == 0 && blockIdx.y == 0) break;
+      if (t == a.withheld_tile && blockIdx.x == 0 && blockIdx.y == 0) withheld = true;
+      if (withheld) return true;
       const int s = t % kStages;
-      if (t >= kStages) ok = tc::mbar_wait(empty_a + 8 * s, (uint32_t)((t / kStages) - 1) & 1u, kScanPolls);
-      if (!__all_sync(0xffffffffu, ok)) {
-        ok = false;
-        break;
-      }
+      bool cok = true;
+      if (t >= kStages) cok = tc::mbar_wait(empty_a + 8 * s, (uint32_t)((t / kStages) - 1) & 1u, kScanPolls);
+      if (!__all_sync(0xffffffffu, cok)) return false;
       const int64_t i0 = item0 + (int64_t)t * kRows;
       const int cnt = (int)(limit - i0 < kRows ? limit - i0 : kRows);
       const uint8_t* src = seq + i0 * kIkBytes;
@@ -530,16 +536,31 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(full_a + 8 * s);
       }
-      issued = t + 1;
+      copied = t + 1;
+      return true;
+    };
+    for (int t = 0; t < ntiles && t < kStages && ok; ++t) ok = copy_tile(t);
+    for (int t = 0; t < ntiles && ok; ++t) {
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(built_a, (uint32_t)t & 1u, kScanPolls));
+      if (!ok || misc[3] != 0u) break;  // no report, or the workers gave up
+      if (lane == 0) {
+        tc::fence_after_sync();
+        issue_tile_mma(tmem + (uint32_t)(kATmemCols + (t & 1) * a.N), tmem, tc::smem_u32(Bs), a.N,
+                       a.G == 1 ? 1 : 2, idesc);
+        tc::commit(dfull_a + 8u * (uint32_t)(t & 1));
+      }
+      mma_issued = t + 1;
+      __syncwarp();
+      if (t + kStages < ntiles) ok = copy_tile(t + kStages);
     }
     if (lane == 0) {
       if (!ok) flag(a.status, CSA2_DEV_TIMEOUT);
-      misc[2] = (uint32_t)issued;
+      misc[2] = (uint32_t)copied;
+      misc[4] = (uint32_t)mma_issued;
     }
   } else {
     // ---- workers ----------------------------------------------------------------------------
     const int row = tid;
-    const uint32_t idesc = tc::idesc_f16(kRows, a.N, false, false);
     // tensor memory: the A tile in columns [0, 64), accumulator u in [64 + u*N, 64 + (u+1)*N)
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
     const uint32_t wq_a = tc::smem_u32(wq), nq_a = tc::smem_u32(nq);
@@ -558,13 +579,12 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
       tc::fence_before_sync();
       return ok;
     };
-    // tile t: the A tile -> accumulator t & 1, completion on dfull[t & 1]
-    auto issue = [&](int t) {
+    // report tile t's A tile built (after the workers' vote, which orders their tensor-memory
+    // stores before it), or that the workers gave up
+    auto report = [&](bool give_up) {
       if (tid == 0) {
-        tc::fence_after_sync();
-        issue_tile_mma(tmem + (uint32_t)(kATmemCols + (t & 1) * a.N), tmem, tc::smem_u32(Bs), a.N,
-                       stacked ? 1 : 2, idesc);
-        tc::commit(dfull_a + 8u * (uint32_t)(t & 1));
+        misc[3] = give_up ? 1u : 0u;
+        tc::mbar_arrive(built_a);
       }
     };
     // dot products -> ReLU-weighted score -> order-preserving keys of tile t
@@ -627,27 +647,24 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
       return ok;
     };
 
-    // step t: once tile t's MMAs have completed (they free the A tile), build and issue tile
-    // t+1, then run the epilogue of tile t while tile t+1's MMAs run
+    // step t: once tile t's MMAs have completed (they free the A tile), build tile t+1 and
+    // report it to the MMA warp, then run the epilogue of tile t while tile t+1's MMAs run
     float sj = 0.f, sj_nxt = 0.f;
     bool v = false, v_nxt = false;
-    int issued = 0;  // tiles whose MMA was issued (their raw buffers were consumed)
+    int consumed = 0;  // tiles whose raw buffers every worker has read
     bool bad = tc::named_sync_or(kWorkerBar, kStreamWorkers, !build(0, sj, v));
-    if (!bad) {
-      issue(0);
-      issued = 1;
-    }
+    report(bad);
+    if (!bad) consumed = 1;
     bool pend = false;  // a failed accumulator wait, voted on at the next barrier
     for (int t = 0; t < ntiles && !bad; ++t) {
       if (t + 1 < ntiles) {
         const bool mok = tc::mbar_wait(dfull_a + 8u * (uint32_t)(t & 1), (uint32_t)(t >> 1) & 1u, kScanPolls);
         tc::fence_after_sync();
         const bool bok = build(t + 1, sj_nxt, v_nxt);  // warp-wide: every worker builds
-        const bool fail = !mok || !bok || pend;
-        bad = tc::named_sync_or(kWorkerBar, kStreamWorkers, fail);
+        bad = tc::named_sync_or(kWorkerBar, kStreamWorkers, !mok || !bok || pend);
+        report(bad);
         if (bad) break;
-        issue(t + 1);
-        issued = t + 2;
+        consumed = t + 2;
       }
       pend |= !epilogue(t, sj, v);
       sj = sj_nxt;
@@ -657,15 +674,16 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
     bad = tc::named_sync_or(kWorkerBar, kStreamWorkers, bad || pend);
     if (tid == 0) {
       if (bad) flag(a.status, CSA2_DEV_TIMEOUT);
-      // let the issued MMAs finish before the accumulators go (they complete in order)
-      if (bad && issued > 0)
-        tc::mbar_wait(dfull_a + 8u * (uint32_t)((issued - 1) & 1), (uint32_t)((issued - 1) >> 1) & 1u, kScanPolls);
-      misc[1] = (uint32_t)(bad ? issued : ntiles);
+      misc[1] = (uint32_t)(bad ? consumed : ntiles);
     }
   }
   __syncthreads();
-  if (tid == kStreamWorkers) {  // copies that landed in no tile the workers consumed
-    for (int t = (int)misc[1]; t < (int)misc[2]; ++t)
+  if (tid == kStreamWorkers) {
+    // the last issued MMAs finish before the accumulators go (they complete in order; no later
+    // commit on that barrier, so its phase is still the one to wait for)
+    const int last = (int)misc[4] - 1;
+    if (last >= 0) tc::mbar_wait(dfull_a + 8u * (uint32_t)(last & 1), (uint32_t)(last >> 1) & 1u, kScanPolls);
+    for (int t = (int)misc[1]; t < (int)misc[2]; ++t)  // copies that landed in no consumed tile
       tc::mbar_wait(full_a + 8 * (t % kStages), (uint32_t)(t / kStages) & 1u, kScanPolls);
   }
   tc::fence_before_sync();
@@ -1854,7 +1872,7 @@ static cudaError_t launch_stream(ScanArgs a, int64_t items, int B, cudaStream_t 
   const int64_t rows = (int64_t)B * a.n_groups;
   if (tiles == 0 || rows == 0) return cudaSuccess;
   const size_t smem = 1024 + 4 * (size_t)a.N * 128 + (size_t)kStages * kRawTile +
-                      (size_t)a.N * 4 + (size_t)a.G * 8 + (2 * kStages + 2) * 8 + 16;
+                      (size_t)a.N * 4 + (size_t)a.G * 8 + (2 * kStages + 3) * 8 + 32;
   // Runs of tiles sized for about `waves` waves of CTAs: 2 when few query rows share the
   // sequence walk, 8 when many do (multi-query verify and prefill, 128 and 256 rows of 4
   // queries), whose longer runs per CTA otherwise leave a tail (8 waves measured 5-7% faster
