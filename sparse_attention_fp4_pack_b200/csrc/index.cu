@@ -775,9 +775,10 @@ __device__ __forceinline__ int64_t item_label(const SelectArgs& a, const int32_t
 
 // Block-wide exclusive prefix sum of one value per thread (kSelThreads threads) of a
 // 64-bit packed pair; ws holds kSelThreads/32 + 1 entries.
+template <int NT = kSelThreads>
 __device__ __forceinline__ uint64_t block_excl_scan64(uint64_t v, uint64_t* ws, uint64_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  constexpr int nw = kSelThreads / 32;
+  constexpr int nw = NT / 32;
   uint64_t x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -1051,7 +1052,6 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
     if (C == 1 && nchunks > 1 && a.gmax != nullptr) {
       constexpr int kGroupList = 8192;
       static_assert(2 * kGroupList <= kKeyWords, "the group list is kept where the chunks would be");
-      constexpr int kWarps = kSelThreads / 32, kU = 8;  // a warp reads kU groups at a time
       const uint32_t* gm = a.gmax + (int64_t)bq * a.gstride;
       const int ng = (int)((n + 31) >> 5);
       uint32_t gc = 0u;
@@ -1113,27 +1113,30 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
         for (int g = g0; g < g1; ++g)
           if (gm[g] >= x) gl[so++] = (uint32_t)g;
         __syncthreads();
-        const int warp = tid >> 5;
-        // the keys of kU listed groups of this warp (0 past the list and past n)
-        auto group_keys = [&](int s0, uint32_t (&kk)[kU]) {
+        // a thread takes whole groups: its 32 keys in eight 16-byte loads, all in flight at
+        // once (keys past n read as 0)
+        auto group_keys = [&](int sidx, uint32_t (&kk)[32]) {
+          const int64_t i0 = (int64_t)gl[sidx] * 32;
+          const uint4* src = reinterpret_cast<const uint4*>(keys + i0);
 #pragma unroll
-          for (int u = 0; u < kU; ++u) {
-            const int sidx = s0 + u * kWarps;
-            kk[u] = 0u;
-            if (sidx < S) {
-              const int64_t i = (int64_t)gl[sidx] * 32 + lane;
-              if (i < n) kk[u] = keys[i];
-            }
+          for (int v = 0; v < 8; ++v) {
+            const uint4 q = i0 + 4 * v + 3 < n ? src[v] : make_uint4(0u, 0u, 0u, 0u);
+            kk[4 * v] = q.x;
+            kk[4 * v + 1] = q.y;
+            kk[4 * v + 2] = q.z;
+            kk[4 * v + 3] = q.w;
           }
+          if (i0 + 32 > n)  // the tail group: word loads of its keys below n
+#pragma unroll
+            for (int e = 0; e < 32; ++e) kk[e] = i0 + e < n ? keys[i0 + e] : 0u;
         };
-        for (int s0 = warp; s0 < S; s0 += kWarps * kU) {
-          uint32_t kk[kU];
-          group_keys(s0, kk);
+        for (int sidx = tid; sidx < S; sidx += kSelThreads) {
+          uint32_t kk[32];
+          group_keys(sidx, kk);
+          uint32_t c = 0u;
 #pragma unroll
-          for (int u = 0; u < kU; ++u) {
-            const uint32_t m = __ballot_sync(0xffffffffu, kk[u] >= x);
-            if (lane == 0 && s0 + u * kWarps < S) goff[s0 + u * kWarps] = (uint32_t)__popc(m);
-          }
+          for (int e = 0; e < 32; ++e) c += kk[e] >= x ? 1u : 0u;
+          goff[sidx] = c;
         }
         __syncthreads();
         const int per2 = (S + kSelThreads - 1) / kSelThreads;
@@ -1150,19 +1153,18 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
             co += c;
           }
           __syncthreads();
-          for (int sw = warp; sw < S; sw += kWarps * kU) {
-            uint32_t kk[kU];
-            group_keys(sw, kk);
+          for (int sidx = tid; sidx < S; sidx += kSelThreads) {
+            uint32_t kk[32];
+            group_keys(sidx, kk);
+            uint32_t pos = goff[sidx];
+            const int32_t gi = (int32_t)gl[sidx] * 32;
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-              const uint32_t m = __ballot_sync(0xffffffffu, kk[u] >= x);
-              if (kk[u] >= x) {
-                const int sidx = sw + u * kWarps;
-                const uint32_t pos = goff[sidx] + (uint32_t)__popc(m & ((1u << lane) - 1u));
-                candk[pos] = kk[u];
-                candi[pos] = (int32_t)(gl[sidx] * 32u + (uint32_t)lane);
+            for (int e = 0; e < 32; ++e)
+              if (kk[e] >= x) {
+                candk[pos] = kk[e];
+                candi[pos] = gi + e;
+                ++pos;
               }
-            }
           }
           if (nc <= K) {  // every valid key (fewer than K groups), in index order, then -1
             __syncthreads();
@@ -1506,6 +1508,314 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
     }
   }
   if (C > 1) cluster.sync();  // keep every CTA's shared memory alive until remote reads are done
+}
+
+// Flat selection with the scan's group maxima, one small CTA per query (many queries: verify,
+// prefill).  The same threshold and list method as select_kernel's one-CTA group path, in 256
+// threads and 48 KB of shared memory, so four CTAs share an SM and a verify step's 512
+// queries take one wave.  The 12-bit histogram of the maxima and the key list share one area
+// (the list is written after the histogram is read), as do the radix histograms and the
+// group list.  When the groups at or above x or their keys do not fit, the CTA selects
+// exactly over all n keys from global memory instead (radix levels, one pass per level).
+constexpr int kGsThreads = 256;
+constexpr int kGsList = 2048;   // groups at or above the threshold
+constexpr int kGsCand = 4096;   // keys at or above the threshold
+constexpr int kGsSmemBytes = (kGsCand * 2 + 2 * kGsList + 64 + 16) * 4;
+
+__global__ void __launch_bounds__(kGsThreads) group_select_kernel(SelectArgs a) {
+  chain_launch_dependents();
+  extern __shared__ __align__(16) uint32_t gs_smem[];
+  uint32_t* sub = gs_smem;                                        // [4096] maxima histogram
+  uint32_t* candk = gs_smem;                                      // [kGsCand] listed keys (after sub)
+  int32_t* candi = reinterpret_cast<int32_t*>(gs_smem + kGsCand);  // [kGsCand] their indices
+  uint32_t* hist = gs_smem + 2 * kGsCand;                         // [kBins]
+  uint32_t* hsum = hist + kBins;                                  // [kBins]
+  uint32_t* gl = hist;                                            // [kGsList] groups (after hist/hsum)
+  uint32_t* goff = gl + kGsList;                                  // [kGsList]
+  uint64_t* scan_ws = reinterpret_cast<uint64_t*>(gl + 2 * kGsList);  // [kGsThreads/32 + 1]
+  uint32_t* misc = reinterpret_cast<uint32_t*>(scan_ws + 32);         // [8]
+  static_assert(2 * kBins <= 2 * kGsList, "the radix histograms fit the group list area");
+  static_assert(4096 <= kGsCand, "the maxima histogram fits the key list area");
+  const int tid = threadIdx.x;
+  const int bq = blockIdx.x;
+  const int b = bq / a.Q;
+  const int K = a.K;
+  for (int i = tid; i < 4096 / 4; i += kGsThreads) reinterpret_cast<uint4*>(sub)[i] = make_uint4(0u, 0u, 0u, 0u);
+  chain_wait();
+  int32_t* out = a.out_idx + (int64_t)bq * K;
+  float* out_s = a.out_score ? a.out_score + (int64_t)bq * K : nullptr;
+  const int64_t base = a.seq_base[b];
+  int64_t n = a.n_vis[bq];
+  if (n < 0 || n > a.max_n_vis || base < 0 || base + n > a.pool_entries) n = 0;
+  const uint32_t* keys = a.keys + (int64_t)bq * a.key_stride;
+  const uint32_t* gm = a.gmax + (int64_t)bq * a.gstride;
+  const int ng = (int)((n + 31) >> 5);
+
+  // the listed keys (nc, index order, sharing `mask` bits with `prefix`, bit p the highest
+  // undecided) resolved into the slots from `base0`: radix levels, then the taken keys and the
+  // first `need` tied keys in index order
+  auto finish_list = [&](int nc, uint32_t base0, uint32_t need, uint32_t prefix, uint32_t mask, int p) {
+    for (int i = tid; i < kBins; i += kGsThreads) {
+      hist[i] = 0u;
+      hsum[i] = 0u;
+    }
+    __syncthreads();
+    int cur = 0;
+    while (p >= 0) {
+      const int sh = p >= kDigitBits - 1 ? p - (kDigitBits - 1) : 0;
+      const uint32_t nb = 1u << (p - sh + 1);
+      uint32_t* h = cur ? hsum : hist;
+      uint32_t* hn = cur ? hist : hsum;
+      for (int i = tid; i < nc; i += kGsThreads) {
+        const uint32_t key = candk[i];
+        if ((key & mask) == prefix) atomicAdd(&h[(key >> sh) & (nb - 1u)], 1u);
+      }
+      for (int i = tid; i < kBins; i += kGsThreads) hn[i] = 0u;
+      __syncthreads();
+      if (tid < 32) {
+        find_bin_warp(h, (int)nb, need, &misc[0], &misc[1]);
+        __syncwarp();
+        if (tid == 0) misc[2] = h[misc[0]];
+      }
+      __syncthreads();
+      const uint32_t T = misc[0], inbin = misc[2];
+      need -= misc[1];
+      prefix |= T << sh;
+      mask |= (nb - 1u) << sh;
+      if (inbin == need || sh == 0) break;
+      p = sh - 1;
+      cur ^= 1;
+    }
+    const int per = (nc + kGsThreads - 1) / kGsThreads;
+    const int c0 = tid * per, c1 = min(nc, c0 + per);
+    uint32_t g2 = 0u, e2 = 0u;
+    for (int i = c0; i < c1; ++i) {
+      const uint32_t kp = candk[i] & mask;
+      if (kp > prefix) ++g2;
+      else if (kp == prefix) ++e2;
+    }
+    uint64_t t2;
+    const uint64_t m2 = block_excl_scan64<kGsThreads>((uint64_t)g2 | ((uint64_t)e2 << 32), scan_ws, &t2);
+    uint32_t lg = base0 + (uint32_t)m2, le = (uint32_t)(m2 >> 32);
+    const uint32_t tie0 = (uint32_t)K - need;
+    for (int i = c0; i < c1; ++i) {
+      const uint32_t key = candk[i], kp = key & mask;
+      if (kp > prefix) {
+        out[lg] = candi[i];
+        if (out_s) out_s[lg] = key_score(key);
+        ++lg;
+      } else if (kp == prefix) {
+        if (le < need) {
+          out[tie0 + le] = candi[i];
+          if (out_s) out_s[tie0 + le] = key_score(key);
+        }
+        ++le;
+      }
+    }
+  };
+
+  // ---- the threshold x from the group maxima ------------------------------------------------
+  uint32_t gc = 0u;
+  for (int g = tid; g < ng; g += kGsThreads) {
+    const uint32_t m = gm[g];
+    if (m != 0u) {
+      atomicAdd(&sub[m >> 20], 1u);
+      ++gc;
+    }
+  }
+  uint64_t gtot;
+  block_excl_scan64<kGsThreads>((uint64_t)gc, scan_ws, &gtot);
+  uint32_t x = 1u;
+  if (gtot >= (uint64_t)K) {
+    for (int g = tid; g < kBins; g += kGsThreads) {
+      hist[g] = sub[4 * g] + sub[4 * g + 1] + sub[4 * g + 2] + sub[4 * g + 3];
+      hsum[g] = 0u;
+    }
+    __syncthreads();
+    if (tid < 32) {
+      find_bin_warp(hist, kBins, (uint32_t)K, &misc[0], &misc[1]);
+      __syncwarp();
+      if (tid == 0) {
+        uint32_t above = misc[1], need1 = (uint32_t)K - above, t = 4 * misc[0] + 3;
+        for (int jj = 3; jj > 0; --jj, --t) {
+          const uint32_t c = sub[t];
+          if (need1 <= c) break;
+          need1 -= c;
+          above += c;
+        }
+        misc[2] = t;
+        misc[3] = above;
+      }
+    }
+    __syncthreads();
+    const uint32_t T1 = misc[2], above1 = misc[3];
+    for (int g = tid; g < ng; g += kGsThreads) {
+      const uint32_t m = gm[g];
+      if ((m >> 20) == T1) atomicAdd(&hsum[(m >> 10) & (kBins - 1)], 1u);
+    }
+    __syncthreads();
+    if (tid < 32) find_bin_warp(hsum, kBins, (uint32_t)K - above1, &misc[4], &misc[5]);
+    __syncthreads();
+    x = max((T1 << 20) | (misc[4] << 10), 1u);
+  }
+  // ---- the groups at or above x, in index order --------------------------------------------
+  const int per = (ng + kGsThreads - 1) / kGsThreads;
+  const int g0 = tid * per, g1 = min(ng, g0 + per);
+  uint32_t sc = 0u;
+  for (int g = g0; g < g1; ++g) sc += gm[g] >= x ? 1u : 0u;
+  uint64_t stot;
+  uint32_t so = (uint32_t)block_excl_scan64<kGsThreads>((uint64_t)sc, scan_ws, &stot);  // ends in a barrier
+  const int S = (int)stot;
+  if (S <= kGsList) {
+    for (int g = g0; g < g1; ++g)
+      if (gm[g] >= x) gl[so++] = (uint32_t)g;
+    __syncthreads();
+    // a thread takes whole groups: its 32 keys in eight 16-byte loads, all in flight at once
+    // (keys past n read as 0)
+    auto group_keys = [&](int sidx, uint32_t (&kk)[32]) {
+      const int64_t i0 = (int64_t)gl[sidx] * 32;
+      const uint4* src = reinterpret_cast<const uint4*>(keys + i0);
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        const uint4 q = i0 + 4 * v + 3 < n ? src[v] : make_uint4(0u, 0u, 0u, 0u);
+        kk[4 * v] = q.x;
+        kk[4 * v + 1] = q.y;
+        kk[4 * v + 2] = q.z;
+        kk[4 * v + 3] = q.w;
+      }
+      if (i0 + 32 > n)  // the tail group: word loads of its keys below n
+#pragma unroll
+        for (int e = 0; e < 32; ++e) kk[e] = i0 + e < n ? keys[i0 + e] : 0u;
+    };
+    for (int sidx = tid; sidx < S; sidx += kGsThreads) {
+      uint32_t kk[32];
+      group_keys(sidx, kk);
+      uint32_t c = 0u;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) c += kk[e] >= x ? 1u : 0u;
+      goff[sidx] = c;
+    }
+    __syncthreads();
+    const int per2 = (S + kGsThreads - 1) / kGsThreads;
+    const int s0 = tid * per2, s1 = min(S, s0 + per2);
+    uint32_t cc = 0u;
+    for (int si = s0; si < s1; ++si) cc += goff[si];
+    uint64_t ctot;
+    uint32_t co = (uint32_t)block_excl_scan64<kGsThreads>((uint64_t)cc, scan_ws, &ctot);
+    const int nc = (int)ctot;
+    if (nc <= kGsCand) {
+      for (int si = s0; si < s1; ++si) {
+        const uint32_t c = goff[si];
+        goff[si] = co;
+        co += c;
+      }
+      __syncthreads();
+      for (int sidx = tid; sidx < S; sidx += kGsThreads) {
+        uint32_t kk[32];
+        group_keys(sidx, kk);
+        uint32_t pos = goff[sidx];
+        const int32_t gi = (int32_t)gl[sidx] * 32;
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (kk[e] >= x) {
+            candk[pos] = kk[e];
+            candi[pos] = gi + e;
+            ++pos;
+          }
+      }
+      __syncthreads();  // the list is complete; the group list is no longer read
+      if (nc <= K) {  // every valid key (fewer than K groups), in index order, then -1
+        for (int i = tid; i < K; i += kGsThreads) {
+          if (i < nc) {
+            out[i] = candi[i];
+            if (out_s) out_s[i] = key_score(candk[i]);
+          } else {
+            out[i] = -1;
+            if (out_s) out_s[i] = -INFINITY;
+          }
+        }
+        return;
+      }
+      finish_list(nc, 0u, (uint32_t)K, 0u, 0u, 31);
+      return;
+    }
+  }
+  __syncthreads();  // every thread has left the lists
+  // ---- heavy ties: exact select over all n keys from global memory -------------------------
+  // counting passes stride over the keys (coalesced); the output passes give thread t the keys
+  // [t * chunk, (t + 1) * chunk), so block prefixes keep index order
+  const int64_t chunk = (n + kGsThreads - 1) / kGsThreads;
+  const int64_t k0 = (int64_t)tid * chunk, k1 = k0 + chunk < n ? k0 + chunk : n;
+  uint32_t vc = 0u;
+  for (int64_t i = k0; i < k1; ++i) vc += keys[i] != 0u ? 1u : 0u;
+  uint64_t vtot;
+  uint64_t vo = block_excl_scan64<kGsThreads>((uint64_t)vc, scan_ws, &vtot);
+  if (vtot <= (uint64_t)K) {  // every valid key, in index order, then -1
+    for (int64_t i = k0; i < k1; ++i)
+      if (keys[i] != 0u) {
+        out[vo] = (int32_t)i;
+        if (out_s) out_s[vo] = key_score(keys[i]);
+        ++vo;
+      }
+    for (int i = (int)vtot + tid; i < K; i += kGsThreads) {
+      out[i] = -1;
+      if (out_s) out_s[i] = -INFINITY;
+    }
+    return;
+  }
+  uint32_t need = (uint32_t)K, prefix = 0u, mask = 0u;
+  int p = 31;
+  while (p >= 0) {
+    const int sh = p >= kDigitBits - 1 ? p - (kDigitBits - 1) : 0;
+    const uint32_t nb = 1u << (p - sh + 1);
+    for (int i = tid; i < kBins; i += kGsThreads) hist[i] = 0u;
+    __syncthreads();
+    for (int64_t i = tid; i < n; i += kGsThreads) {
+      const uint32_t key = keys[i];
+      if (key != 0u && (key & mask) == prefix) atomicAdd(&hist[(key >> sh) & (nb - 1u)], 1u);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      find_bin_warp(hist, (int)nb, need, &misc[0], &misc[1]);
+      __syncwarp();
+      if (tid == 0) misc[2] = hist[misc[0]];
+    }
+    __syncthreads();
+    const uint32_t T = misc[0], inbin = misc[2];
+    need -= misc[1];
+    prefix |= T << sh;
+    mask |= (nb - 1u) << sh;
+    if (inbin == need || sh == 0) break;
+    p = sh - 1;
+  }
+  uint32_t g2 = 0u, e2 = 0u;
+  for (int64_t i = k0; i < k1; ++i) {
+    const uint32_t key = keys[i];
+    if (key == 0u) continue;
+    const uint32_t kp = key & mask;
+    if (kp > prefix) ++g2;
+    else if (kp == prefix) ++e2;
+  }
+  uint64_t t2;
+  const uint64_t m2 = block_excl_scan64<kGsThreads>((uint64_t)g2 | ((uint64_t)e2 << 32), scan_ws, &t2);
+  uint32_t lg = (uint32_t)m2, le = (uint32_t)(m2 >> 32);
+  const uint32_t tie0 = (uint32_t)K - need;
+  for (int64_t i = k0; i < k1; ++i) {
+    const uint32_t key = keys[i];
+    if (key == 0u) continue;
+    const uint32_t kp = key & mask;
+    if (kp > prefix) {
+      out[lg] = (int32_t)i;
+      if (out_s) out_s[lg] = key_score(key);
+      ++lg;
+    } else if (kp == prefix) {
+      if (le < need) {
+        out[tie0 + le] = (int32_t)i;
+        if (out_s) out_s[tie0 + le] = key_score(key);
+      }
+      ++le;
+    }
+  }
 }
 
 // Selection of lists held in registers: a query's keys are split over a cluster of C CTAs
@@ -1916,14 +2226,26 @@ static cudaError_t launch_stream(ScanArgs a, int64_t items, int B, cudaStream_t 
 // Selection of the K best of `items` keys per query row (blockIdx.y = row).
 static cudaError_t launch_select(SelectArgs s, int64_t items, int BQ, cudaStream_t stream) {
   cudaError_t e;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // flat lists with the scan's group maxima, at least one query per SM: one 256-thread CTA per
+  // query, four to an SM (verify: 0.974 -> 0.956 ms per step, prefill 1.780 -> 1.755 against
+  // select_kernel's one-CTA path; with fewer queries select_kernel's 1024 threads per query
+  // finish sooner: full128k's 32 queries took 0.178 ms per step here against 0.172)
+  if (s.gmax != nullptr && items > SelShape<2>::kChunk && BQ >= sms) {
+    s.csize = 1;
+    e = cudaFuncSetAttribute(group_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGsSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = launch_chained(group_select_kernel, dim3((unsigned)BQ), dim3(kGsThreads), (size_t)kGsSmemBytes, stream, 0u, s);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   // Lists whose keys fit the registers of a cluster of at most 8 CTAs, when the clusters of all
   // queries fit two waves: the fewest keys per thread (the most CTAs) that do.  A cluster of
   // 16-key CTAs (lists above 16,384 keys) measured slower than select_kernel (19.4 against
   // 16.5 us for 131,072 keys: each level's cluster barrier and histogram sum cost about a
   // microsecond), so those lists stay with select_kernel.
   {
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     for (int kpt = 4; kpt <= 16; kpt *= 2) {
       const int64_t c = (items + 1024 * kpt - 1) / (1024 * kpt);
       if (c > kMaxCluster || (c > 1 && (int64_t)BQ * c > 2 * (int64_t)sms) || (kpt == 16 && c > 1)) continue;
@@ -1953,8 +2275,6 @@ static cudaError_t launch_select(SelectArgs s, int64_t items, int BQ, cudaStream
     // one wave (one CTA per SM), fewer CTAs per query, each walking several chunks: a second
     // wave costs more than the longer walk (full128k, 32 queries of 131,072 keys: 4 CTAs per
     // query measured 7% faster on the whole step than 8)
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int64_t c = (items + SelShape<4>::kChunk - 1) / SelShape<4>::kChunk;
     c = c < 1 ? 1 : (c > kMaxCluster ? kMaxCluster : c);
     // with the scan's group maxima one CTA reads little more than the groups above the
