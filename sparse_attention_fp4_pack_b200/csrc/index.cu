@@ -490,7 +490,7 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
     }
     const float inv = stacked ? build_b_head(Bs, Bs, a.N, gh, HIPAD + gh, v)
                               : build_b_head(Bs, Bs + 2 * a.N * 128, a.N, gh, gh, v);
-    if (lane == 0) wq[gh] = wv * inv;
+    if (lane == 0) wq[gh] = 0.5f * wv * inv;  // halved: the epilogue weighs z + |z| = 2 max(z, 0)
   }
   if (stacked)  // rows [2 HIPAD, N) of both K-halves are zero
     for (int i = tid; i < 2 * (a.N - 2 * HIPAD) * 32; i += kStreamThreads) {
@@ -602,6 +602,9 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
 #pragma unroll
       for (int g = 0; g < kGmax; ++g) {
         if (g >= G) break;
+        // w * max(z, 0) as (w / 2) * (z + |z|): z + |z| is 2z or 0 exactly and w / 2 exact, so
+        // the products are the same, on the FMA pipe instead of a max on the ALU pipe (the
+        // weights in shared memory are already halved)
         float tot = 0.f;
         if (stacked) {  // one query: head h's hi sum in column h, its lo sum in column HIPAD + h
 #pragma unroll
@@ -612,20 +615,22 @@ __global__ void __launch_bounds__(kStreamThreads, 4) stream_scan_kernel(ScanArgs
             const float z1 = __uint_as_float(r[c + 1]) + __uint_as_float(r[HIPAD + c + 1]);
             const float z2 = __uint_as_float(r[c + 2]) + __uint_as_float(r[HIPAD + c + 2]);
             const float z3 = __uint_as_float(r[c + 3]) + __uint_as_float(r[HIPAD + c + 3]);
-            tot = fmaf(__uint_as_float(w4.x), fmaxf(z0, 0.f), tot);
-            tot = fmaf(__uint_as_float(w4.y), fmaxf(z1, 0.f), tot);
-            tot = fmaf(__uint_as_float(w4.z), fmaxf(z2, 0.f), tot);
-            tot = fmaf(__uint_as_float(w4.w), fmaxf(z3, 0.f), tot);
+            tot = fmaf(__uint_as_float(w4.x), z0 + fabsf(z0), tot);
+            tot = fmaf(__uint_as_float(w4.y), z1 + fabsf(z1), tot);
+            tot = fmaf(__uint_as_float(w4.z), z2 + fabsf(z2), tot);
+            tot = fmaf(__uint_as_float(w4.w), z3 + fabsf(z3), tot);
           }
         } else {
 #pragma unroll
           for (int h4 = 0; h4 < HIPAD / 4; ++h4) {
             const uint4 w4 = tc::ld_shared_v4(wq_a + (uint32_t)(g * HIPAD + h4 * 4) * 4u);
             const int c = g * HIPAD + h4 * 4;
-            tot = fmaf(__uint_as_float(w4.x), fmaxf(__uint_as_float(r[c + 0]), 0.f), tot);
-            tot = fmaf(__uint_as_float(w4.y), fmaxf(__uint_as_float(r[c + 1]), 0.f), tot);
-            tot = fmaf(__uint_as_float(w4.z), fmaxf(__uint_as_float(r[c + 2]), 0.f), tot);
-            tot = fmaf(__uint_as_float(w4.w), fmaxf(__uint_as_float(r[c + 3]), 0.f), tot);
+            const float z0 = __uint_as_float(r[c + 0]), z1 = __uint_as_float(r[c + 1]);
+            const float z2 = __uint_as_float(r[c + 2]), z3 = __uint_as_float(r[c + 3]);
+            tot = fmaf(__uint_as_float(w4.x), z0 + fabsf(z0), tot);
+            tot = fmaf(__uint_as_float(w4.y), z1 + fabsf(z1), tot);
+            tot = fmaf(__uint_as_float(w4.z), z2 + fabsf(z2), tot);
+            tot = fmaf(__uint_as_float(w4.w), z3 + fabsf(z3), tot);
           }
         }
         const int64_t nqg = (int64_t)tc::ld_shared_u64(nq_a + 8u * (uint32_t)g);
