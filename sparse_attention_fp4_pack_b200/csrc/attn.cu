@@ -408,6 +408,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
   const uint32_t rb = 2u * (uint32_t)NQ, pcode = tc::swizzle_code(rb);
   const uint32_t ks_a = tc::smem_u32(Ks), qs_a = tc::smem_u32(Qs), ps_a = tc::smem_u32(Ps);
   uint32_t last_bar = 0, last_par = 0;  // thread 0: the last commit
+  // descriptors of the operands' first bytes; each MMA advances them by a constant
+  const uint64_t kd0 = tc::smem_desc_sw128(ks_a, 16, 1024), qd0 = tc::smem_desc_sw128(qs_a, 16, 1024);
+  const uint64_t kmn0 = tc::smem_desc_sw128(ks_a, 16384, 1024);
+  const uint64_t pd0 = tc::smem_desc(ps_a, 64u * rb, 8u * rb, pcode);
   // S^T = Kt . Qs^T over dims 256 hb .. 256 hb + 255: dim-block db adds to partial sum db mod 4
   auto issue_qk = [&](int hb) {
 #pragma unroll
@@ -415,9 +419,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int db = hb * 4 + i;
-        const uint64_t ad = tc::smem_desc_sw128(ks_a + db * 16384 + kk * 32, 16, 1024);
-        const uint64_t bd = tc::smem_desc_sw128(qs_a + db * 8192 + kk * 32, 16, 1024);
-        tc::mma_f16(tmem + kColS + 64 * i, ad, bd, idesc_s, (hb > 0 || kk > 0) ? 1u : 0u);
+        tc::mma_f16(tmem + kColS + 64 * i, tc::desc_add(kd0, db * 16384 + kk * 32), tc::desc_add(qd0, db * 8192 + kk * 32),
+                    idesc_s, (hb > 0 || kk > 0) ? 1u : 0u);
       }
   };
   // O^T += Kt^T . P^T: B = P^T [128 keys x NQ heads], MN-major, rows of rb = 2 NQ bytes
@@ -427,11 +430,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(AttnArgs a) {
 #pragma unroll
     for (int ks = 0; ks < kTile / 16; ++ks)
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt) {
-        const uint64_t ad = tc::smem_desc_sw128(ks_a + (2 * mt) * 16384 + ks * 2048, 16384, 1024);
-        const uint64_t bd = tc::smem_desc(ps_a + ks * 16 * rb, 64u * rb, 8u * rb, pcode);
-        tc::mma_f16(tmem + kColO + 64 * mt, ad, bd, idesc_o, (ks > 0 || k > 0) ? 1u : 0u);
-      }
+      for (int mt = 0; mt < 4; ++mt)
+        tc::mma_f16(tmem + kColO + 64 * mt, tc::desc_add(kmn0, (2 * mt) * 16384 + ks * 2048),
+                    tc::desc_add(pd0, ks * 16 * rb), idesc_o, (ks > 0 || k > 0) ? 1u : 0u);
   };
 
   {

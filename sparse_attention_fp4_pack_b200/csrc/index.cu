@@ -145,13 +145,14 @@ __device__ __forceinline__ float build_b_head(uint8_t* Bs, uint8_t* Blo, int npa
 __device__ __forceinline__ void issue_tile_mma(uint32_t d, uint32_t a_tmem, uint32_t b_addr, int npad, int parts,
                                                uint32_t idesc) {
   const uint32_t bh = (uint32_t)npad * 128u;  // one K-half of one B operand
+  const uint64_t b0 = tc::smem_desc_sw128(b_addr, 16, 1024);
   for (int p = 0; p < parts; ++p)
 #pragma unroll
     for (int kh = 0; kh < 2; ++kh)
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)  // 16 elements per MMA: 8 columns of A, 32 B of a B row
         tc::mma_f16_ts(d, a_tmem + (uint32_t)(kh * 32 + ks * 8),
-                       tc::smem_desc_sw128(b_addr + (uint32_t)(2 * p + kh) * bh + (uint32_t)ks * 32u, 16, 1024), idesc,
+                       tc::desc_add(b0, (uint32_t)(2 * p + kh) * bh + (uint32_t)ks * 32u), idesc,
                        (p | kh | ks) ? 1u : 0u);
 }
 

@@ -82,6 +82,11 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return smem_desc(saddr, lbo_bytes, sbo_bytes, 2u);
 }
 
+// The descriptor d with its start address advanced by `bytes` (a multiple of 16).  Shared
+// addresses stay below 256 KB, so the 14-bit start field ((address >> 4)) never carries into
+// the fields above it: one 64-bit add instead of rebuilding the descriptor per MMA.
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); }
+
 // kind::f16 with f16 A/B and f32 accumulation.
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn) {
   return (1u << 4) | (0u << 7) | (0u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
