@@ -1843,6 +1843,7 @@ __global__ void __launch_bounds__(1024, 1) select_cl_kernel(SelectArgs a) {
   __shared__ uint32_t wsum[2][32];      // per-warp totals of taken / tied keys
   __shared__ uint32_t xch[8];           // exported to the cluster: [4] taken and [5] tied keys
   __shared__ uint32_t lvl[4];           // bin found, keys above it, keys in it
+  __shared__ uint32_t wtop[32];         // per-warp counts of a level's bins (bin search)
   __shared__ int32_t blk[CSA2_MAX_K];   // Reindex block ids of the query
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int C = a.csize;
@@ -1982,28 +1983,37 @@ __global__ void __launch_bounds__(1024, 1) select_cl_kernel(SelectArgs a) {
       }
       hist[cur ^ 1][tid] = 0u;  // the next level's counters
       __syncthreads();
-      if (warp == 0) {
-        bool few = false;
-        if (C > 1 && level == 0) {  // the cluster's count of valid keys: every one sits in a bin
-          uint32_t t = 0u;
-#pragma unroll 8
-          for (int i = 0; i < kBins / 32; ++i) t += hs[lane + 32 * i];
+      // The bin holding the need-th largest key, by every thread at once: thread t holds bin
+      // t's count, a suffix scan (from the top bin down) over the block gives the keys above
+      // each bin, and the one thread whose bin reaches `need` reports it.
+      const uint32_t cb = tid < (int)nb ? hs[tid] : 0u;
+      uint32_t sfx = cb;  // this warp's bins from this one up
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-          few = t <= need;
-          if (lane == 0) lvl[3] = few ? 1u : 0u;
-        }
-        if (!few) {
-          find_bin_warp(hs, (int)nb, need, &lvl[0], &lvl[1]);
-          __syncwarp();
-          if (lane == 0) lvl[2] = hs[lvl[0]];
-        }
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, sfx, o);
+        if (lane + o < 32) sfx += y;
       }
+      if (lane == 0) wtop[warp] = sfx;
       __syncthreads();
-      if (C > 1 && level == 0 && lvl[3] != 0u) {  // at most K valid keys: every one is taken
+      uint32_t wt = wtop[lane], wsfx = wt;  // the warps' totals, suffix-summed over warps
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, wsfx, o);
+        if (lane + o < 32) wsfx += y;
+      }
+      const uint32_t total = __shfl_sync(0xffffffffu, wsfx, 0);
+      const uint32_t above_warp = __shfl_sync(0xffffffffu, wsfx - wt, warp);  // warps above this one
+      const uint32_t incl = sfx + above_warp, excl = incl - cb;
+      if (C > 1 && level == 0 && total <= need) {  // at most K valid keys: every one is taken
         all_valid = true;
         break;
       }
+      if (cb != 0u && excl < need && incl >= need) {
+        lvl[0] = (uint32_t)tid;
+        lvl[1] = excl;
+        lvl[2] = cb;
+      }
+      __syncthreads();
       const uint32_t T = lvl[0], inbin = lvl[2];
       need -= lvl[1];
       prefix |= T << sh;
