@@ -1050,7 +1050,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
   // The flat scan also leaves the largest key of every 32 (gm).  At least K groups have a
   // maximum at or above x, the K-th largest maximum cut to its top 22 bits, so at least K keys
   // are >= x and the K best are among them.  Only the groups whose maximum reaches x are read
-  // (a warp per group): their keys >= x go, with their item indices and in index order, to the
+  // (a thread per group): their keys >= x go, with their item indices and in index order, to the
   // shared-memory list that the remaining radix levels resolve.  With fewer than K valid
   // groups x = 1, every valid key.  When the groups above x (kGroupList) or their keys
   // (kCand) do not fit, the counters are cleared and the two-pass path below runs instead.
