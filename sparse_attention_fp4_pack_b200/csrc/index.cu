@@ -2257,14 +2257,17 @@ static cudaError_t launch_select(SelectArgs s, int64_t items, int BQ, cudaStream
     return cudaGetLastError();
   }
   // Lists whose keys fit the registers of a cluster of at most 8 CTAs, when the clusters of all
-  // queries fit two waves: the fewest keys per thread (the most CTAs) that do.  A cluster of
-  // 16-key CTAs (lists above 16,384 keys) measured slower than select_kernel (19.4 against
-  // 16.5 us for 131,072 keys: each level's cluster barrier and histogram sum cost about a
-  // microsecond), so those lists stay with select_kernel.
+  // queries fit two waves: the fewest keys per thread (the most CTAs) that do.  Flat lists with
+  // the scan's group maxima and more than 16,384 keys stay with select_kernel's one-CTA group
+  // path (full128k: 0.179 ms per step there against 0.205 in 16-key register clusters); the
+  // hierarchical block select (131,072 block keys) takes a cluster of 8 16-key CTAs (hier1m
+  // 0.521 -> 0.516 ms per step against select_kernel's cluster of 8).
   {
     for (int kpt = 4; kpt <= 16; kpt *= 2) {
       const int64_t c = (items + 1024 * kpt - 1) / (1024 * kpt);
-      if (c > kMaxCluster || (c > 1 && (int64_t)BQ * c > 2 * (int64_t)sms) || (kpt == 16 && c > 1)) continue;
+      if (c > kMaxCluster || (c > 1 && (int64_t)BQ * c > 2 * (int64_t)sms) ||
+          (kpt == 16 && c > 1 && s.gmax != nullptr))
+        continue;
       s.csize = (int)(c < 1 ? 1 : c);
       const dim3 grid((unsigned)s.csize, (unsigned)BQ);
       const unsigned cl = s.csize > 1 ? (unsigned)s.csize : 0u;
