@@ -92,6 +92,22 @@ def test_index_rejects_bad_args(L):
                              None, st) == 0                          # no queries: no-op
 
 
+def test_full_workspace_holds_keys_and_group_maxima(L):
+    """The Full scan's workspace holds the keys (a row of max_n_vis rounded up to 4 words per
+    query) and the largest key of every 32 (a row of ceil(max_n_vis / 32) rounded up to 4),
+    each part 256-byte aligned; one byte less than the size is refused before any launch."""
+    row = lambda n: (n + 3) // 4 * 4
+    r256 = lambda x: (x + 255) // 256 * 256
+    for B, Q, n in ((1, 1, 100), (32, 1, 131072), (8, 64, 131072), (1, 1024, 131072), (3, 5, 1 << 20)):
+        want = r256(B * Q * row(n) * 4) + r256(B * Q * row((n + 31) // 32) * 4)
+        assert L.csa2_index_full_workspace_size(B, Q, 8, 512, n) == want
+    st = ctypes.c_void_p(0)
+    need = L.csa2_index_full_workspace_size(1, 1, 8, 512, 100)
+    args = lambda wsb: (FAKE, FAKE, FAKE, 100, FAKE, FAKE, 1, 1, 8, 512, 100, FAKE, None, FAKE, wsb, None, st)
+    assert L.csa2_index_full(*args(need - 1)) == 1                 # keys only, or one byte short
+    assert L.csa2_index_full(*args(r256(row(100) * 4))) == 1
+
+
 def test_attn_rejects_bad_args(L):
     st = ctypes.c_void_p(0)
     base = lambda H, K, win, sm, swa, S_w: (FAKE, FAKE, 100, FAKE, FAKE, K, swa, S_w, FAKE, FAKE, win, 1, 1, H,
