@@ -885,6 +885,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(SelectArgs a) {
   const int K = a.K;
   for (int i = tid; i < kSubWords / 4; i += kSelThreads)  // counters start at zero
     reinterpret_cast<uint4*>(sub)[i] = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();  // every counter is cleared before any thread counts into it
   chain_wait();
   int32_t* out = a.out_idx + (int64_t)bq * K;
   float* out_s = a.out_score ? a.out_score + (int64_t)bq * K : nullptr;
@@ -1547,6 +1548,7 @@ __global__ void __launch_bounds__(kGsThreads) group_select_kernel(SelectArgs a) 
   const int b = bq / a.Q;
   const int K = a.K;
   for (int i = tid; i < 4096 / 4; i += kGsThreads) reinterpret_cast<uint4*>(sub)[i] = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();  // every counter is cleared before any thread counts into it
   chain_wait();
   int32_t* out = a.out_idx + (int64_t)bq * K;
   float* out_s = a.out_score ? a.out_score + (int64_t)bq * K : nullptr;
@@ -1852,6 +1854,7 @@ __global__ void __launch_bounds__(1024, 1) select_cl_kernel(SelectArgs a) {
   const int b = bq / a.Q;
   const int K = a.K;
   hist[0][tid] = 0u;
+  __syncthreads();  // every counter is cleared before any thread counts into it
   chain_wait();
   auto cluster_sync = [&]() {
     if (C > 1) {
